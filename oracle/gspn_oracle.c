@@ -1,0 +1,263 @@
+/*
+ * gspn_oracle.c -- float64, single-threaded CPU reference of the GSPN 4-direction
+ * line-scan propagation (forward and backward).
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the oracle that the CUDA library is checked
+ * against. Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline / reference
+ * legs may load it. It shares no code, header or table with the CUDA library.
+ *
+ * What it computes (citations are page title + section):
+ *  - "GSPN-2: Efficient Parallel Sequence Modeling" (paper notes), section
+ *    "2D spatial propagation review": the map is propagated line by line; the
+ *    per-line propagation matrix w_{i,c} is W x W, tridiagonal and row-stochastic
+ *    (rows sum to 1), lambda_{i,:,c} is a per-channel scaling of the input, and the
+ *    scan is run in four directions (top->bottom, bottom->top, left->right,
+ *    right->left).
+ *  - "Parallel Sequence Modeling via Generalized Spatial Propagation Network"
+ *    (summary), section "Approach": the weights are made row-stochastic by a sigmoid
+ *    followed by a row normalisation over the three neighbours j-1, j, j+1.
+ *  - "GSPN-2 ..." (paper notes), section "Optimisation 2: compact channel
+ *    propagation": in the channel-shared mode one matrix w_i is used by every channel
+ *    and only lambda stays per channel.
+ *  The display equation that followed "GSPN propagates row by row" was lost in the
+ *  page extraction. The rule implemented here is the plainest reading consistent with
+ *  the surviving text:
+ *      h_{-1} = 0,   h_i = w_i h_{i-1} + lambda_i (.) x_i,
+ *      y = u (.) sum_{d in mask} h^d          (h^d mapped back to image coordinates).
+ *  Edge rows of w have two in-range neighbours; the normalisation runs over the
+ *  in-range neighbours only, so every row sums to exactly one.
+ *
+ * Conventions (shared with the CUDA library by specification, not by code):
+ *  - x, lam, u, y, dy, dx, dlam, du: N x C x H x W, contiguous.
+ *  - a, da: D x N x Cw x 3 x H x W, D = popcount(mask), slots in the order TB, BT, LR,
+ *    RL keeping the directions set in mask; Cw = C (per-channel) or 1 (shared).
+ *  - Scan coordinates: step i along the scan axis, lane j across it.
+ *      TB: r = i,       c = j      (L = H, M = W)
+ *      BT: r = H-1-i,   c = j      (L = H, M = W)
+ *      LR: r = j,       c = i      (L = W, M = H)
+ *      RL: r = j,       c = W-1-i  (L = W, M = H)
+ *  - Neighbour k in {0,1,2} is lane j+k-1, i.e. ordered by increasing image coordinate
+ *    on the axis across the scan. The 3 logits of hidden pixel (r,c) are stored at
+ *    image position (r,c).
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define DIR_TB 1u
+#define DIR_BT 2u
+#define DIR_LR 4u
+#define DIR_RL 8u
+
+/* scan length L and lane count M of direction d */
+static void geom(unsigned d, int H, int W, int *L, int *M) {
+    if (d == DIR_TB || d == DIR_BT) { *L = H; *M = W; }
+    else                            { *L = W; *M = H; }
+}
+
+/* image offset r*W + c of scan position (i, j) in direction d */
+static long pix(unsigned d, int H, int W, int i, int j) {
+    int r, c;
+    switch (d) {
+    case DIR_TB: r = i;         c = j;         break;
+    case DIR_BT: r = H - 1 - i; c = j;         break;
+    case DIR_LR: r = j;         c = i;         break;
+    default:     r = j;         c = W - 1 - i; break; /* RL */
+    }
+    return (long)r * W + c;
+}
+
+static double sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* Weights of hidden lane j (of M) from its three logits a_k: sigmoid, then division by
+ * the sum over in-range neighbours. Out-of-range neighbours get weight 0. Also returns
+ * s_k and the normaliser S for the backward. */
+static void row_weights(const double av[3], int j, int M, double w[3], double s[3], double *S) {
+    double sum = 0.0;
+    for (int k = 0; k < 3; ++k) {
+        int jj = j + k - 1;
+        if (jj >= 0 && jj < M) { s[k] = sigmoid(av[k]); sum += s[k]; }
+        else                   { s[k] = 0.0; }
+    }
+    for (int k = 0; k < 3; ++k) w[k] = s[k] / sum;
+    *S = sum;
+}
+
+static int popcount4(unsigned m) { int n = 0; for (int b = 0; b < 4; ++b) n += (m >> b) & 1u; return n; }
+
+static int check_args(int N, int C, int H, int W, int wmode, unsigned mask) {
+    if (N < 1 || C < 1 || H < 1 || W < 1) return 1;
+    if (wmode != 0 && wmode != 1) return 1;
+    if (mask < 1u || mask > 15u) return 1;
+    return 0;
+}
+
+/* Forward scan of one (n, c, d): fills hbuf[i*M + j] (scan coordinates). */
+static void scan_forward(unsigned d, int H, int W, const double *x, const double *lam,
+                         const double *a3 /* 3 planes of H*W */, double *hbuf) {
+    int L, M;
+    geom(d, H, W, &L, &M);
+    const long HW = (long)H * W;
+    for (int i = 0; i < L; ++i) {
+        for (int j = 0; j < M; ++j) {
+            long p = pix(d, H, W, i, j);
+            double z = lam[p] * x[p];
+            double acc = z;
+            if (i > 0) {
+                double av[3] = {a3[p], a3[HW + p], a3[2 * HW + p]}, w[3], s[3], S;
+                row_weights(av, j, M, w, s, &S);
+                for (int k = 0; k < 3; ++k) {
+                    int jj = j + k - 1;
+                    if (jj >= 0 && jj < M) acc += w[k] * hbuf[(long)(i - 1) * M + jj];
+                }
+            }
+            hbuf[(long)i * M + j] = acc;
+        }
+    }
+}
+
+static long logit_base(int slot, int n, int cw, int N, int Cw, long HW) {
+    return (((long)slot * N + n) * Cw + cw) * 3 * HW;
+}
+
+int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
+                     const double *x, const double *a, const double *lam, const double *u,
+                     double *y) {
+    if (check_args(N, C, H, W, wmode, mask)) return 1;
+    const long HW = (long)H * W;
+    const int Cw = wmode ? 1 : C;
+    const int Lmax = H > W ? H : W;
+    double *hbuf = (double *)malloc(sizeof(double) * (size_t)Lmax * (size_t)Lmax);
+    double *acc = (double *)malloc(sizeof(double) * (size_t)HW);
+    if (!hbuf || !acc) { free(hbuf); free(acc); return 2; }
+    for (int n = 0; n < N; ++n) {
+        for (int c = 0; c < C; ++c) {
+            const long off = ((long)n * C + c) * HW;
+            memset(acc, 0, sizeof(double) * (size_t)HW);
+            int slot = 0;
+            for (unsigned d = DIR_TB; d <= DIR_RL; d <<= 1) {
+                if (!(mask & d)) continue;
+                const double *a3 = a + logit_base(slot, n, wmode ? 0 : c, N, Cw, HW);
+                scan_forward(d, H, W, x + off, lam + off, a3, hbuf);
+                int L, M;
+                geom(d, H, W, &L, &M);
+                for (int i = 0; i < L; ++i)
+                    for (int j = 0; j < M; ++j) acc[pix(d, H, W, i, j)] += hbuf[(long)i * M + j];
+                ++slot;
+            }
+            for (long p = 0; p < HW; ++p) y[off + p] = u[off + p] * acc[p];
+        }
+    }
+    free(hbuf);
+    free(acc);
+    return 0;
+}
+
+/*
+ * Backward (the adjoint of the forward above, written from the chain rule):
+ *   acc = sum_d h^d,  du = dy (.) acc,  g = dy (.) u.
+ *   Per direction, in scan coordinates: delta_{L-1} = g_{L-1},
+ *     delta_i = g_i + w_{i+1}^T delta_{i+1},
+ *     (w^T delta)[j] = w[j-1][2] delta[j-1] + w[j][1] delta[j] + w[j+1][0] delta[j+1]
+ *     (in-range terms only).
+ *   dz = sum_d delta^d (image coordinates), dx = lam (.) dz, dlam = x (.) dz.
+ *   dw_i[j][k] = delta_i[j] h_{i-1}[j+k-1]  (0 on step 0, where h_{-1} = 0).
+ *   w_k = s_k / S with s_k = sigmoid(a_k):
+ *     da_k = s_k (1 - s_k) (dw_k - sum_{k' in range} w_k' dw_k') / S  for in-range k,
+ *     da_k = 0 for out-of-range k. In the shared mode da is summed over channels.
+ */
+int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
+                      const double *x, const double *a, const double *lam, const double *u,
+                      const double *dy, double *dx, double *da, double *dlam, double *du) {
+    if (check_args(N, C, H, W, wmode, mask)) return 1;
+    const long HW = (long)H * W;
+    const int Cw = wmode ? 1 : C;
+    const int D = popcount4(mask);
+    const int Lmax = H > W ? H : W;
+    double *hbuf = (double *)malloc(sizeof(double) * (size_t)Lmax * (size_t)Lmax);
+    double *acc = (double *)malloc(sizeof(double) * (size_t)HW);
+    double *dz = (double *)malloc(sizeof(double) * (size_t)HW);
+    double *dcur = (double *)malloc(sizeof(double) * (size_t)Lmax);
+    double *dnext = (double *)malloc(sizeof(double) * (size_t)Lmax);
+    double *wnext = (double *)malloc(sizeof(double) * 3 * (size_t)Lmax);
+    if (!hbuf || !acc || !dz || !dcur || !dnext || !wnext) {
+        free(hbuf); free(acc); free(dz); free(dcur); free(dnext); free(wnext);
+        return 2;
+    }
+    memset(da, 0, sizeof(double) * (size_t)D * N * Cw * 3 * HW);
+    for (int n = 0; n < N; ++n) {
+        for (int c = 0; c < C; ++c) {
+            const long off = ((long)n * C + c) * HW;
+            const double *xp = x + off, *lp = lam + off, *up = u + off, *dyp = dy + off;
+            /* acc = sum_d h^d, needed for du */
+            memset(acc, 0, sizeof(double) * (size_t)HW);
+            memset(dz, 0, sizeof(double) * (size_t)HW);
+            int slot = 0;
+            for (unsigned d = DIR_TB; d <= DIR_RL; d <<= 1) {
+                if (!(mask & d)) continue;
+                const long ab = logit_base(slot, n, wmode ? 0 : c, N, Cw, HW);
+                const double *a3 = a + ab;
+                double *da3 = da + ab;
+                int L, M;
+                geom(d, H, W, &L, &M);
+                scan_forward(d, H, W, xp, lp, a3, hbuf);
+                for (int i = 0; i < L; ++i)
+                    for (int j = 0; j < M; ++j) acc[pix(d, H, W, i, j)] += hbuf[(long)i * M + j];
+                /* reverse scan */
+                for (int i = L - 1; i >= 0; --i) {
+                    for (int j = 0; j < M; ++j) {
+                        long p = pix(d, H, W, i, j);
+                        double del = dyp[p] * up[p];
+                        if (i < L - 1) {
+                            /* w_{i+1}^T delta_{i+1}: row j' of w_{i+1} touches lane j through k = j - j' + 1 */
+                            for (int jp = j - 1; jp <= j + 1; ++jp) {
+                                if (jp < 0 || jp >= M) continue;
+                                int k = j - jp + 1;
+                                del += wnext[3 * (long)jp + k] * dnext[jp];
+                            }
+                        }
+                        dcur[j] = del;
+                        dz[p] += del;
+                    }
+                    /* weights of step i (used by step i-1's transpose product) and da_i */
+                    for (int j = 0; j < M; ++j) {
+                        long p = pix(d, H, W, i, j);
+                        double av[3] = {a3[p], a3[HW + p], a3[2 * HW + p]}, w[3], s[3], S;
+                        row_weights(av, j, M, w, s, &S);
+                        if (i > 0) {
+                            double dw[3] = {0.0, 0.0, 0.0}, wdw = 0.0;
+                            for (int k = 0; k < 3; ++k) {
+                                int jj = j + k - 1;
+                                if (jj >= 0 && jj < M) {
+                                    dw[k] = dcur[j] * hbuf[(long)(i - 1) * M + jj];
+                                    wdw += w[k] * dw[k];
+                                }
+                            }
+                            for (int k = 0; k < 3; ++k) {
+                                int jj = j + k - 1;
+                                if (jj >= 0 && jj < M)
+                                    da3[k * HW + p] += s[k] * (1.0 - s[k]) * (dw[k] - wdw) / S;
+                            }
+                        } else {
+                            /* w_0 multiplies h_{-1} = 0: no effect on the output */
+                            for (int k = 0; k < 3; ++k) w[k] = 0.0;
+                        }
+                        for (int k = 0; k < 3; ++k) wnext[3 * (long)j + k] = w[k];
+                    }
+                    for (int j = 0; j < M; ++j) dnext[j] = dcur[j];
+                }
+                ++slot;
+            }
+            for (long p = 0; p < HW; ++p) {
+                du[off + p] = dyp[p] * acc[p];
+                dx[off + p] = lp[p] * dz[p];
+                dlam[off + p] = xp[p] * dz[p];
+            }
+        }
+    }
+    free(hbuf); free(acc); free(dz); free(dcur); free(dnext); free(wnext);
+    return 0;
+}
+
+/* Version tag so that a loader can check it got this file's build. */
+int gspn_ref_abi_version(void) { return 1; }
