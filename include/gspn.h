@@ -1,0 +1,152 @@
+/*
+ * gspn.h -- C ABI of libgspn, the sm_100a (B200) implementation of the GSPN 4-direction
+ * line-scan propagation.
+ *
+ * The operation ("GSPN-2: Efficient Parallel Sequence Modeling" paper notes, section
+ * "2D spatial propagation review"; "Parallel Sequence Modeling via Generalized Spatial
+ * Propagation Network" summary, section "Approach"):
+ *
+ *   for every plane (n, c) and every direction d in dir_mask, in scan coordinates
+ *   (step i along the scan axis, lane j across it):
+ *       h_{-1} = 0,   h_i[j] = sum_{k in range} w_i[j][k] h_{i-1}[j+k-1] + lam_i[j] x_i[j]
+ *   with w_i[j][k] = sigmoid(a_k) / sum_{k' in range} sigmoid(a_k') over the neighbours
+ *   j-1, j, j+1 that lie inside the line (a tridiagonal, row-stochastic matrix), and
+ *       y = u * sum_{d in dir_mask} h^d      (h^d taken back to image coordinates).
+ *   The display equation of the pages did not survive extraction; this is the reading the
+ *   library implements (stated in full in the repository's design notes).
+ *
+ * Directions and scan coordinates (r = image row, c = image column):
+ *   TB: r = i, c = j     BT: r = H-1-i, c = j     LR: r = j, c = i     RL: r = j, c = W-1-i
+ * Neighbour k = 0, 1, 2 is lane j-1, j, j+1: ordered by increasing image coordinate on the
+ * axis across the scan, for every direction. The three logits of hidden pixel (r, c) are
+ * stored at image position (r, c).
+ *
+ * Weight modes: per-channel w_{i,c} (GSPN-1) or one w_i shared by all channels of a batch
+ * item with per-channel lam (GSPN-2, "GSPN-2 ..." paper notes, section "Optimisation 2:
+ * compact channel propagation").
+ *
+ * Layouts (all contiguous, all in the one storage dtype of the descriptor):
+ *   x, lam, u, y, dy, dx, dlam, du : N x C x H x W
+ *   a, da                          : D x N x Cw x 3 x H x W
+ *     D  = popcount(dir_mask); slots in the fixed order TB, BT, LR, RL keeping only the
+ *          directions in the mask;
+ *     Cw = C (GSPN_W_PER_CHANNEL) or 1 (GSPN_W_SHARED).
+ * Arithmetic is fp32 for both storage dtypes (bf16 values are widened on load and rounded to
+ * nearest-even on store).
+ *
+ * Ownership and conventions:
+ *   - The caller owns every buffer. The library never allocates, never keeps a pointer after
+ *     a call returns, and never synchronises except in gspn_device_status and
+ *     gspn_forward_host.
+ *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy stream).
+ *   - Outputs are overwritten, never accumulated into. In the shared mode da is the sum over
+ *     channels.
+ *   - Device pointers must be 16-byte aligned (else GSPN_ERR_ALIGNMENT), shapes must have
+ *     N, C, H, W >= 1 and 1 <= dir_mask <= 15 (else GSPN_ERR_INVALID_ARG), and the workspace
+ *     must be at least gspn_workspace_size() bytes (else GSPN_ERR_WORKSPACE). All of these
+ *     are checked on the host before anything is launched.
+ *   - A launch failure returns GSPN_ERR_CUDA. Kernels never trap; a bounded device-side wait
+ *     that runs out records GSPN_ERR_DEVICE_TIMEOUT in the workspace status word, which
+ *     gspn_device_status reports.
+ *   - Calls sharing one workspace must not overlap on the GPU.
+ */
+#ifndef GSPN_H
+#define GSPN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GSPN_API __attribute__((visibility("default")))
+#else
+#define GSPN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GSPN_OK = 0,
+    GSPN_ERR_INVALID_ARG = 1,
+    GSPN_ERR_UNSUPPORTED = 2,
+    GSPN_ERR_ALIGNMENT = 3,
+    GSPN_ERR_WORKSPACE = 4,
+    GSPN_ERR_CUDA = 5,
+    GSPN_ERR_DEVICE_TIMEOUT = 6
+} gspn_status;
+
+typedef enum { GSPN_F32 = 0, GSPN_BF16 = 1 } gspn_dtype;
+typedef enum { GSPN_W_PER_CHANNEL = 0, GSPN_W_SHARED = 1 } gspn_wmode;
+enum { GSPN_DIR_TB = 1, GSPN_DIR_BT = 2, GSPN_DIR_LR = 4, GSPN_DIR_RL = 8, GSPN_DIR_ALL = 15 };
+
+/* Kernel family. AUTO picks the fastest one that supports the shape; the others force a
+ * family (GSPN_ERR_UNSUPPORTED if it cannot run the shape) so that every path can be tested
+ * on the same inputs.
+ *   GENERIC: any shape; one CTA per plane and direction, hidden line in shared memory.
+ *   PLANE:   small maps; the whole plane stays on chip and all directions run in one pass.
+ *   SWEEP:   large maps; persistent TMA-fed line sweeps, one direction pair per kernel. */
+enum { GSPN_ALGO_AUTO = 0, GSPN_ALGO_GENERIC = 1, GSPN_ALGO_PLANE = 2, GSPN_ALGO_SWEEP = 3 };
+
+typedef struct {
+    int N, C, H, W;
+    int wmode;          /* gspn_wmode */
+    unsigned dir_mask;  /* GSPN_DIR_* bits */
+    int dtype;          /* gspn_dtype */
+    int algo;           /* GSPN_ALGO_*, 0 = AUTO */
+} gspn_desc;
+
+/* Bytes of device workspace that gspn_forward (for_backward = 0) or gspn_backward
+ * (for_backward = 1) needs for this descriptor; 0 if the descriptor is invalid or its
+ * forced algo cannot run it. The first 256 bytes hold the device status word. */
+GSPN_API size_t gspn_workspace_size(const gspn_desc *desc, int for_backward);
+
+/* Kernel family that AUTO (or the forced algo) uses for this descriptor, or -1. */
+GSPN_API int gspn_selected_algo(const gspn_desc *desc, int for_backward);
+
+/* y = u * sum_d h^d (definition above). x, a, lam, u, y, ws: device pointers. */
+GSPN_API gspn_status gspn_forward(const gspn_desc *desc, const void *x, const void *a, const void *lam,
+                         const void *u, void *y, void *ws, size_t ws_bytes, void *stream);
+
+/* Gradients of the scalar sum(dy * y) with respect to x, a, lam and u (reverse scans):
+ *   g = u * dy; per direction delta_i = g_i + w_{i+1}^T delta_{i+1}; dz = sum_d delta^d;
+ *   dx = lam * dz; dlam = x * dz; du = dy * sum_d h^d;
+ *   da_k = s_k (1 - s_k) (dw_k - sum_k' w_k' dw_k') / S with dw_i[j][k] = delta_i[j] h_{i-1}[j+k-1],
+ *   zero for out-of-range k and on the first step of each scan.
+ * All pointers are device pointers; da has the layout of a. */
+GSPN_API gspn_status gspn_backward(const gspn_desc *desc, const void *x, const void *a, const void *lam,
+                          const void *u, const void *dy, void *dx, void *da, void *dlam, void *du,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/* Bytes of device staging buffer that gspn_forward_host needs (inputs, output and
+ * workspace, each 256-byte aligned). */
+GSPN_API size_t gspn_forward_host_buffer_size(const gspn_desc *desc);
+
+/* End-to-end forward from HOST buffers: copies x, a, lam, u from host memory (pinned memory
+ * gives asynchronous copies) into the caller's device buffer `dev`, runs gspn_forward there,
+ * copies y back to host memory `hy` and synchronises `stream`. Returns the first error. */
+GSPN_API gspn_status gspn_forward_host(const gspn_desc *desc, const void *hx, const void *ha,
+                              const void *hlam, const void *hu, void *hy, void *dev,
+                              size_t dev_bytes, void *stream);
+
+/* Synchronises `stream`, reads and clears the device status word at the start of `ws`.
+ * Returns GSPN_OK, GSPN_ERR_DEVICE_TIMEOUT (a bounded device wait ran out) or GSPN_ERR_CUDA. */
+GSPN_API gspn_status gspn_device_status(void *ws, void *stream);
+
+/* Test hook for the failure path: launches one CTA that waits, through the same bounded
+ * wait the TMA pipelines use, on a flag in `ws` that nothing sets, giving up after
+ * `limit_ns` nanoseconds and recording GSPN_ERR_DEVICE_TIMEOUT in the status word. */
+GSPN_API gspn_status gspn_debug_wait_timeout(void *ws, size_t ws_bytes, unsigned long long limit_ns,
+                                    void *stream);
+
+/* Plain device-to-device copy of `bytes` (multiple of 16, 16-byte aligned pointers) with a
+ * vectorised grid-stride kernel: the bandwidth ceiling the sweeps are compared with. */
+GSPN_API gspn_status gspn_copy_ceiling(const void *src, void *dst, size_t bytes, void *stream);
+
+GSPN_API const char *gspn_status_string(gspn_status s);
+GSPN_API int gspn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSPN_H */

@@ -1,0 +1,239 @@
+"""Python binding of libgspn, the sm_100a implementation of the GSPN 4-direction line scan.
+
+Argument marshalling only: every step of the propagation runs in the CUDA kernels of
+``libgspn.so`` (built in-tree by ``build.py``). PyTorch provides device memory and streams;
+no computation on this path happens in PyTorch or on the CPU. If the library is missing the
+calls raise instead of falling back.
+
+Operation (see ``include/gspn.h`` for the full contract):
+    h_{-1} = 0, h_i = w_i h_{i-1} + lam_i * x_i along each scan direction,
+    y = u * sum_{d in dir_mask} h^d,
+with w_i tridiagonal and row-stochastic, formed from sigmoid logits normalised over the
+in-range neighbours ("Parallel Sequence Modeling via Generalized Spatial Propagation
+Network" summary, section "Approach"; "GSPN-2: Efficient Parallel Sequence Modeling" paper
+notes, sections "2D spatial propagation review" and "Optimisation 2: compact channel
+propagation").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build_mod
+
+LIB_PATH = _build_mod.LIB
+
+GSPN_OK, GSPN_ERR_INVALID_ARG, GSPN_ERR_UNSUPPORTED, GSPN_ERR_ALIGNMENT = 0, 1, 2, 3
+GSPN_ERR_WORKSPACE, GSPN_ERR_CUDA, GSPN_ERR_DEVICE_TIMEOUT = 4, 5, 6
+F32, BF16 = 0, 1
+PER_CHANNEL, SHARED = 0, 1
+DIR_TB, DIR_BT, DIR_LR, DIR_RL, DIR_ALL = 1, 2, 4, 8, 15
+ALGO_AUTO, ALGO_GENERIC, ALGO_PLANE, ALGO_SWEEP = 0, 1, 2, 3
+ALGO_NAMES = {ALGO_GENERIC: "generic", ALGO_PLANE: "plane", ALGO_SWEEP: "sweep"}
+
+
+class GspnDesc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int), ("C", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("wmode", ctypes.c_int), ("dir_mask", ctypes.c_uint), ("dtype", ctypes.c_int),
+                ("algo", ctypes.c_int)]
+
+
+class GspnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+# (name, restype, argtypes) of every symbol include/gspn.h declares.
+_VP, _SZ, _I, _U64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_ulonglong
+_DP = ctypes.POINTER(GspnDesc)
+SIGNATURES = {
+    "gspn_workspace_size": (_SZ, [_DP, _I]),
+    "gspn_selected_algo": (_I, [_DP, _I]),
+    "gspn_forward": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "gspn_backward": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "gspn_forward_host_buffer_size": (_SZ, [_DP]),
+    "gspn_forward_host": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "gspn_device_status": (_I, [_VP, _VP]),
+    "gspn_debug_wait_timeout": (_I, [_VP, _SZ, _U64, _VP]),
+    "gspn_copy_ceiling": (_I, [_VP, _VP, _SZ, _VP]),
+    "gspn_status_string": (ctypes.c_char_p, [_I]),
+    "gspn_version": (_I, []),
+}
+
+
+def build(force: bool = False) -> str:
+    """Compiles libgspn.so in-tree (nvcc, sm_100a)."""
+    return _build_mod.build(force=force)
+
+
+def lib():
+    """The loaded libgspn. Raises if it has not been built: there is no fallback path."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgspn.so is not built ({LIB_PATH}); run "
+                               "`python -m linear_spatial_propagation_gspn_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().gspn_status_string(int(s)).decode()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return F32
+    if t == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t} (float32 or bfloat16)")
+
+
+def make_desc(N, C, H, W, wmode=PER_CHANNEL, dir_mask=DIR_ALL, dtype=F32, algo=ALGO_AUTO) -> GspnDesc:
+    return GspnDesc(int(N), int(C), int(H), int(W), int(wmode), int(dir_mask), int(dtype), int(algo))
+
+
+def desc_for(x: torch.Tensor, wmode: int, dir_mask: int, algo: int = ALGO_AUTO) -> GspnDesc:
+    N, C, H, W = x.shape
+    return make_desc(N, C, H, W, wmode, dir_mask, _dtype_code(x.dtype), algo)
+
+
+def workspace_size(desc: GspnDesc, backward: bool = False) -> int:
+    return int(lib().gspn_workspace_size(ctypes.byref(desc), int(backward)))
+
+
+def selected_algo(desc: GspnDesc, backward: bool = False) -> int:
+    return int(lib().gspn_selected_algo(ctypes.byref(desc), int(backward)))
+
+
+def logits_shape(N, C, H, W, wmode, dir_mask):
+    return (bin(dir_mask & 15).count("1"), N, 1 if wmode == SHARED else C, 3, H, W)
+
+
+def _check(tensors, like: torch.Tensor):
+    for name, t in tensors.items():
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.device.type != "cuda":
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dtype != like.dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}, expected {like.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_ptr(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def alloc_workspace(desc: GspnDesc, backward: bool, device) -> torch.Tensor:
+    n = workspace_size(desc, backward)
+    if n == 0:
+        raise GspnError(GSPN_ERR_UNSUPPORTED, "workspace size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def forward(x, a, lam, u, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, algo: int = ALGO_AUTO,
+            y=None, ws=None, stream=None) -> torch.Tensor:
+    """y = u * sum_d h^d. x, lam, u: (N, C, H, W); a: (D, N, Cw, 3, H, W); all one dtype."""
+    _check({"x": x, "a": a, "lam": lam, "u": u}, x)
+    if tuple(a.shape) != logits_shape(*x.shape, wmode, dir_mask):
+        raise ValueError(f"logits shape {tuple(a.shape)}, expected {logits_shape(*x.shape, wmode, dir_mask)}")
+    if lam.shape != x.shape or u.shape != x.shape:
+        raise ValueError("lam and u must have the shape of x")
+    desc = desc_for(x, wmode, dir_mask, algo)
+    if y is None:
+        y = torch.empty_like(x)
+    _check({"y": y}, x)
+    if ws is None:
+        ws = alloc_workspace(desc, False, x.device)
+    s = lib().gspn_forward(ctypes.byref(desc), x.data_ptr(), a.data_ptr(), lam.data_ptr(), u.data_ptr(),
+                           y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_forward")
+    return y
+
+
+def backward(x, a, lam, u, dy, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, algo: int = ALGO_AUTO,
+             out=None, ws=None, stream=None):
+    """Gradients (dx, da, dlam, du) of sum(dy * y)."""
+    _check({"x": x, "a": a, "lam": lam, "u": u, "dy": dy}, x)
+    if tuple(a.shape) != logits_shape(*x.shape, wmode, dir_mask):
+        raise ValueError("logits shape mismatch")
+    desc = desc_for(x, wmode, dir_mask, algo)
+    if out is None:
+        out = (torch.empty_like(x), torch.empty_like(a), torch.empty_like(x), torch.empty_like(x))
+    dx, da, dlam, du = out
+    _check({"dx": dx, "da": da, "dlam": dlam, "du": du}, x)
+    if ws is None:
+        ws = alloc_workspace(desc, True, x.device)
+    s = lib().gspn_backward(ctypes.byref(desc), x.data_ptr(), a.data_ptr(), lam.data_ptr(), u.data_ptr(),
+                            dy.data_ptr(), dx.data_ptr(), da.data_ptr(), dlam.data_ptr(), du.data_ptr(),
+                            ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_backward")
+    return dx, da, dlam, du
+
+
+def forward_host_buffer_size(desc: GspnDesc) -> int:
+    return int(lib().gspn_forward_host_buffer_size(ctypes.byref(desc)))
+
+
+def forward_host(desc: GspnDesc, hx, ha, hlam, hu, hy, dev: torch.Tensor, stream=None):
+    """End-to-end forward from host tensors (pinned for asynchronous copies) into host ``hy``."""
+    for name, t in {"hx": hx, "ha": ha, "hlam": hlam, "hu": hu, "hy": hy}.items():
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    s = lib().gspn_forward_host(ctypes.byref(desc), hx.data_ptr(), ha.data_ptr(), hlam.data_ptr(), hu.data_ptr(),
+                                hy.data_ptr(), dev.data_ptr(), dev.numel() * dev.element_size(),
+                                _stream_ptr(stream))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_forward_host")
+    return hy
+
+
+def device_status(ws: torch.Tensor, stream=None) -> int:
+    return int(lib().gspn_device_status(ws.data_ptr(), _stream_ptr(stream)))
+
+
+def debug_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> int:
+    return int(lib().gspn_debug_wait_timeout(ws.data_ptr(), ws.numel(), int(limit_ns), _stream_ptr(stream)))
+
+
+def copy_ceiling(src: torch.Tensor, dst: torch.Tensor, stream=None):
+    nbytes = src.numel() * src.element_size()
+    s = lib().gspn_copy_ceiling(src.data_ptr(), dst.data_ptr(), nbytes, _stream_ptr(stream))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_copy_ceiling")
+
+
+class GSPNFunction(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run in libgspn."""
+
+    @staticmethod
+    def forward(ctx, x, a, lam, u, wmode, dir_mask):
+        ctx.save_for_backward(x, a, lam, u)
+        ctx.wmode, ctx.dir_mask = wmode, dir_mask
+        return forward(x, a, lam, u, wmode, dir_mask)
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, a, lam, u = ctx.saved_tensors
+        dx, da, dlam, du = backward(x, a, lam, u, dy.contiguous(), ctx.wmode, ctx.dir_mask)
+        return dx, da, dlam, du, None, None
+
+
+def gspn(x, a, lam, u, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL):
+    """Differentiable GSPN propagation (libgspn forward and backward)."""
+    return GSPNFunction.apply(x, a, lam, u, wmode, dir_mask)

@@ -1,0 +1,72 @@
+// gspn_internal.h -- host-side declarations shared by the libgspn translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gspn.h"
+
+namespace gspn {
+
+struct Problem {
+    int N, C, H, W;
+    int Cw;          // C (per-channel) or 1 (shared)
+    int D;           // number of directions in the mask
+    int wmode;
+    unsigned mask;
+    int dtype;       // GSPN_F32 / GSPN_BF16
+    long long HW;    // H * W
+    long long U;     // N * C * H * W
+    long long A;     // D * N * Cw * 3 * H * W
+    int esize() const { return dtype == GSPN_F32 ? 4 : 2; }
+};
+
+inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Workspace carving: a bump allocator over the caller's buffer (never allocates memory).
+struct WsCarver {
+    char* base;
+    size_t off;
+    explicit WsCarver(void* ws) : base((char*)ws), off(256) {}
+    template <typename T> T* take(size_t count) {
+        T* p = (T*)(base + off);
+        off += align256(count * sizeof(T));
+        return p;
+    }
+};
+
+// ---- generic family (any shape) -------------------------------------------------------
+size_t generic_ws_bytes(const Problem& p, bool bwd);
+bool generic_supports(const Problem& p, bool bwd);
+cudaError_t generic_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                            void* y, void* ws, cudaStream_t st);
+cudaError_t generic_backward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                             const void* dy, void* dx, void* da, void* dlam, void* du, void* ws,
+                             cudaStream_t st);
+
+// ---- plane family (small maps, whole plane on chip) ------------------------------------
+size_t plane_ws_bytes(const Problem& p, bool bwd);
+bool plane_supports(const Problem& p, bool bwd);
+cudaError_t plane_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                          void* y, void* ws, cudaStream_t st);
+cudaError_t plane_backward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                           const void* dy, void* dx, void* da, void* dlam, void* du, void* ws,
+                           cudaStream_t st);
+
+// ---- sweep family (large maps, TMA-fed line sweeps) ------------------------------------
+size_t sweep_ws_bytes(const Problem& p, bool bwd);
+bool sweep_supports(const Problem& p, bool bwd);
+cudaError_t sweep_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                          void* y, void* ws, cudaStream_t st);
+cudaError_t sweep_backward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                           const void* dy, void* dx, void* da, void* dlam, void* du, void* ws,
+                           cudaStream_t st);
+
+// ---- misc ------------------------------------------------------------------------------
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
+cudaError_t launch_wait_probe(unsigned* status, const unsigned* flag, unsigned long long limit_ns,
+                              cudaStream_t st);
+int device_sm_count();
+
+}  // namespace gspn
