@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of libgspn's 4-direction GSPN forward on one B200 per process.
+
+Default workload: N=16, C=8, H=W=1024, all four directions summed, channel-shared weights
+(logits N x 1 x 3 x H x W per direction) with per-channel lambda and u, fp32 storage.
+
+A step is one full forward (all directions, weight formation, injection, merge and gate)
+over one batch of synthetic input already resident in HBM. ``value`` is the compulsory HBM
+throughput of the whole job: (x, lambda, u read once + logits read once + y written once) x
+number of ranks / max-over-ranks device time. The inputs (2.95 GB per rank) are larger than L2,
+so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libgspn|reference]
+
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the data
+path); timing is bracketed by a barrier and a device synchronise and the max over ranks is
+reported. ``--impl reference`` times the float64 CPU oracle instead, on bounded samples of the
+same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gspn_inputs  # noqa: E402
+
+METRIC = "4-dir GSPN scan fwd ms & achieved HBM GB/s (frac of peak), 1024² B16 C8"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_highres.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="libgspn", choices=["libgspn", "reference"])
+    ap.add_argument("--workload", default="highres", choices=sorted(gspn_inputs.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-planes", type=int, default=24, help="planes of the CPU oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def env_rank():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def dtype_name(wl):
+    return "f32" if wl.dtype == "f32" else "bf16"
+
+
+def config_of(wl, world):
+    return {
+        "workload": wl.name,
+        "N": wl.N, "C": wl.C, "H": wl.H, "W": wl.W,
+        "directions": "TB+BT+LR+RL" if wl.mask == 15 else wl.mask,
+        "weights": "channel-shared" if wl.wmode else "per-channel",
+        "storage": wl.dtype,
+        "per_rank_batch": wl.N,
+        "global_batch": wl.N * world,
+        "parallelism": f"dp{world}" if world > 1 else "single",
+        "l2": "inputs larger than L2 (no flush)",
+    }
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+def oracle_plane_seconds_only(wl, planes):
+    """Oracle time excluding input generation."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(1)
+    H, W, D = wl.H, wl.W, wl.D
+    x = rng.standard_normal((1, 1, H, W))
+    a = rng.standard_normal((D, 1, 1, 3, H, W)) * wl.a_std
+    lam = rng.uniform(0, 1, (1, 1, H, W))
+    u = rng.standard_normal((1, 1, H, W))
+    t0 = time.perf_counter()
+    for _ in range(planes):
+        oracle.forward(x, a, lam, u, wl.wmode, wl.mask)
+    return time.perf_counter() - t0
+
+
+def plane_bytes(wl):
+    return (4 * wl.H * wl.W + (wl.D * 3 * wl.H * wl.W) // (wl.C if wl.wmode else 1)) * wl.elem_bytes
+
+
+def run_reference(args):
+    rank, _, world = env_rank()
+    wl = gspn_inputs.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    planes_per_step = 2
+    times = []
+    for s in range(args.warmup + args.steps):
+        dt = oracle_plane_seconds_only(wl, planes_per_step)
+        if s >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    nbytes = plane_bytes(wl) * planes_per_step * len(times)
+    value = nbytes / tot / 1e9
+    ms_per_step = tot / len(times) * 1e3 * (wl.N * wl.C) / planes_per_step
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, world),
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{planes_per_step} of {wl.N * wl.C} planes per step, float64 C oracle, "
+                                   "one thread; ms_per_step extrapolated to the full batch"},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- clocks sampler
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"gspn_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_spatial_propagation_gspn_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload):
+    """DRAM bytes per forward from the committed ncu summary, if the kernels are unchanged."""
+    if workload != "highres" or not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    if d.get("source_sha") != kernel_source_sha():
+        return None
+    return d.get("dram_bytes_per_forward")
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_libgspn(args):
+    import torch
+    import torch.distributed as dist
+    import linear_spatial_propagation_gspn_b200 as g
+
+    rank, local_rank, world = env_rank()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
+    wl = gspn_inputs.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    t = gspn_inputs.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
+    x, a, lam, u = t["x"], t["a"], t["lam"], t["u"]
+    desc = g.desc_for(x, wl.wmode, wl.mask)
+    algo = g.selected_algo(desc)
+    ws = g.alloc_workspace(desc, False, dev)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        g.forward(x, a, lam, u, wl.wmode, wl.mask, y=y, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if g.device_status(ws) != g.GSPN_OK:
+        raise RuntimeError("device status reports a timeout during warm-up")
+
+    # ---- timed region: K steps, events on the launching stream
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms_total = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    comp = wl.compulsory_fwd_bytes()
+    value = comp * world / (ms_step * 1e-3) / 1e9
+
+    # ---- per-kernel timing pass (events recorded by the library around each launch)
+    nk = 8
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]
+    for e in evs:
+        e.record(stream)  # materialise the event handles
+    torch.cuda.synchronize()
+    reps = max(5, min(50, args.steps // 4))
+    per = None
+    launches = 0
+    for _ in range(reps):
+        launches = g.forward_timed(x, a, lam, u, y, ws, desc, evs)
+        torch.cuda.synchronize()
+        d = [evs[2 * k].elapsed_time(evs[2 * k + 1]) for k in range(launches)]
+        per = d if per is None else [p + q for p, q in zip(per, d)]
+    per = [p / reps for p in per]
+    peak, peak_kind = measured_peak()
+    kern_ms = sum(per)
+    names = [n for n, bit in zip(("TB", "BT", "LR", "RL"), (1, 2, 4, 8)) if wl.mask & bit]
+    achieved = comp / (kern_ms * 1e-3) / 1e9
+    roofline = {
+        "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+        "frac": round(achieved / peak, 4), "traffic": committed_traffic(wl.name),
+        "peak_kind": peak_kind,
+        "what": (f"whole forward = {launches} sweep launches ({'+'.join(names)}); algorithmic bytes = compulsory "
+                 f"x, lam, u, a read once + y written once = {comp} B per forward"),
+        "kernels_ms": [round(p, 4) for p in per],
+    }
+
+    # ---- copy ceiling on the same byte volume
+    nb = (comp // 2) // 16 * 16
+    src = torch.empty(nb, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    for _ in range(3):
+        g.copy_ceiling(src, dst)
+    c0 = torch.cuda.Event(enable_timing=True)
+    c1 = torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(10):
+        g.copy_ceiling(src, dst)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    copy_gbs = 2 * nb * 10 / (c0.elapsed_time(c1) * 1e-3) / 1e9
+    del src, dst
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hx, ha, hl, hu = (tt.cpu().pin_memory() for tt in (x, a, lam, u))
+        hy = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+        dev_buf = torch.empty(g.forward_host_buffer_size(desc), dtype=torch.uint8, device=dev)
+        g.forward_host(desc, hx, ha, hl, hu, hy, dev_buf)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        q0 = torch.cuda.Event(enable_timing=True)
+        q1 = torch.cuda.Event(enable_timing=True)
+        q0.record(stream)
+        for _ in range(args.e2e_steps):
+            g.forward_host(desc, hx, ha, hl, hu, hy, dev_buf)
+        q1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = q0.elapsed_time(q1) / args.e2e_steps
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        h2d = sum(tt.numel() * tt.element_size() for tt in (hx, ha, hl, hu))
+        d2h = hy.numel() * hy.element_size()
+        e2e = {"value": round(comp * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "gspn_forward_host (pinned host buffers)"}
+        del dev_buf
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs = oracle_plane_seconds_only(wl, args.cpu_planes)
+        cpu = {"value": round(plane_bytes(wl) * args.cpu_planes / secs / 1e9, 6), "unit": "GB/s", "cores": 1,
+               "kind": "oracle",
+               "sample": f"{args.cpu_planes} of {wl.N * wl.C} (n,c) planes, float64 C oracle, one thread, "
+                         f"{secs:.1f} s"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": dtype_name(wl), "data": "synthetic (seeded torch.randn/rand on device)",
+            "config": config_of(wl, world),
+            "algo": g.ALGO_NAMES.get(algo, str(algo)),
+            "roofline": roofline,
+            "copy_ceiling_gbs": round(copy_gbs, 1),
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_libgspn(args)
+
+
+if __name__ == "__main__":
+    main()

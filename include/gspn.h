@@ -117,6 +117,14 @@ GSPN_API gspn_status gspn_backward(const gspn_desc *desc, const void *x, const v
                           const void *u, const void *dy, void *dx, void *da, void *dlam, void *du,
                           void *ws, size_t ws_bytes, void *stream);
 
+/* gspn_forward that also records CUDA events around each kernel launch it makes, for
+ * per-kernel timing on the launching stream: events[2k] before and events[2k+1] after launch k
+ * (cudaEvent_t handles created by the caller). *n_launches receives the number of launches;
+ * launches beyond n_events/2 are not timed. Otherwise identical to gspn_forward. */
+GSPN_API gspn_status gspn_forward_timed(const gspn_desc *desc, const void *x, const void *a, const void *lam,
+                               const void *u, void *y, void *ws, size_t ws_bytes, void *stream,
+                               void *const *events, int n_events, int *n_launches);
+
 /* Bytes of device staging buffer that gspn_forward_host needs (inputs, output and
  * workspace, each 256-byte aligned). */
 GSPN_API size_t gspn_forward_host_buffer_size(const gspn_desc *desc);

@@ -56,6 +56,7 @@ SIGNATURES = {
     "gspn_selected_algo": (_I, [_DP, _I]),
     "gspn_forward": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "gspn_backward": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "gspn_forward_timed": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP, _VP, _I, ctypes.POINTER(_I)]),
     "gspn_forward_host_buffer_size": (_SZ, [_DP]),
     "gspn_forward_host": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "gspn_device_status": (_I, [_VP, _VP]),
@@ -184,6 +185,19 @@ def backward(x, a, lam, u, dy, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL
     if s != GSPN_OK:
         raise GspnError(s, "gspn_backward")
     return dx, da, dlam, du
+
+
+def forward_timed(x, a, lam, u, y, ws, desc: GspnDesc, events, stream=None) -> int:
+    """gspn_forward recording ``events`` (materialised torch.cuda.Event objects, two per launch)
+    around each kernel launch; returns the number of launches."""
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    n = ctypes.c_int(0)
+    s = lib().gspn_forward_timed(ctypes.byref(desc), x.data_ptr(), a.data_ptr(), lam.data_ptr(), u.data_ptr(),
+                                 y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream), arr, len(events),
+                                 ctypes.byref(n))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_forward_timed")
+    return n.value
 
 
 def forward_host_buffer_size(desc: GspnDesc) -> int:

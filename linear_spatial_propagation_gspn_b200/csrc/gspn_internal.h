@@ -63,6 +63,12 @@ cudaError_t sweep_backward(const Problem& p, const void* x, const void* a, const
                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws,
                            cudaStream_t st);
 
+// ---- per-launch timing hooks (gspn_forward_timed) ---------------------------------------
+// Kernel families call launch_begin / launch_end around every kernel launch. When a timed
+// call is active on this host thread they record the caller's events on the launch stream.
+void launch_begin(cudaStream_t st);
+void launch_end(cudaStream_t st);
+
 // ---- misc ------------------------------------------------------------------------------
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_wait_probe(unsigned* status, const unsigned* flag, unsigned long long limit_ns,

@@ -200,7 +200,9 @@ cudaError_t gen_forward_t(const Problem& P, const void* x, const void* a, const 
         const int M = is_vertical(d) ? P.W : P.H;
         const size_t smem = 2 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        launch_begin(st);
         k_gen_fwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(g);
+        launch_end(st);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         ++slot;
