@@ -150,6 +150,25 @@ GSPN_API gspn_status gspn_debug_wait_timeout(void *ws, size_t ws_bytes, unsigned
  * vectorised grid-stride kernel: the bandwidth ceiling the sweeps are compared with. */
 GSPN_API gspn_status gspn_copy_ceiling(const void *src, void *dst, size_t bytes, void *stream);
 
+/* Size of the fixed device scratch array used by gspn_forward_noalloc (64 MiB). */
+#define GSPN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* gspn_forward without any allocation by anyone: the workspace comes from a fixed device array
+ * of GSPN_NOALLOC_SCRATCH_BYTES compiled into the library (the pages have no counterpart; this
+ * exists for callers that cannot allocate device memory at call time, e.g. code running under
+ * another component's allocator or on a path where cudaMalloc/cudaFree would synchronise the
+ * device). x, a, lam, u, y are device pointers on the current device; `stream` belongs to it.
+ *   - Returns GSPN_ERR_WORKSPACE, before touching the device, if the descriptor needs more
+ *     workspace than GSPN_NOALLOC_SCRATCH_BYTES (gspn_workspace_size(desc, 0) tells).
+ *   - The first call on each device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the last call's contents (each
+ *     call rewrites what it reads): calls that overlap on the GPU, from any stream or thread,
+ *     race on it. Serialise them.
+ *   - Every GPU that loads the library holds the array until the process exits. */
+GSPN_API gspn_status gspn_forward_noalloc(const gspn_desc *desc, const void *x, const void *a,
+                                          const void *lam, const void *u, void *y, void *stream);
+
 GSPN_API const char *gspn_status_string(gspn_status s);
 GSPN_API int gspn_version(void);
 

@@ -62,6 +62,7 @@ SIGNATURES = {
     "gspn_device_status": (_I, [_VP, _VP]),
     "gspn_debug_wait_timeout": (_I, [_VP, _SZ, _U64, _VP]),
     "gspn_copy_ceiling": (_I, [_VP, _VP, _SZ, _VP]),
+    "gspn_forward_noalloc": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "gspn_status_string": (ctypes.c_char_p, [_I]),
     "gspn_version": (_I, []),
 }
