@@ -279,14 +279,16 @@ def run_libgspn(args):
     peak, peak_kind = measured_peak()
     kern_ms = sum(per)
     names = [n for n, bit in zip(("TB", "BT", "LR", "RL"), (1, 2, 4, 8)) if wl.mask & bit]
+    if launches == len(names) + 1:
+        names = ["weights"] + names
     achieved = comp / (kern_ms * 1e-3) / 1e9
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4), "traffic": committed_traffic(wl.name),
         "peak_kind": peak_kind,
-        "what": (f"whole forward = {launches} sweep launches ({'+'.join(names)}); algorithmic bytes = compulsory "
-                 f"x, lam, u, a read once + y written once = {comp} B per forward"),
-        "kernels_ms": [round(p, 4) for p in per],
+        "what": (f"whole forward = {launches} launches ({'+'.join(names)}); algorithmic bytes = compulsory "
+                 f"x, lam, u, a read once + y written once = {comp} B per forward; time = sum of the launches"),
+        "kernels_ms": {n: round(p, 4) for n, p in zip(names, per)} if len(names) == len(per) else [round(p, 4) for p in per],
     }
 
     # ---- copy ceiling on the same byte volume

@@ -55,54 +55,70 @@ __host__ __device__ __forceinline__ int dir_slot(unsigned mask, unsigned d) {
 // with D = p1 p2 + p0 p2 + p0 p1: three exponentials and one reciprocal per lane. The
 // products stay finite while every in-range logit is >= -40; below that the weights are
 // formed from log-sigmoids shifted by their maximum, which is finite for every finite logit.
-static __device__ __noinline__ void weights_slow(float a0, float a1, float a2, bool has_l, bool has_r,
-                                          float& w0, float& w1, float& w2) {
-    // log sigmoid(a) = -softplus(-a) = -(max(-a, 0) + log1p(exp(-|a|)))
+// Everything here is inline and returns by value, so no weight ever touches local memory.
+struct Wts {
+    float w0, w1, w2;
+};
+
+constexpr float kShiftBelow = -40.f;
+
+// True when some in-range logit is below kShiftBelow (then the shifted form must be used).
+__device__ __forceinline__ bool weights_need_shift(float a0, float a1, float a2, bool has_l, bool has_r) {
+    const float amin = fminf(a1, fminf(has_l ? a0 : a1, has_r ? a2 : a1));
+    return amin < kShiftBelow;
+}
+
+// log sigmoid(a) = -softplus(-a) = -(max(-a, 0) + log1p(exp(-|a|))); weights = exp(l_k - max l).
+__device__ __forceinline__ Wts weights_shifted(float a0, float a1, float a2, bool has_l, bool has_r) {
     auto logsig = [](float a) { return -(fmaxf(-a, 0.f) + log1pf(expf(-fabsf(a)))); };
-    float l0 = has_l ? logsig(a0) : -INFINITY;
-    float l1 = logsig(a1);
-    float l2 = has_r ? logsig(a2) : -INFINITY;
-    float m = fmaxf(l1, fmaxf(l0, l2));
-    float e0 = has_l ? expf(l0 - m) : 0.f;
-    float e1 = expf(l1 - m);
-    float e2 = has_r ? expf(l2 - m) : 0.f;
-    float inv = 1.0f / (e0 + e1 + e2);
-    w0 = e0 * inv;
-    w1 = e1 * inv;
-    w2 = e2 * inv;
+    const float l0 = has_l ? logsig(a0) : -INFINITY;
+    const float l1 = logsig(a1);
+    const float l2 = has_r ? logsig(a2) : -INFINITY;
+    const float m = fmaxf(l1, fmaxf(l0, l2));
+    const float e0 = has_l ? expf(l0 - m) : 0.f;
+    const float e1 = expf(l1 - m);
+    const float e2 = has_r ? expf(l2 - m) : 0.f;
+    const float inv = 1.0f / (e0 + e1 + e2);
+    return Wts{e0 * inv, e1 * inv, e2 * inv};
+}
+
+// Common-denominator numerators with the out-of-range terms removed (branch-free in edge lanes):
+// interior q = (p1 p2, p0 p2, p0 p1); no left (0, p2, p1); no right (p1, p0, 0); single (0, 1, 0).
+__device__ __forceinline__ Wts weights_from_p(float p0, float p1, float p2, bool has_l, bool has_r) {
+    const float l = has_l ? p0 : 1.f;
+    const float r = has_r ? p2 : 1.f;
+    return Wts{has_l ? p1 * r : 0.f, l * r, has_r ? p1 * l : 0.f};
+}
+
+// Accurate form (expf, IEEE reciprocal); used by the generic family and the backward.
+__device__ __forceinline__ Wts lane_weights_acc(float a0, float a1, float a2, bool has_l, bool has_r) {
+    if (weights_need_shift(a0, a1, a2, has_l, has_r)) return weights_shifted(a0, a1, a2, has_l, has_r);
+    const Wts q = weights_from_p(1.f + expf(-a0), 1.f + expf(-a1), 1.f + expf(-a2), has_l, has_r);
+    const float inv = __frcp_rn(q.w0 + q.w1 + q.w2);
+    return Wts{q.w0 * inv, q.w1 * inv, q.w2 * inv};
 }
 
 __device__ __forceinline__ void lane_weights(float a0, float a1, float a2, bool has_l, bool has_r,
                                              float& w0, float& w1, float& w2) {
-    float amin = fminf(a1, fminf(has_l ? a0 : a1, has_r ? a2 : a1));
-    if (amin < -40.f) {
-        weights_slow(a0, a1, a2, has_l, has_r, w0, w1, w2);
-        return;
-    }
-    float p0 = 1.f + expf(-a0);
-    float p1 = 1.f + expf(-a1);
-    float p2 = 1.f + expf(-a2);
-    if (has_l && has_r) {
-        float q0 = p1 * p2, q1 = p0 * p2, q2 = p0 * p1;
-        float inv = __frcp_rn(q0 + q1 + q2);
-        w0 = q0 * inv;
-        w1 = q1 * inv;
-        w2 = q2 * inv;
-    } else if (has_r) {          // lane 0: neighbours k = 1, 2
-        float inv = __frcp_rn(p1 + p2);
-        w0 = 0.f;
-        w1 = p2 * inv;
-        w2 = p1 * inv;
-    } else if (has_l) {          // last lane: neighbours k = 0, 1
-        float inv = __frcp_rn(p0 + p1);
-        w0 = p1 * inv;
-        w1 = p0 * inv;
-        w2 = 0.f;
-    } else {                     // single lane
-        w0 = 0.f;
-        w1 = 1.f;
-        w2 = 0.f;
-    }
+    const Wts w = lane_weights_acc(a0, a1, a2, has_l, has_r);
+    w0 = w.w0;
+    w1 = w.w1;
+    w2 = w.w2;
+}
+
+// Fast form from the MUFU approximations (__expf: relative error about 2 ulp plus the rounding
+// of the scaled argument; __fdividef: about 2 ulp). The normalisation is applied after the
+// approximations, so every row still sums to one up to a few ulp and the small weight errors do
+// not compound along the scan. Branch-free: the arguments are clamped at kShiftBelow so the
+// products never overflow; a caller must redo lanes for which weights_need_shift() holds with
+// weights_shifted() (kernels do that behind one warp vote per step, the path is rare).
+__device__ __forceinline__ Wts lane_weights_fast_nocheck(float a0, float a1, float a2, bool has_l, bool has_r) {
+    const float p0 = 1.f + __expf(-fmaxf(a0, kShiftBelow));
+    const float p1 = 1.f + __expf(-fmaxf(a1, kShiftBelow));
+    const float p2 = 1.f + __expf(-fmaxf(a2, kShiftBelow));
+    const Wts q = weights_from_p(p0, p1, p2, has_l, has_r);
+    const float inv = __fdividef(1.f, q.w0 + q.w1 + q.w2);
+    return Wts{q.w0 * inv, q.w1 * inv, q.w2 * inv};
 }
 
 // Weights and Jacobian factors of one lane for the backward:

@@ -1,28 +1,32 @@
-// k_sweep.cu -- large-map kernel family of libgspn: persistent, TMA-fed line sweeps.
+// k_sweep.cu -- large-map kernel family of libgspn: persistent line sweeps.
 //
 // One sweep per direction in the mask, in the order TB, BT, LR, RL. Every sweep is one
-// persistent kernel: each CTA owns whole planes (a line of a scan couples all its lanes, so
-// a line cannot be split across CTAs without a per-step exchange) and runs the sequential
-// scan over the plane with the running line h_{i-1} in registers. Inputs stream through a
-// shared-memory ring filled by the TMA engine; every step ends with one named barrier that
-// also exchanges the neighbour values across warps, and after it thread 0 refills the stage
-// that was just consumed. No direction issues strided HBM traffic:
-//   - vertical sweeps (TB, BT) read whole image rows with 1D bulk copies; each thread owns 4
-//     consecutive lanes, read with one 16-byte (fp32) or 8-byte (bf16) shared load;
-//   - horizontal sweeps (LR, RL) read [H rows x 16 bytes] column tiles with 2D tensor copies
-//     (a staged transpose); each thread owns rows t, t+T, ... and reads 16 bytes (4 fp32 or
-//     8 bf16 steps) of each of its rows, conflict-free; outputs are gathered for the tile and
-//     written back as 16-byte row segments.
-// The first sweep reads x and lambda and writes z = lambda * x and the partial sum; later
-// sweeps read z and the partial sum (both in the storage dtype); the last one reads u and
-// writes y = u * (partial + h). ("GSPN-2: Efficient Parallel Sequence Modeling" paper notes,
-// section "Optimisation 3: efficient CUDA extension": coalesced access and on-chip reuse of
-// h_{i-1} were the decisive optimisations on A100; here the line stays in registers.)
+// persistent kernel: each CTA owns whole planes (a line of a scan couples all its lanes, so a
+// line cannot be split across CTAs without a per-step exchange) and runs the sequential scan
+// over the plane with the running line h_{i-1} in registers; one barrier per step exchanges the
+// neighbour values across warps. Inputs stream through a shared-memory ring filled with
+// per-thread asynchronous copies (cp.async): each thread copies exactly the lanes it will read,
+// several steps ahead, so no thread waits for another's data. (Measured on B200: a TMA bulk copy
+// costs about 285 ns per operation per SM whatever its size up to 32 KB, and the operations of
+// one SM are serialised; a sweep needs 5-7 row-sized copies per step, which capped it near
+// 1.2-1.9 us per step. Per-thread copies have no such per-operation cost.)
+//   - vertical sweeps (TB, BT): thread t owns LPT consecutive lanes of a row; its copies are
+//     contiguous across the warp (fully coalesced);
+//   - horizontal sweeps (LR, RL): column tiles of 16 bytes per row (4 fp32 or 8 bf16 steps, a
+//     staged transpose); thread t owns rows t, t+T, ..., copies and reads 16 bytes per row per
+//     tensor (conflict-free), and writes its outputs back as 16-byte row segments.
+// No direction issues strided per-element HBM traffic. The first sweep reads x and lambda and
+// writes z = lambda * x and the partial sum; later sweeps read z and the partial sum (both in the
+// storage dtype); the last one reads u and writes y = u * (partial + h). ("GSPN-2: Efficient
+// Parallel Sequence Modeling" paper notes, section "Optimisation 3: efficient CUDA extension":
+// coalesced access and on-chip reuse of h_{i-1} were the decisive optimisations on A100.)
+#include <stdlib.h>
+
 #include <algorithm>
+#include <type_traits>
 
 #include "gspn_common.cuh"
 #include "gspn_internal.h"
-#include "tma.cuh"
 
 namespace gspn {
 namespace {
@@ -34,54 +38,48 @@ template <int MODE> struct ModeT {
     static constexpr bool ACCIN = MODE == M_MID || MODE == M_LAST;    // read the partial sum
     static constexpr bool FINAL = MODE == M_ONLY || MODE == M_LAST;   // read u, write y
     static constexpr bool ZOUT = MODE == M_FIRST;                     // write z
-    // tensors per stage: a0 a1 a2, x lam | z, [acc], [u]
-    static constexpr int NTEN = 3 + (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (FINAL ? 1 : 0);
+    // storage-dtype tensors per stage: x lam | z, [acc], [u]  (plus the two fp32 weight rows)
+    static constexpr int NTEN = (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (FINAL ? 1 : 0);
 };
 
 struct SweepArgs {
     const void* x;
     const void* lam;
     const void* u;
-    const void* a;
-    void* z;       // workspace, storage dtype
-    void* acc;     // workspace, storage dtype
+    const float* wt;  // weight table of this direction's slot: [N][Cw][2][H][W] fp32 (w0, w2)
+    void* z;          // workspace, storage dtype
+    void* acc;        // workspace, storage dtype
     void* y;
     int N, C, H, W, Cw;
-    int slot;
-    int ns;        // pipeline stages
-    unsigned* status;
-    unsigned long long limit_ns;
 };
 
-constexpr unsigned long long kWaitLimitNs = 2000000000ULL;  // 2 s
-
-// ------------------------------------------------------------------ 4-lane vectors
-template <typename T> struct V4;
-template <> struct V4<float> {
-    static __device__ __forceinline__ void ld(const void* p, float v[4]) {
-        float4 q = *(const float4*)p;
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    }
-    static __device__ __forceinline__ void st(void* p, const float v[4]) { *(float4*)p = make_float4(v[0], v[1], v[2], v[3]); }
-};
-template <> struct V4<__nv_bfloat16> {
-    static __device__ __forceinline__ void ld(const void* p, float v[4]) {
-        uint2 q = *(const uint2*)p;
-        float2 f0 = __bfloat1622float2(*(const __nv_bfloat162*)&q.x);
-        float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&q.y);
-        v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
-    }
-    static __device__ __forceinline__ void st(void* p, const float v[4]) {
-        __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
-        __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
-        uint2 q;
-        q.x = *(const uint32_t*)&b0;
-        q.y = *(const uint32_t*)&b1;
-        *(uint2*)p = q;
-    }
+struct WeightArgs {
+    const void* a;    // logits [D][N][Cw][3][H][W]
+    float* wt;        // table  [D][N][Cw][2][H][W]
+    int N, Cw, H, W, D;
+    unsigned dirs[4]; // direction bit of each slot
 };
 
-// 16-byte row segment: 4 fp32 or 8 bf16 consecutive steps of one lane.
+// ------------------------------------------------------------------ async copies
+__device__ __forceinline__ uint32_t smem_u32(const void* ptr) { return (uint32_t)__cvta_generic_to_shared(ptr); }
+
+// Global -> shared copy of BYTES (4, 8 or 16) bytes, both addresses aligned to BYTES. 16-byte
+// copies bypass L1 (.cg); smaller ones must use .ca.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void* dst, const void* src) {
+    if constexpr (BYTES == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_u32(dst)), "l"(src), "n"(BYTES)
+                     : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ------------------------------------------------------------------ 16-byte row segments
+// 16 bytes = 4 fp32 or 8 bf16 consecutive steps of one lane.
 template <typename T> struct Seg;
 template <> struct Seg<float> {
     static constexpr int S = 4;
@@ -107,279 +105,466 @@ template <> struct Seg<__nv_bfloat16> {
     }
 };
 
-__device__ __forceinline__ unsigned char* align128(unsigned char* p) {
-    return (unsigned char*)(((uintptr_t)p + 127) & ~(uintptr_t)127);
+__device__ __forceinline__ unsigned char* align128(unsigned char* ptr) {
+    return (unsigned char*)(((uintptr_t)ptr + 127) & ~(uintptr_t)127);
+}
+
+// L consecutive lanes of storage type T (aligned to L elements).
+template <typename T, int L>
+__device__ __forceinline__ void ld_lanes(const void* ptr, float (&v)[L]) {
+    if constexpr (L == 8) {
+        if constexpr (std::is_same<T, float>::value) {
+            const float4 q0 = *(const float4*)ptr, q1 = *((const float4*)ptr + 1);
+            v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
+            v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
+        } else {
+            const uint4 q = *(const uint4*)ptr;
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&w[k]);
+                v[2 * k] = f.x;
+                v[2 * k + 1] = f.y;
+            }
+        }
+    } else if constexpr (std::is_same<T, float>::value) {
+        if constexpr (L == 1) {
+            v[0] = *(const float*)ptr;
+        } else if constexpr (L == 2) {
+            const float2 q = *(const float2*)ptr;
+            v[0] = q.x; v[1] = q.y;
+        } else {
+            const float4 q = *(const float4*)ptr;
+            v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+        }
+    } else {
+        if constexpr (L == 1) {
+            v[0] = __bfloat162float(*(const __nv_bfloat16*)ptr);
+        } else if constexpr (L == 2) {
+            const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)ptr);
+            v[0] = f.x; v[1] = f.y;
+        } else {
+            const uint2 q = *(const uint2*)ptr;
+            const float2 f0 = __bfloat1622float2(*(const __nv_bfloat162*)&q.x);
+            const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&q.y);
+            v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+        }
+    }
+}
+
+template <typename T, int L>
+__device__ __forceinline__ void st_lanes(void* ptr, const float (&v)[L]) {
+    if constexpr (L == 8) {
+        if constexpr (std::is_same<T, float>::value) {
+            *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
+            *((float4*)ptr + 1) = make_float4(v[4], v[5], v[6], v[7]);
+        } else {
+            uint4 q;
+            uint32_t* w = &q.x;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+                w[k] = *(const uint32_t*)&b;
+            }
+            *(uint4*)ptr = q;
+        }
+    } else if constexpr (std::is_same<T, float>::value) {
+        if constexpr (L == 1) *(float*)ptr = v[0];
+        else if constexpr (L == 2) *(float2*)ptr = make_float2(v[0], v[1]);
+        else *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+        if constexpr (L == 1) {
+            *(__nv_bfloat16*)ptr = __float2bfloat16_rn(v[0]);
+        } else if constexpr (L == 2) {
+            *(__nv_bfloat162*)ptr = __floats2bfloat162_rn(v[0], v[1]);
+        } else {
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
+            uint2 q;
+            q.x = *(const uint32_t*)&b0;
+            q.y = *(const uint32_t*)&b1;
+            *(uint2*)ptr = q;
+        }
+    }
+}
+
+// A thread's LPT lanes of one row in shared memory. With fp32 and LPT = 8 a thread owns 32
+// bytes, and threads t and t+4 would hit the same banks in a 16-byte load phase; the thread
+// therefore stores its two 16-byte chunks in swapped order when bit 2 of its index is set
+// (`sw`), which makes every load phase conflict-free. Each thread writes and reads only its own
+// chunks, so the swizzle is private to the thread.
+template <typename T, int LPT>
+__device__ __forceinline__ void copy_lanes(unsigned char* dst, const T* src, int sw) {
+    constexpr int VB = LPT * (int)sizeof(T);
+    if constexpr (VB == 32) {
+        cp_async<16>(dst + 16 * sw, src);
+        cp_async<16>(dst + 16 * (1 - sw), src + 4);
+    } else {
+        cp_async<VB>(dst, src);
+    }
+}
+template <typename T, int LPT>
+__device__ __forceinline__ void read_lanes(const unsigned char* srcs, float (&v)[LPT], int sw) {
+    constexpr int VB = LPT * (int)sizeof(T);
+    if constexpr (VB == 32) {
+        const float4 q0 = *(const float4*)(srcs + 16 * sw), q1 = *(const float4*)(srcs + 16 * (1 - sw));
+        v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
+        v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
+    } else {
+        ld_lanes<T, LPT>(srcs, v);
+    }
+}
+
+
+// ================================================================== weight formation (A1)
+// Turns the logits of every (slot, n, cw) plane into the two outer weights w0, w2 of each
+// normalised tridiagonal row; the sweeps re-derive w1 = 1 - w0 - w2, so every row sums to one.
+// Elementwise and memory-bound: one thread per 4 consecutive pixels of a row, accurate expf and
+// IEEE reciprocal. blockIdx.y = plane, so no 64-bit division is needed.
+template <typename T>
+__global__ void __launch_bounds__(256) k_sweep_weights(WeightArgs p) {
+    const long long HW = (long long)p.H * p.W;
+    const int plane = blockIdx.y;                      // (slot, n, cw)
+    const int slot = plane / (p.N * p.Cw);
+    const unsigned d = p.dirs[slot];
+    const T* a3 = (const T*)p.a + (long long)plane * 3 * HW;
+    float* wt = p.wt + (long long)plane * 2 * HW;
+    const int quads = (int)(HW / 4);
+    for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < quads; q += gridDim.x * blockDim.x) {
+        const int pix = q * 4;
+        const int r = pix / p.W, c0 = pix - r * p.W;
+        float a0[4], a1[4], a2[4], w0[4], w2[4];
+        ld_lanes<T, 4>(a3 + pix, a0);
+        ld_lanes<T, 4>(a3 + HW + pix, a1);
+        ld_lanes<T, 4>(a3 + 2 * HW + pix, a2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int c = c0 + k;
+            const bool hl = is_vertical(d) ? c > 0 : r > 0;
+            const bool hr = is_vertical(d) ? c < p.W - 1 : r < p.H - 1;
+            const Wts w = lane_weights_acc(a0[k], a1[k], a2[k], hl, hr);
+            w0[k] = w.w0;
+            w2[k] = w.w2;
+        }
+        st_lanes<float, 4>(wt + pix, w0);
+        st_lanes<float, 4>(wt + HW + pix, w2);
+    }
 }
 
 // ================================================================== vertical sweep
-// CTA = one plane at a time (persistent over planes b, b + grid, ...), blockDim = W/4 rounded
-// up to a warp multiple. Stage = one image row of each input tensor.
-template <typename T, unsigned DIR, int MODE>
-__global__ void __launch_bounds__(1024, 1) k_vsweep(SweepArgs p) {
+// CTA = one plane at a time (persistent over planes b, b + grid, ...); thread t owns lanes
+// [LPT t, LPT t + LPT). Ring of NS stages; a stage is one image row of the two fp32 weight
+// rows and of each storage-dtype input. Every thread keeps NS rows of its own lanes in flight.
+// The loop is software-pipelined by one step: while step g's new line is exchanged at the
+// barrier, every thread has already pulled step g+1's inputs out of the ring.
+template <typename T, unsigned DIR, int MODE, int LPT, int NS>
+__global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p) {
     using Md = ModeT<MODE>;
     constexpr int NTEN = Md::NTEN;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align128(smem_raw);
-    const int H = p.H, W = p.W, NS = p.ns;
+    const int H = p.H, W = p.W;
     const int rowB = W * (int)sizeof(T);
-    const int stageB = NTEN * rowB;
-    unsigned char* stages = smem;
+    const int wrowB = W * 4;
+    const int stageB = 2 * wrowB + NTEN * rowB;
     float* halo = (float*)(smem + (size_t)NS * stageB);   // [2 parity][2 lo/hi][32 warps]
-    uint64_t* full = (uint64_t*)(halo + 128);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    const int j0 = tid * 4;
+    const int j0 = tid * LPT;
     const bool active = j0 < W;
+    const int sw = (tid >> 2) & 1;
     const long long HW = (long long)H * W;
     const int nplanes = p.N * p.C;
     const int my_planes = (nplanes - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const long long total = (long long)my_planes * H;
+    const size_t wofs = (size_t)j0 * 4;                                  // this thread in a weight row
+    const size_t tofs = 2 * (size_t)wrowB + (size_t)j0 * sizeof(T);      // ... in the first T row
 
-    if (tid == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    auto issue = [&](long long g) {
-        const int k = (int)(g / H), i = (int)(g % H);
-        const int plane = (int)blockIdx.x + k * (int)gridDim.x;
-        const int n = plane / p.C, c = plane % p.C;
-        const int r = DIR == kTB ? i : H - 1 - i;
-        unsigned char* st = stages + (size_t)(g % NS) * stageB;
-        uint64_t* bar = &full[g % NS];
-        mbar_arrive_expect_tx(bar, (uint32_t)stageB);
-        const T* a3 = (const T*)p.a + (((long long)p.slot * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW +
-                      (long long)r * W;
-        tma_load_1d(st, a3, rowB, bar);
-        tma_load_1d(st + rowB, a3 + HW, rowB, bar);
-        tma_load_1d(st + 2 * rowB, a3 + 2 * HW, rowB, bar);
-        const long long off = (long long)plane * HW + (long long)r * W;
-        int t = 3;
-        if (Md::XL) {
-            tma_load_1d(st + (t++) * rowB, (const T*)p.x + off, rowB, bar);
-            tma_load_1d(st + (t++) * rowB, (const T*)p.lam + off, rowB, bar);
-        } else {
-            tma_load_1d(st + (t++) * rowB, (const T*)p.z + off, rowB, bar);
-        }
-        if (Md::ACCIN) tma_load_1d(st + (t++) * rowB, (const T*)p.acc + off, rowB, bar);
-        if (Md::FINAL) tma_load_1d(st + (t++) * rowB, (const T*)p.u + off, rowB, bar);
+    // Issue cursor: rows are requested strictly in step order, so plane, row and stage advance
+    // incrementally (no division inside the loop).
+    long long iss_left = total;
+    int iss_i = 0, iss_s = 0, iss_plane = (int)blockIdx.x;
+    const float* iss_wt = nullptr;
+    long long iss_poff = 0;
+    auto iss_plane_setup = [&]() {
+        const int n = iss_plane / p.C, c = iss_plane % p.C;
+        iss_wt = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
+        iss_poff = (long long)iss_plane * HW;
     };
-    if (tid == 0)
-        for (long long g = 0; g < NS && g < total; ++g) issue(g);
-
-    float h[4] = {0.f, 0.f, 0.f, 0.f};
-    long long g = 0;
-    bool failed = false;
-    for (; g < total; ++g) {
-        const int i = (int)(g % H);
-        const int k = (int)(g / H);
-        if (i == 0) { h[0] = h[1] = h[2] = h[3] = 0.f; }
-        const int s = (int)(g % NS);
-        const bool ok = mbar_wait_bounded(&full[s], (uint32_t)((g / NS) & 1), p.limit_ns, p.status);
-        // neighbours from the previous step: lane j0-1 and lane j0+4
-        const float* hprev = halo + ((g + 1) & 1) * 64;
-        float hl = __shfl_up_sync(0xffffffffu, h[3], 1);
-        float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
-        if (lane == 0) hl = warp > 0 ? hprev[32 + warp - 1] : 0.f;
-        if (lane == 31) hr = warp < nw - 1 ? hprev[warp + 1] : 0.f;
-        float hn[4] = {0.f, 0.f, 0.f, 0.f};
-        if (active) {
-            const unsigned char* st = stages + (size_t)s * stageB + (size_t)j0 * sizeof(T);
-            float zz[4], src1[4];
-            V4<T>::ld(st + (Md::XL ? 3 : 3) * rowB, zz);
-            if (Md::XL) {
-                V4<T>::ld(st + 4 * rowB, src1);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) zz[e] *= src1[e];   // z = x * lam
+    auto issue = [&]() {
+        if (iss_left > 0) {
+            if (active) {
+                const int r = DIR == kTB ? iss_i : H - 1 - iss_i;
+                unsigned char* st = smem + (size_t)iss_s * stageB;
+                const long long ro = (long long)r * W + j0;
+                copy_lanes<float, LPT>(st + wofs, iss_wt + ro, sw);
+                copy_lanes<float, LPT>(st + wrowB + wofs, iss_wt + HW + ro, sw);
+                const long long off = iss_poff + ro;
+                unsigned char* sd = st + tofs;
+                int t = 0;
+                if (Md::XL) {
+                    copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.x + off, sw);
+                    copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.lam + off, sw);
+                } else {
+                    copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.z + off, sw);
+                }
+                if (Md::ACCIN) copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.acc + off, sw);
+                if (Md::FINAL) copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.u + off, sw);
             }
+            --iss_left;
+            if (++iss_s == NS) iss_s = 0;
+            if (++iss_i == H) {
+                iss_i = 0;
+                iss_plane += (int)gridDim.x;
+                if (iss_plane < nplanes) iss_plane_setup();
+            }
+        }
+        cp_async_commit();   // always one group per call, so the wait counts stay uniform
+    };
+    iss_plane_setup();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) hn[e] = zz[e];
-            if (i > 0) {
-                float a0[4], a1[4], a2[4];
-                V4<T>::ld(st, a0);
-                V4<T>::ld(st + rowB, a1);
-                V4<T>::ld(st + 2 * rowB, a2);
+    for (int q = 0; q < NS; ++q) issue();
+
+    // inputs of the next step, already out of shared memory
+    float nz[LPT], nacc[LPT], nu[LPT], nw0[LPT], nw2[LPT];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = j0 + e;
-                    float w0, w1, w2;
-                    lane_weights(a0[e], a1[e], a2[e], j > 0, j < W - 1, w0, w1, w2);
+    for (int e = 0; e < LPT; ++e) nz[e] = nacc[e] = nu[e] = nw0[e] = nw2[e] = 0.f;
+    int fs = 0;   // consumer stage
+    auto fetch = [&]() {
+        cp_async_wait<NS - 1>();
+        if (active) {
+            const unsigned char* st = smem + (size_t)fs * stageB;
+            read_lanes<float, LPT>(st + wofs, nw0, sw);
+            read_lanes<float, LPT>(st + wrowB + wofs, nw2, sw);
+            const unsigned char* sd = st + tofs;
+            read_lanes<T, LPT>(sd, nz, sw);
+            if (Md::XL) {
+                float l2[LPT];
+                read_lanes<T, LPT>(sd + rowB, l2, sw);
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) nz[e] *= l2[e];     // z = x * lam
+            }
+            int t = Md::XL ? 2 : 1;
+            if (Md::ACCIN) read_lanes<T, LPT>(sd + (t++) * rowB, nacc, sw);
+            if (Md::FINAL) read_lanes<T, LPT>(sd + (t++) * rowB, nu, sw);
+        }
+        if (++fs == NS) fs = 0;
+        issue();   // this thread has consumed its lanes of the stage: refill it NS steps ahead
+    };
+
+    fetch();
+    float h[LPT];
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+    int i = 0;                                   // step within the plane
+    long long poff = (long long)blockIdx.x * HW;
+    int plane = (int)blockIdx.x;
+    for (long long g = 0; g < total; ++g) {
+        float cz[LPT], cacc[LPT], cu[LPT], cw0[LPT], cw2[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            cz[e] = nz[e]; cacc[e] = nacc[e]; cu[e] = nu[e]; cw0[e] = nw0[e]; cw2[e] = nw2[e];
+            if (i == 0) h[e] = 0.f;
+        }
+        // neighbours from the previous step: lane j0-1 and lane j0+LPT
+        const float* hprev = halo + ((g + 1) & 1) * 64;
+        float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
+        float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
+        const float edge = lane == 0 ? hprev[32 + warp - 1 + (warp == 0)] : hprev[warp + 1 - (warp == nw - 1)];
+        if (lane == 0) hl = warp > 0 ? edge : 0.f;
+        if (lane == 31) hr = warp < nw - 1 ? edge : 0.f;
+        float hn[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) hn[e] = 0.f;
+        if (active) {
+#pragma unroll
+            for (int e = 0; e < LPT; ++e) {
+                hn[e] = cz[e];
+                if (i > 0) {
                     const float left = e == 0 ? hl : h[e - 1];
-                    const float right = e == 3 ? hr : h[e + 1];
-                    hn[e] = fmaf(w0, left, fmaf(w1, h[e], fmaf(w2, right, hn[e])));
+                    const float right = e == LPT - 1 ? hr : h[e + 1];
+                    const float w1 = 1.f - cw0[e] - cw2[e];
+                    hn[e] = fmaf(cw0[e], left, fmaf(w1, h[e], fmaf(cw2[e], right, hn[e])));
                 }
             }
-            const int plane = (int)blockIdx.x + k * (int)gridDim.x;
             const int r = DIR == kTB ? i : H - 1 - i;
-            const long long off = (long long)plane * HW + (long long)r * W + j0;
-            int t = Md::XL ? 5 : 4;
-            float acc[4];
-            if (Md::ACCIN) {
-                V4<T>::ld(st + (t++) * rowB, acc);
+            const long long off = poff + (long long)r * W + j0;
+            float o[LPT];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[e] += hn[e];
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[e] = hn[e];
+            for (int e = 0; e < LPT; ++e) {
+                o[e] = Md::ACCIN ? cacc[e] + hn[e] : hn[e];
+                if (Md::FINAL) o[e] *= cu[e];
             }
-            if (Md::FINAL) {
-                float uu[4];
-                V4<T>::ld(st + (t++) * rowB, uu);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) uu[e] *= acc[e];
-                V4<T>::st((T*)p.y + off, uu);
-            } else {
-                V4<T>::st((T*)p.acc + off, acc);
-            }
-            if (Md::ZOUT) V4<T>::st((T*)p.z + off, zz);
+            st_lanes<T, LPT>((T*)(Md::FINAL ? p.y : p.acc) + off, o);
+            if (Md::ZOUT) st_lanes<T, LPT>((T*)p.z + off, cz);
         }
         float* hcur = halo + (g & 1) * 64;
         if (lane == 0) hcur[warp] = hn[0];
-        if (lane == 31) hcur[32 + warp] = hn[3];
-        const bool any_fail = bar_red_or(1, blockDim.x, !ok);
+        if (lane == 31) hcur[32 + warp] = hn[LPT - 1];
+        if (g + 1 < total) fetch();
+        __syncthreads();
 #pragma unroll
-        for (int e = 0; e < 4; ++e) h[e] = hn[e];
-        if (any_fail) { failed = true; break; }
-        if (tid == 0 && g + NS < total) issue(g + NS);
+        for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+        if (++i == H) {
+            i = 0;
+            plane += (int)gridDim.x;
+            poff = (long long)plane * HW;
+        }
     }
-    if (failed && tid == 0) {
-        // drain the copies still in flight before the CTA's shared memory is released
-        for (long long q = g + 1; q < total && q < g + NS; ++q)
-            mbar_wait_bounded(&full[q % NS], (uint32_t)((q / NS) & 1), p.limit_ns, p.status);
-    }
+    cp_async_wait<0>();
 }
 
 // ================================================================== horizontal sweep
-struct HMaps {
-    CUtensorMap a, src0, src1, acc, u;   // src0/src1 = x/lam, or z/-
-};
+__device__ __forceinline__ float u4_get(const uint4& r, int c) {
+    return __uint_as_float(c == 0 ? r.x : c == 1 ? r.y : c == 2 ? r.z : r.w);
+}
 
-// CTA = one plane at a time. blockDim T = min(512, H rounded up to 32); thread t owns rows
-// t + T*g for g < G. Stage = one column tile [Hpad rows x 16 bytes] of each input tensor.
-template <typename T, unsigned DIR, int MODE, int G>
-__global__ void __launch_bounds__(512, 1) k_hsweep(SweepArgs p, const __grid_constant__ HMaps maps, int box_rows,
-                                                   int nbox) {
+// CTA = one plane at a time. Thread t owns rows t + T*g for g < G. Ring of NS column tiles; a
+// tile holds, for every row, S steps: 16 bytes of each storage-dtype input and S*4 bytes of each
+// fp32 weight row (WC = S/4 chunks of 16 bytes), laid out [slot][row][16 B] so that
+// consecutive threads read consecutive 16-byte chunks.
+template <typename T, unsigned DIR, int MODE, int G, int NS>
+__global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsweep(SweepArgs p, int Hpad) {
     using Md = ModeT<MODE>;
     using SG = Seg<T>;
     constexpr int NTEN = Md::NTEN;
     constexpr int S = SG::S;
+    constexpr int WC = S / 4;                             // 16-byte chunks per weight row segment
+    constexpr int NSLOT = 2 * WC + NTEN;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align128(smem_raw);
-    const int H = p.H, W = p.W, NS = p.ns;
-    const int Hpad = box_rows * nbox;
-    const int tenB = Hpad * 16;
-    const int stageB = NTEN * tenB;
-    unsigned char* stages = smem;
-    float* halo = (float*)(smem + (size_t)NS * stageB);    // [2 parity][2 lo/hi][G][16 warps]
-    uint64_t* full = (uint64_t*)(halo + 2 * 2 * G * 16);
+    const int H = p.H, W = p.W;
+    const int slotB = Hpad * 16;
+    const int stageB = NSLOT * slotB;
+    float* halo = (float*)(smem + (size_t)NS * stageB);    // [2 parity][2 lo/hi][G][32 warps]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int T_ = blockDim.x;
     const long long HW = (long long)H * W;
-    const int nb = (W + S - 1) / S;                       // column tiles per plane
+    const int nb = W / S;                                 // column tiles per plane (W % S == 0)
     const int nplanes = p.N * p.C;
     const int my_planes = (nplanes - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const long long total = (long long)my_planes * nb;
 
-    if (tid == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    auto issue = [&](long long tg) {
-        const int k = (int)(tg / nb), bt = (int)(tg % nb);
-        const int b = DIR == kLR ? bt : nb - 1 - bt;
-        const int plane = (int)blockIdx.x + k * (int)gridDim.x;
-        const int n = plane / p.C, c = plane % p.C;
-        unsigned char* st = stages + (size_t)(tg % NS) * stageB;
-        uint64_t* bar = &full[tg % NS];
-        mbar_arrive_expect_tx(bar, (uint32_t)stageB);
-        const int x0 = b * S;
-        const int arow = (int)((((long long)p.slot * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * H);
-        const int prow = plane * H;
-        for (int bx = 0; bx < nbox; ++bx) {
-            const int ro = bx * box_rows;
-            unsigned char* d = st + (size_t)ro * 16;
-            tma_load_2d(d, &maps.a, x0, arow + ro, bar);
-            tma_load_2d(d + tenB, &maps.a, x0, arow + H + ro, bar);
-            tma_load_2d(d + 2 * tenB, &maps.a, x0, arow + 2 * H + ro, bar);
-            int t = 3;
-            tma_load_2d(d + (t++) * tenB, &maps.src0, x0, prow + ro, bar);
-            if (Md::XL) tma_load_2d(d + (t++) * tenB, &maps.src1, x0, prow + ro, bar);
-            if (Md::ACCIN) tma_load_2d(d + (t++) * tenB, &maps.acc, x0, prow + ro, bar);
-            if (Md::FINAL) tma_load_2d(d + (t++) * tenB, &maps.u, x0, prow + ro, bar);
-        }
+    // Issue cursor (per thread): tiles are requested strictly in order.
+    long long iss_left = total;
+    int iss_bt = 0, iss_s = 0, iss_plane = (int)blockIdx.x;
+    const float* iss_wt = nullptr;
+    long long iss_poff = 0;
+    auto iss_plane_setup = [&]() {
+        const int n = iss_plane / p.C, c = iss_plane % p.C;
+        iss_wt = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
+        iss_poff = (long long)iss_plane * HW;
     };
-    if (tid == 0)
-        for (long long q = 0; q < NS && q < total; ++q) issue(q);
+    auto issue = [&]() {
+        if (iss_left > 0) {
+            const int b = DIR == kLR ? iss_bt : nb - 1 - iss_bt;
+            unsigned char* st = smem + (size_t)iss_s * stageB;
+#pragma unroll
+            for (int gg = 0; gg < G; ++gg) {
+                const int row = tid + T_ * gg;
+                if (row < H) {
+                    const long long ro = (long long)row * W + (long long)b * S;
+                    unsigned char* d = st + (size_t)row * 16;
+#pragma unroll
+                    for (int k = 0; k < WC; ++k) {
+                        cp_async<16>(d + k * slotB, iss_wt + ro + 4 * k);
+                        cp_async<16>(d + (WC + k) * slotB, iss_wt + HW + ro + 4 * k);
+                    }
+                    const long long off = iss_poff + ro;
+                    unsigned char* dt = d + 2 * WC * slotB;
+                    int t = 0;
+                    if (Md::XL) {
+                        cp_async<16>(dt + (t++) * slotB, (const T*)p.x + off);
+                        cp_async<16>(dt + (t++) * slotB, (const T*)p.lam + off);
+                    } else {
+                        cp_async<16>(dt + (t++) * slotB, (const T*)p.z + off);
+                    }
+                    if (Md::ACCIN) cp_async<16>(dt + (t++) * slotB, (const T*)p.acc + off);
+                    if (Md::FINAL) cp_async<16>(dt + (t++) * slotB, (const T*)p.u + off);
+                }
+            }
+            --iss_left;
+            if (++iss_s == NS) iss_s = 0;
+            if (++iss_bt == nb) {
+                iss_bt = 0;
+                iss_plane += (int)gridDim.x;
+                if (iss_plane < nplanes) iss_plane_setup();
+            }
+        }
+        cp_async_commit();
+    };
+    iss_plane_setup();
+#pragma unroll
+    for (int q = 0; q < NS; ++q) issue();
 
     float h[G];
 #pragma unroll
     for (int gg = 0; gg < G; ++gg) h[gg] = 0.f;
-    long long tg = 0;
     long long gstep = 0;   // global step counter (halo parity)
-    bool failed = false;
-    for (; tg < total; ++tg) {
-        const int k = (int)(tg / nb), bt = (int)(tg % nb);
+    int bt = 0, cs = 0;    // tile within plane, consumer stage
+    long long poff = (long long)blockIdx.x * HW;
+    int plane = (int)blockIdx.x;
+    for (long long tg = 0; tg < total; ++tg) {
         const int b = DIR == kLR ? bt : nb - 1 - bt;
         if (bt == 0) {
 #pragma unroll
             for (int gg = 0; gg < G; ++gg) h[gg] = 0.f;
         }
-        const int s = (int)(tg % NS);
-        const bool ok = mbar_wait_bounded(&full[s], (uint32_t)((tg / NS) & 1), p.limit_ns, p.status);
-        // pull this thread's rows of the tile into registers
-        uint4 ra0[G], ra1[G], ra2[G], rs0[G], rs1[G], racc[G], ru[G], out0[G], out1[G];
-        const unsigned char* st = stages + (size_t)s * stageB;
+        // pull this thread's rows of the tile into registers, then refill the stage
+        cp_async_wait<NS - 1>();
+        uint4 rw0[G][WC], rw2[G][WC], rs0[G], rs1[G], racc[G], ru[G], out0[G], out1[G];
+        const unsigned char* st = smem + (size_t)cs * stageB;
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
             const int row = tid + T_ * gg;
             const size_t o = (size_t)row * 16;
+#pragma unroll
+            for (int k = 0; k < WC; ++k) rw0[gg][k] = rw2[gg][k] = make_uint4(0, 0, 0, 0);
+            rs0[gg] = rs1[gg] = racc[gg] = ru[gg] = make_uint4(0, 0, 0, 0);
             if (row < H) {
-                ra0[gg] = *(const uint4*)(st + o);
-                ra1[gg] = *(const uint4*)(st + tenB + o);
-                ra2[gg] = *(const uint4*)(st + 2 * tenB + o);
-                int t = 3;
-                rs0[gg] = *(const uint4*)(st + (t++) * tenB + o);
-                if (Md::XL) rs1[gg] = *(const uint4*)(st + (t++) * tenB + o);
-                if (Md::ACCIN) racc[gg] = *(const uint4*)(st + (t++) * tenB + o);
-                if (Md::FINAL) ru[gg] = *(const uint4*)(st + (t++) * tenB + o);
+#pragma unroll
+                for (int k = 0; k < WC; ++k) {
+                    rw0[gg][k] = *(const uint4*)(st + k * slotB + o);
+                    rw2[gg][k] = *(const uint4*)(st + (WC + k) * slotB + o);
+                }
+                const unsigned char* dt = st + 2 * WC * slotB + o;
+                int t = 0;
+                rs0[gg] = *(const uint4*)(dt + (t++) * slotB);
+                if (Md::XL) rs1[gg] = *(const uint4*)(dt + (t++) * slotB);
+                if (Md::ACCIN) racc[gg] = *(const uint4*)(dt + (t++) * slotB);
+                if (Md::FINAL) ru[gg] = *(const uint4*)(dt + (t++) * slotB);
             }
             out0[gg] = make_uint4(0, 0, 0, 0);
             out1[gg] = make_uint4(0, 0, 0, 0);
         }
-        const int plane = (int)blockIdx.x + k * (int)gridDim.x;
+        if (++cs == NS) cs = 0;
+        issue();
 #pragma unroll
         for (int sj = 0; sj < S; ++sj) {
             const int sl = DIR == kLR ? sj : S - 1 - sj;     // segment slot (column b*S + sl)
             const int col = b * S + sl;
-            const bool valid = col < W;                      // uniform across the CTA
             const int i = DIR == kLR ? col : W - 1 - col;    // scan step
-            const float* hprev = halo + ((gstep + 1) & 1) * (2 * G * 16);
+            const float* hprev = halo + ((gstep + 1) & 1) * (2 * G * 32);
             float hn[G];
 #pragma unroll
             for (int gg = 0; gg < G; ++gg) {
                 const int row = tid + T_ * gg;
                 float hl = __shfl_up_sync(0xffffffffu, h[gg], 1);
                 float hr = __shfl_down_sync(0xffffffffu, h[gg], 1);
-                if (lane == 0) {
-                    if (warp > 0) hl = hprev[G * 16 + gg * 16 + warp - 1];
-                    else hl = gg > 0 ? hprev[G * 16 + (gg - 1) * 16 + nw - 1] : 0.f;
-                }
-                if (lane == 31) {
-                    if (warp < nw - 1) hr = hprev[gg * 16 + warp + 1];
-                    else hr = gg < G - 1 ? hprev[(gg + 1) * 16] : 0.f;
-                }
+                // edge lanes take the neighbour warp's value (or the previous / next row group's)
+                const int il = warp > 0 ? G * 32 + gg * 32 + warp - 1 : G * 32 + (gg > 0 ? gg - 1 : 0) * 32 + nw - 1;
+                const int ir = warp < nw - 1 ? gg * 32 + warp + 1 : (gg < G - 1 ? gg + 1 : gg) * 32;
+                const float eh = hprev[lane == 0 ? il : ir];
+                if (lane == 0) hl = (warp > 0 || gg > 0) ? eh : 0.f;
+                if (lane == 31) hr = (warp < nw - 1 || gg < G - 1) ? eh : 0.f;
                 float v = 0.f;
-                if (valid && row < H) {
+                if (row < H) {
                     float zz = SG::get(rs0[gg], sl);
                     if (Md::XL) zz *= SG::get(rs1[gg], sl);
                     v = zz;
                     if (i > 0) {
-                        float w0, w1, w2;
-                        lane_weights(SG::get(ra0[gg], sl), SG::get(ra1[gg], sl), SG::get(ra2[gg], sl), row > 0,
-                                     row < H - 1, w0, w1, w2);
-                        v = fmaf(w0, hl, fmaf(w1, h[gg], fmaf(w2, hr, v)));
+                        const float w0 = u4_get(rw0[gg][sl >> 2], sl & 3);
+                        const float w2 = u4_get(rw2[gg][sl >> 2], sl & 3);
+                        v = fmaf(w0, hl, fmaf(1.f - w0 - w2, h[gg], fmaf(w2, hr, v)));
                     }
                     float accv = v;
                     if (Md::ACCIN) accv += SG::get(racc[gg], sl);
@@ -387,82 +572,39 @@ __global__ void __launch_bounds__(512, 1) k_hsweep(SweepArgs p, const __grid_con
                     else SG::put(out0[gg], sl, accv);
                     if (Md::ZOUT) SG::put(out1[gg], sl, zz);
                 }
-                hn[gg] = valid ? v : h[gg];
+                hn[gg] = v;
             }
-            float* hcur = halo + (gstep & 1) * (2 * G * 16);
+            float* hcur = halo + (gstep & 1) * (2 * G * 32);
 #pragma unroll
             for (int gg = 0; gg < G; ++gg) {
-                if (lane == 0) hcur[gg * 16 + warp] = hn[gg];
-                if (lane == 31) hcur[G * 16 + gg * 16 + warp] = hn[gg];
+                if (lane == 0) hcur[gg * 32 + warp] = hn[gg];
+                if (lane == 31) hcur[G * 32 + gg * 32 + warp] = hn[gg];
                 h[gg] = hn[gg];
             }
-            const bool any_fail = bar_red_or(1, blockDim.x, !ok);
+            __syncthreads();
             ++gstep;
-            if (any_fail) { failed = true; break; }
-            // every thread copied its rows of this stage into registers before the first
-            // barrier of the tile, so the stage can be refilled now
-            if (sj == 0 && tid == 0 && tg + NS < total) issue(tg + NS);
         }
-        if (failed) break;
         // write back the tile's outputs as 16-byte row segments
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
             const int row = tid + T_ * gg;
             if (row < H) {
-                const long long off = (long long)plane * HW + (long long)row * W + (long long)b * S;
-                const bool full_seg = (b + 1) * S <= W;
-                T* dst = Md::FINAL ? (T*)p.y : (T*)p.acc;
-                if (full_seg) {
-                    *(uint4*)(dst + off) = out0[gg];
-                    if (Md::ZOUT) *(uint4*)((T*)p.z + off) = out1[gg];
-                } else {
-                    for (int sl = 0; sl < W - b * S; ++sl) {
-                        Io<T>::st(dst + off + sl, SG::get(out0[gg], sl));
-                        if (Md::ZOUT) Io<T>::st((T*)p.z + off + sl, SG::get(out1[gg], sl));
-                    }
-                }
+                const long long off = poff + (long long)row * W + (long long)b * S;
+                *(uint4*)((T*)(Md::FINAL ? p.y : p.acc) + off) = out0[gg];
+                if (Md::ZOUT) *(uint4*)((T*)p.z + off) = out1[gg];
             }
         }
+        if (++bt == nb) {
+            bt = 0;
+            plane += (int)gridDim.x;
+            poff = (long long)plane * HW;
+        }
     }
-    if (failed && tid == 0) {
-        for (long long q = tg + 1; q < total && q < tg + NS; ++q)
-            mbar_wait_bounded(&full[q % NS], (uint32_t)((q / NS) & 1), p.limit_ns, p.status);
-    }
+    cp_async_wait<0>();
 }
 
 // ================================================================== host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (EncodeTiledFn)ptr;
-    }
-    return fn;
-}
-
-// 2D map over a [rows x W] row-major tensor with a box of [box_rows x 16 bytes].
-bool make_map(CUtensorMap* m, const void* base, int dtype, long long rows, int W, int box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const int es = dtype == GSPN_F32 ? 4 : 2;
-    cuuint64_t dims[2] = {(cuuint64_t)W, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)W * es};
-    cuuint32_t box[2] = {(cuuint32_t)(16 / es), (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, dtype == GSPN_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-constexpr int kSmemBudget = 225 * 1024;
+constexpr size_t kSmemBudget = 225 * 1024;
 
 int ntensors(int mode) {
     switch (mode) {
@@ -473,113 +615,152 @@ int ntensors(int mode) {
     }
 }
 
-int v_stages(const Problem& P, int mode) {
-    const size_t stageB = (size_t)ntensors(mode) * P.W * P.esize();
-    int ns = (int)((kSmemBudget - 1024) / stageB);
-    return std::min(ns, 4);
-}
-
-void h_geometry(const Problem& P, int* box_rows, int* nbox, int* threads, int* G) {
-    *box_rows = std::min(256, ((P.H + 7) / 8) * 8);
-    *nbox = (P.H + *box_rows - 1) / *box_rows;
-    *threads = std::min(512, ((P.H + 31) / 32) * 32);
-    *G = (*nbox * *box_rows + *threads - 1) / *threads;
-}
-
-int h_stages(const Problem& P, int mode) {
-    int br, nbox, thr, G;
-    h_geometry(P, &br, &nbox, &thr, &G);
-    const size_t stageB = (size_t)ntensors(mode) * br * nbox * 16;
-    int ns = (int)((kSmemBudget - 4096) / stageB);
-    return std::min(ns, 3);
-}
-
 int mode_of(int v, int D) {
     if (D == 1) return M_ONLY;
     if (v == 0) return M_FIRST;
     return v == D - 1 ? M_LAST : M_MID;
 }
 
-template <typename T, unsigned DIR, int MODE>
-cudaError_t launch_v(const Problem& P, SweepArgs a, cudaStream_t st) {
-    a.ns = v_stages(P, MODE);
-    const int threads = std::max(32, ((P.W / 4 + 31) / 32) * 32);
-    const size_t smem = 128 + (size_t)a.ns * ModeT<MODE>::NTEN * P.W * sizeof(T) + 128 * sizeof(float) + 8 * 8;
+// ---- vertical geometry: lanes per thread (8, or 4 when W is not a multiple of 8), ring depth
+int v_lanes(const Problem& P) {
+    int lpt = 8;
+    if (const char* e = getenv("GSPN_VLPT")) lpt = atoi(e) == 4 ? 4 : 8;
+    if (P.W % 8 != 0) lpt = 4;   // 8 lanes per thread only when every thread's lanes lie in the row
+    return lpt;
+}
+int v_threads(const Problem& P) { return std::max(32, ((P.W / v_lanes(P) + 31) / 32) * 32); }
+size_t v_smem(const Problem& P, int mode, int ns) {
+    return 128 + (size_t)ns * (2 * (size_t)P.W * 4 + (size_t)ntensors(mode) * P.W * P.esize()) + 512;
+}
+int v_stages(const Problem& P, int mode) {
+    if (v_smem(P, mode, 4) <= kSmemBudget) return 4;
+    return v_smem(P, mode, 2) <= kSmemBudget ? 2 : 0;
+}
+
+// ---- horizontal geometry: threads, rows per thread (as instantiated), padded rows, ring depth
+int h_pref_rows() {
+    if (const char* e = getenv("GSPN_HROWS")) {
+        const int g = atoi(e);
+        if (g == 1 || g == 2 || g == 4) return g;
+    }
+    return 1;
+}
+int h_threads(const Problem& P) {
+    const int t = ((P.H + h_pref_rows() - 1) / h_pref_rows() + 31) / 32 * 32;
+    return std::min(1024, std::max(t, ((P.H + 3) / 4 + 31) / 32 * 32));
+}
+// Rows per thread as instantiated (1, 2 or 4): the kernel's halo and the shared-memory size
+// below are both laid out for this value, never for the raw quotient.
+int h_rows(const Problem& P) {
+    const int g = (P.H + h_threads(P) - 1) / h_threads(P);
+    return g <= 1 ? 1 : (g <= 2 ? 2 : 4);
+}
+int h_pad(const Problem& P) { return ((P.H + 7) / 8) * 8; }
+int h_slots(const Problem& P, int mode) { return 2 * ((16 / P.esize()) / 4) + ntensors(mode); }
+size_t h_smem(const Problem& P, int mode, int ns) {
+    return 128 + (size_t)ns * h_slots(P, mode) * h_pad(P) * 16 + 2 * 2 * h_rows(P) * 32 * sizeof(float);
+}
+int h_stages(const Problem& P, int mode) {
+    if (h_smem(P, mode, 4) <= kSmemBudget) return 4;
+    return h_smem(P, mode, 2) <= kSmemBudget ? 2 : 0;
+}
+
+template <typename T, unsigned DIR, int MODE, int LPT, int NS>
+cudaError_t launch_v4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    const size_t smem = v_smem(P, MODE, NS);
     const int grid = std::min(P.N * P.C, device_sm_count());
-    cudaFuncSetAttribute(k_vsweep<T, DIR, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_vsweep<T, DIR, MODE, LPT, NS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     launch_begin(st);
-    k_vsweep<T, DIR, MODE><<<grid, threads, smem, st>>>(a);
+    k_vsweep<T, DIR, MODE, LPT, NS><<<grid, v_threads(P), smem, st>>>(a);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+template <typename T, unsigned DIR, int MODE, int LPT>
+cudaError_t launch_v3(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    return v_stages(P, MODE) == 4 ? launch_v4<T, DIR, MODE, LPT, 4>(P, a, st)
+                                  : launch_v4<T, DIR, MODE, LPT, 2>(P, a, st);
+}
+
+template <typename T, unsigned DIR, int MODE>
+cudaError_t launch_v(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    return v_lanes(P) == 4 ? launch_v3<T, DIR, MODE, 4>(P, a, st) : launch_v3<T, DIR, MODE, 8>(P, a, st);
+}
+
+template <typename T, unsigned DIR, int MODE, int G, int NS>
+cudaError_t launch_h4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    const size_t smem = h_smem(P, MODE, NS);
+    const int grid = std::min(P.N * P.C, device_sm_count());
+    cudaError_t e = cudaFuncSetAttribute(k_hsweep<T, DIR, MODE, G, NS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    launch_begin(st);
+    k_hsweep<T, DIR, MODE, G, NS><<<grid, h_threads(P), smem, st>>>(a, h_pad(P));
     launch_end(st);
     return cudaGetLastError();
 }
 
 template <typename T, unsigned DIR, int MODE, int G>
-cudaError_t launch_h_g(const Problem& P, SweepArgs a, const HMaps& maps, int br, int nbox, int threads,
-                       cudaStream_t st) {
-    a.ns = h_stages(P, MODE);
-    const size_t smem = 128 + (size_t)a.ns * ModeT<MODE>::NTEN * br * nbox * 16 + 2 * 2 * G * 16 * sizeof(float) + 8 * 8;
-    const int grid = std::min(P.N * P.C, device_sm_count());
-    cudaFuncSetAttribute(k_hsweep<T, DIR, MODE, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    launch_begin(st);
-    k_hsweep<T, DIR, MODE, G><<<grid, threads, smem, st>>>(a, maps, br, nbox);
-    launch_end(st);
-    return cudaGetLastError();
+cudaError_t launch_h3(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    return h_stages(P, MODE) == 4 ? launch_h4<T, DIR, MODE, G, 4>(P, a, st)
+                                  : launch_h4<T, DIR, MODE, G, 2>(P, a, st);
 }
 
 template <typename T, unsigned DIR, int MODE>
-cudaError_t launch_h(const Problem& P, SweepArgs a, const HMaps& maps, cudaStream_t st) {
-    int br, nbox, threads, G;
-    h_geometry(P, &br, &nbox, &threads, &G);
-    switch (G) {
-    case 1: return launch_h_g<T, DIR, MODE, 1>(P, a, maps, br, nbox, threads, st);
-    case 2: return launch_h_g<T, DIR, MODE, 2>(P, a, maps, br, nbox, threads, st);
-    default: return cudaErrorNotSupported;
+cudaError_t launch_h(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    switch (h_rows(P)) {
+    case 1: return launch_h3<T, DIR, MODE, 1>(P, a, st);
+    case 2: return launch_h3<T, DIR, MODE, 2>(P, a, st);
+    default: return launch_h3<T, DIR, MODE, 4>(P, a, st);
     }
 }
 
 template <typename T, unsigned DIR>
-cudaError_t launch_dir(const Problem& P, SweepArgs a, int mode, const HMaps* maps, cudaStream_t st) {
-    const bool vert = DIR == kTB || DIR == kBT;
+cudaError_t launch_dir(const Problem& P, const SweepArgs& a, int mode, cudaStream_t st) {
+    constexpr bool vert = DIR == kTB || DIR == kBT;
     switch (mode) {
-    case M_FIRST: return vert ? launch_v<T, DIR, M_FIRST>(P, a, st) : launch_h<T, DIR, M_FIRST>(P, a, *maps, st);
-    case M_ONLY: return vert ? launch_v<T, DIR, M_ONLY>(P, a, st) : launch_h<T, DIR, M_ONLY>(P, a, *maps, st);
-    case M_MID: return vert ? launch_v<T, DIR, M_MID>(P, a, st) : launch_h<T, DIR, M_MID>(P, a, *maps, st);
-    default: return vert ? launch_v<T, DIR, M_LAST>(P, a, st) : launch_h<T, DIR, M_LAST>(P, a, *maps, st);
+    case M_FIRST: return vert ? launch_v<T, DIR, M_FIRST>(P, a, st) : launch_h<T, DIR, M_FIRST>(P, a, st);
+    case M_ONLY: return vert ? launch_v<T, DIR, M_ONLY>(P, a, st) : launch_h<T, DIR, M_ONLY>(P, a, st);
+    case M_MID: return vert ? launch_v<T, DIR, M_MID>(P, a, st) : launch_h<T, DIR, M_MID>(P, a, st);
+    default: return vert ? launch_v<T, DIR, M_LAST>(P, a, st) : launch_h<T, DIR, M_LAST>(P, a, st);
     }
 }
+
+size_t table_floats(const Problem& P) { return (size_t)P.D * P.N * P.Cw * 2 * (size_t)P.HW; }
 
 template <typename T>
 cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
                             void* ws, cudaStream_t st) {
     WsCarver wc(ws);
+    float* table = wc.take<float>(table_floats(P));
     void* z = P.D > 1 ? wc.take<T>(P.U) : nullptr;
     void* acc = P.D > 1 ? wc.take<T>(P.U) : nullptr;
-    SweepArgs args{x, lam, u, a, z, acc, y, P.N, P.C, P.H, P.W, P.Cw, 0, 2, (unsigned*)ws, kWaitLimitNs};
+    // A1: weight formation for every direction, once per (n, cw) plane
+    WeightArgs wa{a, table, P.N, P.Cw, P.H, P.W, P.D, {0u, 0u, 0u, 0u}};
+    for (int v = 0, k = 0; k < 4; ++k)
+        if (P.mask & (1u << k)) wa.dirs[v++] = 1u << k;
+    const int quads = (int)(P.HW / 4);
+    const dim3 wgrid((unsigned)std::max(1, std::min((quads + 255) / 256, 64)), (unsigned)(P.D * P.N * P.Cw));
+    launch_begin(st);
+    k_sweep_weights<T><<<wgrid, 256, 0, st>>>(wa);
+    launch_end(st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // A2-A6: one sweep per direction
+    SweepArgs args{x, lam, u, nullptr, z, acc, y, P.N, P.C, P.H, P.W, P.Cw};
+    const size_t slot_floats = (size_t)P.N * P.Cw * 2 * (size_t)P.HW;
     int v = 0;
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
         const int mode = mode_of(v, P.D);
-        args.slot = v;
-        HMaps maps;
-        if (!is_vertical(d)) {
-            int br, nbox, thr, G;
-            h_geometry(P, &br, &nbox, &thr, &G);
-            const long long prow = (long long)P.N * P.C * P.H;
-            const long long arow = (long long)P.D * P.N * P.Cw * 3 * P.H;
-            const bool xl = mode == M_FIRST || mode == M_ONLY;
-            bool ok = make_map(&maps.a, a, P.dtype, arow, P.W, br);
-            ok = ok && make_map(&maps.src0, xl ? x : z, P.dtype, prow, P.W, br);
-            ok = ok && make_map(&maps.src1, xl ? lam : x, P.dtype, prow, P.W, br);
-            ok = ok && make_map(&maps.acc, acc ? acc : x, P.dtype, prow, P.W, br);
-            ok = ok && make_map(&maps.u, u, P.dtype, prow, P.W, br);
-            if (!ok) return cudaErrorInvalidValue;
-        }
-        cudaError_t e;
+        args.wt = table + v * slot_floats;
         switch (d) {
-        case kTB: e = launch_dir<T, kTB>(P, args, mode, nullptr, st); break;
-        case kBT: e = launch_dir<T, kBT>(P, args, mode, nullptr, st); break;
-        case kLR: e = launch_dir<T, kLR>(P, args, mode, &maps, st); break;
-        default: e = launch_dir<T, kRL>(P, args, mode, &maps, st); break;
+        case kTB: e = launch_dir<T, kTB>(P, args, mode, st); break;
+        case kBT: e = launch_dir<T, kBT>(P, args, mode, st); break;
+        case kLR: e = launch_dir<T, kLR>(P, args, mode, st); break;
+        default: e = launch_dir<T, kRL>(P, args, mode, st); break;
         }
         if (e != cudaSuccess) return e;
         ++v;
@@ -591,21 +772,21 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
 
 bool sweep_supports(const Problem& P, bool bwd) {
     if (bwd) return false;
-    if ((P.W * P.esize()) % 16 != 0) return false;
+    if ((P.W * P.esize()) % 16 != 0) return false;   // 16-byte rows and column tiles
     if (P.W > 4096 || P.H > 1024) return false;
-    // TMA row coordinates are 32-bit
-    if ((long long)P.D * P.N * P.Cw * 3 * P.H >= (1LL << 31) || (long long)P.N * P.C * P.H >= (1LL << 31)) return false;
-    if (!encode_fn()) return false;
-    for (int mode = 0; mode < 4; ++mode) {
-        if ((P.mask & (kTB | kBT)) && v_stages(P, mode) < 2) return false;
-        if ((P.mask & (kLR | kRL)) && h_stages(P, mode) < 2) return false;
+    if ((long long)P.D * P.N * P.Cw > 65535) return false;   // weight-formation grid.y
+    for (int v = 0, k = 0; k < 4; ++k) {
+        const unsigned d = 1u << k;
+        if (!(P.mask & d)) continue;
+        const int mode = mode_of(v++, P.D);
+        if (is_vertical(d) ? v_stages(P, mode) == 0 : h_stages(P, mode) == 0) return false;
     }
     return true;
 }
 
 size_t sweep_ws_bytes(const Problem& P, bool bwd) {
     if (bwd) return 0;
-    size_t b = 256;
+    size_t b = 256 + align256(table_floats(P) * sizeof(float));
     if (P.D > 1) b += 2 * align256((size_t)P.U * P.esize());
     return b;
 }
