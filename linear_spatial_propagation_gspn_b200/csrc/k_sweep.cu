@@ -33,30 +33,43 @@ namespace {
 
 enum { M_FIRST = 0, M_ONLY = 1, M_MID = 2, M_LAST = 3 };
 
-template <int MODE> struct ModeT {
+// TOUT: outputs leave through a shared-memory staging block and are written lane-major
+// (transposed); a final sweep then applies u while flushing, so u is not in the ring.
+template <int MODE, bool TOUT = false> struct ModeT {
     static constexpr bool XL = MODE == M_FIRST || MODE == M_ONLY;     // read x, lam (else z)
     static constexpr bool ACCIN = MODE == M_MID || MODE == M_LAST;    // read the partial sum
     static constexpr bool FINAL = MODE == M_ONLY || MODE == M_LAST;   // read u, write y
-    static constexpr bool ZOUT = MODE == M_FIRST;                     // write z
+    static constexpr bool ZOUT = MODE == M_FIRST || (TOUT && !FINAL); // write z (z^T when TOUT)
+    static constexpr bool URING = FINAL && !TOUT;                     // u comes through the ring
     // storage-dtype tensors per stage: x lam | z, [acc], [u]  (plus the two fp32 weight rows)
-    static constexpr int NTEN = (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (FINAL ? 1 : 0);
+    static constexpr int NTEN = (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (URING ? 1 : 0);
+    // staged outputs when TOUT: z and acc, or the unscaled sum for a final sweep
+    static constexpr int NSTG = TOUT ? (FINAL ? 1 : 2) : 0;
 };
 
+// Steps per staging block of a transposed-output sweep (64 bytes of fp32 per lane).
+constexpr int kTB_STEPS = 16;
+
+// Sweep arguments in scan coordinates: H = scan length (steps), W = lanes. A horizontal scan
+// over transposed buffers passes (H, W) = (image width, image height).
 struct SweepArgs {
     const void* x;
     const void* lam;
-    const void* u;
+    const void* u;    // scan-major, or lane-major (image layout) for a transposed-output final sweep
     const float* wt;  // weight table of this direction's slot: [N][Cw][2][H][W] fp32 (w0, w2)
-    void* z;          // workspace, storage dtype
-    void* acc;        // workspace, storage dtype
-    void* y;
+    void* z;          // workspace, storage dtype, scan-major
+    void* acc;        // workspace, storage dtype, scan-major
+    void* y;          // output (scan-major, or lane-major when TOUT)
+    void* zt;         // lane-major z   (TOUT, non-final)
+    void* acct;       // lane-major acc (TOUT, non-final)
     int N, C, H, W, Cw;
 };
 
 struct WeightArgs {
     const void* a;    // logits [D][N][Cw][3][H][W]
-    float* wt;        // table  [D][N][Cw][2][H][W]
+    float* wt;        // table  [D][N][Cw][2][H][W] (transposed planes: [W][H])
     int N, Cw, H, W, D;
+    int plane0;       // first (slot, n, cw) plane handled by the launch
     unsigned dirs[4]; // direction bit of each slot
 };
 
@@ -224,7 +237,7 @@ __device__ __forceinline__ void read_lanes(const unsigned char* srcs, float (&v)
 template <typename T>
 __global__ void __launch_bounds__(256) k_sweep_weights(WeightArgs p) {
     const long long HW = (long long)p.H * p.W;
-    const int plane = blockIdx.y;                      // (slot, n, cw)
+    const int plane = p.plane0 + (int)blockIdx.y;      // (slot, n, cw)
     const int slot = plane / (p.N * p.Cw);
     const unsigned d = p.dirs[slot];
     const T* a3 = (const T*)p.a + (long long)plane * 3 * HW;
@@ -251,15 +264,56 @@ __global__ void __launch_bounds__(256) k_sweep_weights(WeightArgs p) {
     }
 }
 
+// Same table, written transposed ([W][H] per plane: element (column c, row r) at c*H + r) for
+// horizontal scans run over transposed buffers. 32x32 pixel tiles through shared memory keep
+// both the logit reads and the table writes coalesced.
+template <typename T>
+__global__ void __launch_bounds__(256) k_sweep_weights_t(WeightArgs p) {
+    __shared__ float tile[2][32][33];
+    const long long HW = (long long)p.H * p.W;
+    const int plane = p.plane0 + (int)blockIdx.z;
+    const int slot = plane / (p.N * p.Cw);
+    const unsigned d = p.dirs[slot];
+    const T* a3 = (const T*)p.a + (long long)plane * 3 * HW;
+    float* wt = p.wt + (long long)plane * 2 * HW;
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int r = r0 + ty + 8 * k, c = c0 + tx;
+        float w0 = 0.f, w2 = 0.f;
+        if (r < p.H && c < p.W) {
+            const long long q = (long long)r * p.W + c;
+            const bool hl = is_vertical(d) ? c > 0 : r > 0;
+            const bool hr = is_vertical(d) ? c < p.W - 1 : r < p.H - 1;
+            const Wts w = lane_weights_acc(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q), Io<T>::ld(a3 + 2 * HW + q), hl, hr);
+            w0 = w.w0;
+            w2 = w.w2;
+        }
+        tile[0][ty + 8 * k][tx] = w0;
+        tile[1][ty + 8 * k][tx] = w2;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int c = c0 + ty + 8 * k, r = r0 + tx;
+        if (r < p.H && c < p.W) {
+            const long long q = (long long)c * p.H + r;
+            wt[q] = tile[0][tx][ty + 8 * k];
+            wt[HW + q] = tile[1][tx][ty + 8 * k];
+        }
+    }
+}
+
 // ================================================================== vertical sweep
 // CTA = one plane at a time (persistent over planes b, b + grid, ...); thread t owns lanes
 // [LPT t, LPT t + LPT). Ring of NS stages; a stage is one image row of the two fp32 weight
 // rows and of each storage-dtype input. Every thread keeps NS rows of its own lanes in flight.
 // The loop is software-pipelined by one step: while step g's new line is exchanged at the
 // barrier, every thread has already pulled step g+1's inputs out of the ring.
-template <typename T, unsigned DIR, int MODE, int LPT, int NS>
+template <typename T, unsigned DIR, int MODE, int LPT, int NS, bool TOUT>
 __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p) {
-    using Md = ModeT<MODE>;
+    using Md = ModeT<MODE, TOUT>;
     constexpr int NTEN = Md::NTEN;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align128(smem_raw);
@@ -268,6 +322,14 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
     const int wrowB = W * 4;
     const int stageB = 2 * wrowB + NTEN * rowB;
     float* halo = (float*)(smem + (size_t)NS * stageB);   // [2 parity][2 lo/hi][32 warps]
+    // TOUT staging: Md::NSTG blocks of [kTB_STEPS][R] fp32, row stride R = 4 (mod 32) so the
+    // column reads of the flush hit at most two lanes per bank.
+    float* stg = halo + 128;
+    const int R = ((W + 31) / 32) * 32 + 4;
+    // TOUT final: u of the next staging block, prefetched lane-major, 16 bytes per chunk id
+    constexpr int CH = 16 / (int)sizeof(T);          // steps per 16-byte chunk
+    constexpr int CPL = kTB_STEPS / CH;              // chunks per lane segment
+    uint4* ubuf = (uint4*)(stg + (size_t)Md::NSTG * kTB_STEPS * R);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int j0 = tid * LPT;
     const bool active = j0 < W;
@@ -308,7 +370,7 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
                     copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.z + off, sw);
                 }
                 if (Md::ACCIN) copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.acc + off, sw);
-                if (Md::FINAL) copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.u + off, sw);
+                if (Md::URING) copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.u + off, sw);
             }
             --iss_left;
             if (++iss_s == NS) iss_s = 0;
@@ -320,6 +382,22 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
         }
         cp_async_commit();   // always one group per call, so the wait counts stay uniform
     };
+    // Final transposed-output sweep: copy u of the staging block that contains scan row `row`
+    // of plane offset `po` into ubuf (same chunk ids as the flush). The copies join the ring's
+    // next commit group, which is complete at least kTB_STEPS - NS steps before the flush.
+    auto prefetch_u = [&](int row, long long po) {
+        if constexpr (TOUT && Md::FINAL) {
+            const int s_base = row - row % kTB_STEPS;
+            const int nvalid = min(kTB_STEPS, H - s_base);
+            const int q = tid % CPL, jstep = (int)blockDim.x / CPL;
+            if (q * CH < nvalid) {
+                const T* src = (const T*)p.u + po + (long long)(tid / CPL) * H + s_base + q * CH;
+                for (int j = tid / CPL; j < W; j += jstep, src += (long long)jstep * H)
+                    cp_async<16>(ubuf + j * CPL + q, src);
+            }
+        }
+    };
+    prefetch_u(DIR == kTB ? 0 : H - 1, (long long)blockIdx.x * HW);
     iss_plane_setup();
 #pragma unroll
     for (int q = 0; q < NS; ++q) issue();
@@ -345,7 +423,7 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
             }
             int t = Md::XL ? 2 : 1;
             if (Md::ACCIN) read_lanes<T, LPT>(sd + (t++) * rowB, nacc, sw);
-            if (Md::FINAL) read_lanes<T, LPT>(sd + (t++) * rowB, nu, sw);
+            if (Md::URING) read_lanes<T, LPT>(sd + (t++) * rowB, nu, sw);
         }
         if (++fs == NS) fs = 0;
         issue();   // this thread has consumed its lanes of the stage: refill it NS steps ahead
@@ -364,6 +442,14 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
         for (int e = 0; e < LPT; ++e) {
             cz[e] = nz[e]; cacc[e] = nacc[e]; cu[e] = nu[e]; cw0[e] = nw0[e]; cw2[e] = nw2[e];
             if (i == 0) h[e] = 0.f;
+        }
+        if constexpr (TOUT && Md::FINAL) {
+            // first step of a staging block (after the first): the previous block was flushed
+            // behind a barrier at the end of the last iteration, so ubuf is free. The copies
+            // join the commit group of this iteration's fetch.
+            const int rc = DIR == kTB ? i : H - 1 - i;
+            const bool starts = DIR == kTB ? rc % kTB_STEPS == 0 : (rc % kTB_STEPS == kTB_STEPS - 1 || rc == H - 1);
+            if (g > 0 && starts) prefetch_u(rc, poff);
         }
         // neighbours from the previous step: lane j0-1 and lane j0+LPT
         const float* hprev = halo + ((g + 1) & 1) * 64;
@@ -392,10 +478,20 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
 #pragma unroll
             for (int e = 0; e < LPT; ++e) {
                 o[e] = Md::ACCIN ? cacc[e] + hn[e] : hn[e];
-                if (Md::FINAL) o[e] *= cu[e];
+                if (Md::URING) o[e] *= cu[e];
             }
-            st_lanes<T, LPT>((T*)(Md::FINAL ? p.y : p.acc) + off, o);
-            if (Md::ZOUT) st_lanes<T, LPT>((T*)p.z + off, cz);
+            if constexpr (TOUT) {
+                float* srow = stg + (size_t)(r % kTB_STEPS) * R + j0;
+                if constexpr (Md::FINAL) {
+                    st_lanes<float, LPT>(srow, o);
+                } else {
+                    st_lanes<float, LPT>(srow, cz);
+                    st_lanes<float, LPT>(srow + kTB_STEPS * R, o);
+                }
+            } else {
+                st_lanes<T, LPT>((T*)(Md::FINAL ? p.y : p.acc) + off, o);
+                if (Md::ZOUT) st_lanes<T, LPT>((T*)p.z + off, cz);
+            }
         }
         float* hcur = halo + (g & 1) * 64;
         if (lane == 0) hcur[warp] = hn[0];
@@ -404,6 +500,56 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
         __syncthreads();
 #pragma unroll
         for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+        if constexpr (TOUT) {
+            // a staging block is complete: write it lane-major, 16 bytes per chunk
+            const int r = DIR == kTB ? i : H - 1 - i;
+            const bool flush = DIR == kTB ? (r % kTB_STEPS == kTB_STEPS - 1 || r == H - 1) : (r % kTB_STEPS == 0);
+            if (flush) {
+                const int s_base = r - r % kTB_STEPS;
+                const int nvalid = min(kTB_STEPS, H - s_base);
+                // The ring's waits already cover the u copies of a block longer than NS steps
+                // (issued with the block's first step); short blocks and the last step wait here.
+                if constexpr (Md::FINAL)
+                    if (nvalid <= NS || g + 1 >= total) cp_async_wait<0>();
+                // Thread t writes chunk q = t % CPL of lanes t / CPL, t / CPL + T / CPL, ...: a warp
+                // covers 32 / CPL whole lane segments per store; its shared reads are runs of
+                // consecutive lanes in CPL staging rows (R = 4 mod 32: at most two threads per bank).
+                const int q = tid % CPL, jstep = (int)blockDim.x / CPL;
+                if (q * CH < nvalid) {
+                    const long long gstep = (long long)jstep * H;
+                    const float* sp = stg + (size_t)(q * CH) * R + tid / CPL;
+                    const long long g0 = poff + (long long)(tid / CPL) * H + s_base + q * CH;
+                    if constexpr (Md::FINAL) {
+                        T* gp = (T*)p.y + g0;
+                        const uint4* up = ubuf + (tid / CPL) * CPL + q;
+#pragma unroll 4
+                        for (int j = tid / CPL; j < W; j += jstep, sp += jstep, gp += gstep, up += jstep * CPL) {
+                            float v[CH], uu[CH];
+                            ld_lanes<T, CH>(up, uu);
+#pragma unroll
+                            for (int k = 0; k < CH; ++k) v[k] = sp[k * R] * uu[k];
+                            st_lanes<T, CH>(gp, v);
+                        }
+                    } else {
+                        T* gz = (T*)p.zt + g0;
+                        T* ga = (T*)p.acct + g0;
+                        const size_t second = (size_t)kTB_STEPS * R;
+#pragma unroll 4
+                        for (int j = tid / CPL; j < W; j += jstep, sp += jstep, gz += gstep, ga += gstep) {
+                            float v[CH], va[CH];
+#pragma unroll
+                            for (int k = 0; k < CH; ++k) {
+                                v[k] = sp[k * R];
+                                va[k] = sp[second + k * R];
+                            }
+                            st_lanes<T, CH>(gz, v);
+                            st_lanes<T, CH>(ga, va);
+                        }
+                    }
+                }
+                __syncthreads();   // the staging block is reused by the next step
+            }
+        }
         if (++i == H) {
             i = 0;
             plane += (int)gridDim.x;
@@ -606,13 +752,17 @@ __global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsw
 // ================================================================== host side
 constexpr size_t kSmemBudget = 225 * 1024;
 
-int ntensors(int mode) {
+int ntensors(int mode, bool tout = false) {
     switch (mode) {
-    case M_FIRST: return ModeT<M_FIRST>::NTEN;
+    case M_FIRST: return tout ? ModeT<M_FIRST, true>::NTEN : ModeT<M_FIRST>::NTEN;
     case M_ONLY: return ModeT<M_ONLY>::NTEN;
-    case M_MID: return ModeT<M_MID>::NTEN;
-    default: return ModeT<M_LAST>::NTEN;
+    case M_MID: return tout ? ModeT<M_MID, true>::NTEN : ModeT<M_MID>::NTEN;
+    default: return tout ? ModeT<M_LAST, true>::NTEN : ModeT<M_LAST>::NTEN;
     }
+}
+int nstaged(int mode, bool tout) {
+    if (!tout) return 0;
+    return (mode == M_LAST || mode == M_ONLY) ? 1 : 2;
 }
 
 int mode_of(int v, int D) {
@@ -629,12 +779,16 @@ int v_lanes(const Problem& P) {
     return lpt;
 }
 int v_threads(const Problem& P) { return std::max(32, ((P.W / v_lanes(P) + 31) / 32) * 32); }
-size_t v_smem(const Problem& P, int mode, int ns) {
-    return 128 + (size_t)ns * (2 * (size_t)P.W * 4 + (size_t)ntensors(mode) * P.W * P.esize()) + 512;
+size_t v_smem(const Problem& P, int mode, int ns, bool tout) {
+    const size_t R = ((size_t)(P.W + 31) / 32) * 32 + 4;
+    const bool ubuf = tout && (mode == M_LAST || mode == M_ONLY);
+    return 128 + (size_t)ns * (2 * (size_t)P.W * 4 + (size_t)ntensors(mode, tout) * P.W * P.esize()) + 512 +
+           (size_t)nstaged(mode, tout) * kTB_STEPS * R * sizeof(float) +
+           (ubuf ? (size_t)P.W * kTB_STEPS * P.esize() : 0);
 }
-int v_stages(const Problem& P, int mode) {
-    if (v_smem(P, mode, 4) <= kSmemBudget) return 4;
-    return v_smem(P, mode, 2) <= kSmemBudget ? 2 : 0;
+int v_stages(const Problem& P, int mode, bool tout = false) {
+    if (v_smem(P, mode, 4, tout) <= kSmemBudget) return 4;
+    return v_smem(P, mode, 2, tout) <= kSmemBudget ? 2 : 0;
 }
 
 // ---- horizontal geometry: threads, rows per thread (as instantiated), padded rows, ring depth
@@ -665,28 +819,29 @@ int h_stages(const Problem& P, int mode) {
     return h_smem(P, mode, 2) <= kSmemBudget ? 2 : 0;
 }
 
-template <typename T, unsigned DIR, int MODE, int LPT, int NS>
+template <typename T, unsigned DIR, int MODE, bool TOUT, int LPT, int NS>
 cudaError_t launch_v4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
-    const size_t smem = v_smem(P, MODE, NS);
+    const size_t smem = v_smem(P, MODE, NS, TOUT);
     const int grid = std::min(P.N * P.C, device_sm_count());
-    cudaError_t e = cudaFuncSetAttribute(k_vsweep<T, DIR, MODE, LPT, NS>,
+    cudaError_t e = cudaFuncSetAttribute(k_vsweep<T, DIR, MODE, LPT, NS, TOUT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     launch_begin(st);
-    k_vsweep<T, DIR, MODE, LPT, NS><<<grid, v_threads(P), smem, st>>>(a);
+    k_vsweep<T, DIR, MODE, LPT, NS, TOUT><<<grid, v_threads(P), smem, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
 }
 
-template <typename T, unsigned DIR, int MODE, int LPT>
+template <typename T, unsigned DIR, int MODE, bool TOUT, int LPT>
 cudaError_t launch_v3(const Problem& P, const SweepArgs& a, cudaStream_t st) {
-    return v_stages(P, MODE) == 4 ? launch_v4<T, DIR, MODE, LPT, 4>(P, a, st)
-                                  : launch_v4<T, DIR, MODE, LPT, 2>(P, a, st);
+    return v_stages(P, MODE, TOUT) == 4 ? launch_v4<T, DIR, MODE, TOUT, LPT, 4>(P, a, st)
+                                        : launch_v4<T, DIR, MODE, TOUT, LPT, 2>(P, a, st);
 }
 
-template <typename T, unsigned DIR, int MODE>
+template <typename T, unsigned DIR, int MODE, bool TOUT = false>
 cudaError_t launch_v(const Problem& P, const SweepArgs& a, cudaStream_t st) {
-    return v_lanes(P) == 4 ? launch_v3<T, DIR, MODE, 4>(P, a, st) : launch_v3<T, DIR, MODE, 8>(P, a, st);
+    return v_lanes(P) == 4 ? launch_v3<T, DIR, MODE, TOUT, 4>(P, a, st)
+                           : launch_v3<T, DIR, MODE, TOUT, 8>(P, a, st);
 }
 
 template <typename T, unsigned DIR, int MODE, int G, int NS>
@@ -719,48 +874,105 @@ cudaError_t launch_h(const Problem& P, const SweepArgs& a, cudaStream_t st) {
 
 template <typename T, unsigned DIR>
 cudaError_t launch_dir(const Problem& P, const SweepArgs& a, int mode, cudaStream_t st) {
-    constexpr bool vert = DIR == kTB || DIR == kBT;
-    switch (mode) {
-    case M_FIRST: return vert ? launch_v<T, DIR, M_FIRST>(P, a, st) : launch_h<T, DIR, M_FIRST>(P, a, st);
-    case M_ONLY: return vert ? launch_v<T, DIR, M_ONLY>(P, a, st) : launch_h<T, DIR, M_ONLY>(P, a, st);
-    case M_MID: return vert ? launch_v<T, DIR, M_MID>(P, a, st) : launch_h<T, DIR, M_MID>(P, a, st);
-    default: return vert ? launch_v<T, DIR, M_LAST>(P, a, st) : launch_h<T, DIR, M_LAST>(P, a, st);
+    if constexpr (DIR == kTB || DIR == kBT) {
+        switch (mode) {
+        case M_FIRST: return launch_v<T, DIR, M_FIRST>(P, a, st);
+        case M_ONLY: return launch_v<T, DIR, M_ONLY>(P, a, st);
+        case M_MID: return launch_v<T, DIR, M_MID>(P, a, st);
+        default: return launch_v<T, DIR, M_LAST>(P, a, st);
+        }
+    } else {
+        switch (mode) {
+        case M_FIRST: return launch_h<T, DIR, M_FIRST>(P, a, st);
+        case M_ONLY: return launch_h<T, DIR, M_ONLY>(P, a, st);
+        case M_MID: return launch_h<T, DIR, M_MID>(P, a, st);
+        default: return launch_h<T, DIR, M_LAST>(P, a, st);
+        }
     }
 }
 
 size_t table_floats(const Problem& P) { return (size_t)P.D * P.N * P.Cw * 2 * (size_t)P.HW; }
 
+// The transposed path: when the mask has vertical and horizontal directions and both image
+// axes give 16-byte rows, the last vertical sweep writes z and the partial sum transposed and
+// the horizontal scans run as vertical-style sweeps over those transposed buffers.
+Problem swapped(const Problem& P) {
+    Problem Q = P;
+    std::swap(Q.H, Q.W);
+    return Q;
+}
+bool tpath(const Problem& P) {
+    return (P.mask & (kTB | kBT)) && (P.mask & (kLR | kRL)) && (P.H * P.esize()) % 16 == 0 &&
+           (P.W * P.esize()) % 16 == 0 && P.H <= 4096;
+}
+int n_vertical(const Problem& P) { return ((P.mask & kTB) ? 1 : 0) + ((P.mask & kBT) ? 1 : 0); }
+
+template <typename T, unsigned DIR>
+cudaError_t launch_vt(const Problem& P, const SweepArgs& a, int mode, bool tout, cudaStream_t st) {
+    if (!tout) return launch_dir<T, DIR>(P, a, mode, st);
+    switch (mode) {
+    case M_FIRST: return launch_v<T, DIR, M_FIRST, true>(P, a, st);
+    case M_MID: return launch_v<T, DIR, M_MID, true>(P, a, st);
+    case M_LAST: return launch_v<T, DIR, M_LAST, true>(P, a, st);
+    default: return cudaErrorNotSupported;
+    }
+}
+
 template <typename T>
 cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
                             void* ws, cudaStream_t st) {
+    const bool tp = tpath(P);
+    const int nV = n_vertical(P);
     WsCarver wc(ws);
     float* table = wc.take<float>(table_floats(P));
     void* z = P.D > 1 ? wc.take<T>(P.U) : nullptr;
     void* acc = P.D > 1 ? wc.take<T>(P.U) : nullptr;
+    void* zt = tp ? wc.take<T>(P.U) : nullptr;
+    void* acct = tp ? wc.take<T>(P.U) : nullptr;
     // A1: weight formation for every direction, once per (n, cw) plane
-    WeightArgs wa{a, table, P.N, P.Cw, P.H, P.W, P.D, {0u, 0u, 0u, 0u}};
+    WeightArgs wa{a, table, P.N, P.Cw, P.H, P.W, P.D, 0, {0u, 0u, 0u, 0u}};
     for (int v = 0, k = 0; k < 4; ++k)
         if (P.mask & (1u << k)) wa.dirs[v++] = 1u << k;
-    const int quads = (int)(P.HW / 4);
-    const dim3 wgrid((unsigned)std::max(1, std::min((quads + 255) / 256, 64)), (unsigned)(P.D * P.N * P.Cw));
-    launch_begin(st);
-    k_sweep_weights<T><<<wgrid, 256, 0, st>>>(wa);
-    launch_end(st);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    const int per_slot = P.N * P.Cw;
+    const int row_planes = (tp ? nV : P.D) * per_slot;
+    cudaError_t e;
+    if (row_planes > 0) {
+        const int quads = (int)(P.HW / 4);
+        const dim3 wgrid((unsigned)std::max(1, std::min((quads + 255) / 256, 64)), (unsigned)row_planes);
+        launch_begin(st);
+        k_sweep_weights<T><<<wgrid, 256, 0, st>>>(wa);
+        launch_end(st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (tp) {
+        wa.plane0 = nV * per_slot;
+        const dim3 tgrid((unsigned)((P.W + 31) / 32), (unsigned)((P.H + 31) / 32), (unsigned)((P.D - nV) * per_slot));
+        launch_begin(st);
+        k_sweep_weights_t<T><<<tgrid, 256, 0, st>>>(wa);
+        launch_end(st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     // A2-A6: one sweep per direction
-    SweepArgs args{x, lam, u, nullptr, z, acc, y, P.N, P.C, P.H, P.W, P.Cw};
-    const size_t slot_floats = (size_t)P.N * P.Cw * 2 * (size_t)P.HW;
+    const size_t slot_floats = (size_t)per_slot * 2 * (size_t)P.HW;
+    const Problem PS = swapped(P);
     int v = 0;
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
         const int mode = mode_of(v, P.D);
-        args.wt = table + v * slot_floats;
-        switch (d) {
-        case kTB: e = launch_dir<T, kTB>(P, args, mode, st); break;
-        case kBT: e = launch_dir<T, kBT>(P, args, mode, st); break;
-        case kLR: e = launch_dir<T, kLR>(P, args, mode, st); break;
-        default: e = launch_dir<T, kRL>(P, args, mode, st); break;
+        SweepArgs args{x, lam, u, table + v * slot_floats, z, acc, y, zt, acct, P.N, P.C, P.H, P.W, P.Cw};
+        if (is_vertical(d)) {
+            const bool tout = tp && v == nV - 1;
+            e = d == kTB ? launch_vt<T, kTB>(P, args, mode, tout, st) : launch_vt<T, kBT>(P, args, mode, tout, st);
+        } else if (tp) {
+            // horizontal scan over the transposed buffers: scan length W, lanes H
+            args.z = zt;
+            args.acc = acct;
+            args.H = PS.H;
+            args.W = PS.W;
+            const bool tout = v == P.D - 1;
+            e = d == kLR ? launch_vt<T, kTB>(PS, args, mode, tout, st) : launch_vt<T, kBT>(PS, args, mode, tout, st);
+        } else {
+            e = d == kLR ? launch_dir<T, kLR>(P, args, mode, st) : launch_dir<T, kRL>(P, args, mode, st);
         }
         if (e != cudaSuccess) return e;
         ++v;
@@ -773,13 +985,21 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
 bool sweep_supports(const Problem& P, bool bwd) {
     if (bwd) return false;
     if ((P.W * P.esize()) % 16 != 0) return false;   // 16-byte rows and column tiles
-    if (P.W > 4096 || P.H > 1024) return false;
-    if ((long long)P.D * P.N * P.Cw > 65535) return false;   // weight-formation grid.y
+    if (P.W > 4096) return false;
+    if ((long long)P.D * P.N * P.Cw > 65535) return false;   // weight-formation grid.y / grid.z
+    const bool tp = tpath(P);
+    const int nV = n_vertical(P);
+    const Problem PS = swapped(P);
     for (int v = 0, k = 0; k < 4; ++k) {
         const unsigned d = 1u << k;
         if (!(P.mask & d)) continue;
-        const int mode = mode_of(v++, P.D);
-        if (is_vertical(d) ? v_stages(P, mode) == 0 : h_stages(P, mode) == 0) return false;
+        const int mode = mode_of(v, P.D);
+        bool ok;
+        if (is_vertical(d)) ok = v_stages(P, mode, tp && v == nV - 1) > 0;
+        else if (tp) ok = v_stages(PS, mode, v == P.D - 1) > 0;
+        else ok = P.H <= 1024 && h_stages(P, mode) > 0;
+        if (!ok) return false;
+        ++v;
     }
     return true;
 }
@@ -788,6 +1008,7 @@ size_t sweep_ws_bytes(const Problem& P, bool bwd) {
     if (bwd) return 0;
     size_t b = 256 + align256(table_floats(P) * sizeof(float));
     if (P.D > 1) b += 2 * align256((size_t)P.U * P.esize());
+    if (tpath(P)) b += 2 * align256((size_t)P.U * P.esize());
     return b;
 }
 
