@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "gspn.h"
 
 namespace gspn {
@@ -24,6 +26,86 @@ template <> struct Io<__nv_bfloat16> {
     static __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
     static __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 };
+
+// ------------------------------------------------------------------ vector lanes
+// L consecutive lanes of storage type T (aligned to L elements).
+template <typename T, int L>
+__device__ __forceinline__ void ld_lanes(const void* ptr, float (&v)[L]) {
+    if constexpr (L == 8) {
+        if constexpr (std::is_same<T, float>::value) {
+            const float4 q0 = *(const float4*)ptr, q1 = *((const float4*)ptr + 1);
+            v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
+            v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
+        } else {
+            const uint4 q = *(const uint4*)ptr;
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&w[k]);
+                v[2 * k] = f.x;
+                v[2 * k + 1] = f.y;
+            }
+        }
+    } else if constexpr (std::is_same<T, float>::value) {
+        if constexpr (L == 1) {
+            v[0] = *(const float*)ptr;
+        } else if constexpr (L == 2) {
+            const float2 q = *(const float2*)ptr;
+            v[0] = q.x; v[1] = q.y;
+        } else {
+            const float4 q = *(const float4*)ptr;
+            v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+        }
+    } else {
+        if constexpr (L == 1) {
+            v[0] = __bfloat162float(*(const __nv_bfloat16*)ptr);
+        } else if constexpr (L == 2) {
+            const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)ptr);
+            v[0] = f.x; v[1] = f.y;
+        } else {
+            const uint2 q = *(const uint2*)ptr;
+            const float2 f0 = __bfloat1622float2(*(const __nv_bfloat162*)&q.x);
+            const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&q.y);
+            v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+        }
+    }
+}
+
+template <typename T, int L>
+__device__ __forceinline__ void st_lanes(void* ptr, const float (&v)[L]) {
+    if constexpr (L == 8) {
+        if constexpr (std::is_same<T, float>::value) {
+            *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
+            *((float4*)ptr + 1) = make_float4(v[4], v[5], v[6], v[7]);
+        } else {
+            uint4 q;
+            uint32_t* w = &q.x;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+                w[k] = *(const uint32_t*)&b;
+            }
+            *(uint4*)ptr = q;
+        }
+    } else if constexpr (std::is_same<T, float>::value) {
+        if constexpr (L == 1) *(float*)ptr = v[0];
+        else if constexpr (L == 2) *(float2*)ptr = make_float2(v[0], v[1]);
+        else *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+        if constexpr (L == 1) {
+            *(__nv_bfloat16*)ptr = __float2bfloat16_rn(v[0]);
+        } else if constexpr (L == 2) {
+            *(__nv_bfloat162*)ptr = __floats2bfloat162_rn(v[0], v[1]);
+        } else {
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
+            uint2 q;
+            q.x = *(const uint32_t*)&b0;
+            q.y = *(const uint32_t*)&b1;
+            *(uint2*)ptr = q;
+        }
+    }
+}
 
 // ------------------------------------------------------------------ geometry
 // Directions as bit masks, slot order TB, BT, LR, RL.

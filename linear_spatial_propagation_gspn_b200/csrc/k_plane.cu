@@ -1,11 +1,459 @@
-// k_plane.cu -- small-map kernel family (placeholder until the fused kernel lands).
+// k_plane.cu -- small-map kernel family of libgspn: the whole plane stays on chip.
+//
+// One CTA owns one (n, c) plane at a time (persistent over planes). Shared memory holds the
+// plane's z = lambda * x, the running sum over directions and the current direction's weights,
+// all fp32 with an odd row stride so that walking a row (vertical scans) or a column
+// (horizontal scans) across the 32 lanes of a warp is bank-conflict-free. x, lambda and u are
+// read once, every logit is read once, y is written once: the HBM traffic is the compulsory
+// one. Per direction, all threads form the normalised weights from coalesced logit reads
+// ("Parallel Sequence Modeling via Generalized Spatial Propagation Network" summary, section
+// "Approach": sigmoid then normalisation over the in-range neighbours), then one warp runs the
+// sequential scan with the line held in registers and the j +- 1 neighbours exchanged by warp
+// shuffles ("GSPN-2: Efficient Parallel Sequence Modeling" paper notes, section "Optimisation 3":
+// keep h_{i-1} on chip). Several CTAs per SM overlap one plane's scan with another's loads.
+// Directions are added to the sum one after another in the fixed order TB, BT, LR, RL, so the
+// result is deterministic.
+#include <algorithm>
+
+#include "gspn_common.cuh"
 #include "gspn_internal.h"
 
 namespace gspn {
-bool plane_supports(const Problem&, bool) { return false; }
-size_t plane_ws_bytes(const Problem&, bool) { return 0; }
-cudaError_t plane_forward(const Problem&, const void*, const void*, const void*, const void*, void*, void*,
-                          cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t plane_backward(const Problem&, const void*, const void*, const void*, const void*, const void*, void*,
-                           void*, void*, void*, void*, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kPlaneThreads = 128;
+constexpr int kPlaneMaxLanes = 128;            // scan lanes held by one warp (4 per thread)
+constexpr size_t kPlaneSmemBudget = 225 * 1024;
+
+struct PlaneArgs {
+    const void* x;
+    const void* lam;
+    const void* u;
+    const void* a;
+    void* y;
+    int N, C, H, W, Cw, Wp;
+    unsigned mask;
+};
+
+// Weights of one pixel for direction d (w1 = 1 - w0 - w2 is re-derived by the scan). Fast MUFU
+// form; the rare max-shifted form for logits below -40 is applied behind a warp vote.
+template <unsigned D>
+__device__ __forceinline__ void pixel_weights(float a0, float a1, float a2, int r, int col, int H, int W,
+                                              float& w0, float& w2) {
+    constexpr bool V = D == kTB || D == kBT;
+    const bool hl = V ? col > 0 : r > 0;
+    const bool hr = V ? col < W - 1 : r < H - 1;
+    Wts w = lane_weights_fast_nocheck(a0, a1, a2, hl, hr);
+    const bool shift = weights_need_shift(a0, a1, a2, hl, hr);
+    if (__any_sync(__activemask(), shift) && shift) w = weights_shifted(a0, a1, a2, hl, hr);
+    w0 = w.w0;
+    w2 = w.w2;
+}
+
+// Shared-memory offset of scan position (i, j) of direction D.
+template <unsigned D>
+__device__ __forceinline__ int plane_pix(int H, int W, int Wp, int i, int j) {
+    if (D == kTB) return i * Wp + j;
+    if (D == kBT) return (H - 1 - i) * Wp + j;
+    if (D == kLR) return j * Wp + i;
+    return j * Wp + (W - 1 - i);
+}
+
+// One warp scans the whole plane for direction D; lane j is held by thread j / LPT.
+template <unsigned D, int LPT>
+__device__ __forceinline__ void plane_scan(const float* z, const float* w0b, const float* w2b, float* acc, int H,
+                                           int W, int Wp, int lane) {
+    constexpr bool V = D == kTB || D == kBT;
+    const int L = V ? H : W, M = V ? W : H;
+    float h[LPT];
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+    for (int i = 0; i < L; ++i) {
+        float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
+        float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
+        if (lane == 0) hl = 0.f;
+        if (lane == 31) hr = 0.f;
+        float hn[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            const int j = lane * LPT + e;
+            hn[e] = 0.f;
+            if (j < M) {
+                const int q = plane_pix<D>(H, W, Wp, i, j);
+                float v = z[q];
+                if (i > 0) {
+                    const float w0 = w0b[q], w2 = w2b[q];
+                    const float left = e == 0 ? hl : h[e - 1];
+                    const float right = e == LPT - 1 ? hr : h[e + 1];
+                    v = fmaf(w0, left, fmaf(1.f - w0 - w2, h[e], fmaf(w2, right, v)));
+                }
+                acc[q] += v;
+                hn[e] = v;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+    }
+}
+
+// Weights of direction D for the whole plane into w0b / w2b (all threads; 4 pixels per
+// iteration when a row is a multiple of 4 long).
+template <typename T, unsigned D>
+__device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2b, int H, int W, int Wp, int tid) {
+    const int HW = H * W;
+    if (W % 4 == 0) {
+        for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
+            const int r = e / W, col = e - r * W;
+            float a0[4], a1[4], a2[4];
+            ld_lanes<T, 4>(a3 + e, a0);
+            ld_lanes<T, 4>(a3 + HW + e, a1);
+            ld_lanes<T, 4>(a3 + 2 * HW + e, a2);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                pixel_weights<D>(a0[k], a1[k], a2[k], r, col + k, H, W, w0b[r * Wp + col + k], w2b[r * Wp + col + k]);
+        }
+    } else {
+        for (int e = tid; e < HW; e += kPlaneThreads) {
+            const int r = e / W, col = e - r * W;
+            pixel_weights<D>(Io<T>::ld(a3 + e), Io<T>::ld(a3 + HW + e), Io<T>::ld(a3 + 2 * HW + e), r, col, H, W,
+                             w0b[r * Wp + col], w2b[r * Wp + col]);
+        }
+    }
+}
+
+template <typename T, unsigned D, int LPT>
+__device__ __forceinline__ void plane_direction(const T* a3, const float* z, float* w0b, float* w2b, float* acc, int H,
+                                                int W, int Wp, int tid) {
+    plane_weights<T, D>(a3, w0b, w2b, H, W, Wp, tid);
+    __syncthreads();
+    if (tid < 32) plane_scan<D, LPT>(z, w0b, w2b, acc, H, W, Wp, tid);
+    __syncthreads();
+}
+
+template <typename T, int LPT>
+__global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
+    extern __shared__ float sm[];
+    const int H = p.H, W = p.W, Wp = p.Wp;
+    const int HWs = H * Wp;
+    float* z = sm;
+    float* acc = z + HWs;
+    float* w0b = acc + HWs;
+    float* w2b = w0b + HWs;
+    const int tid = threadIdx.x;
+    const int HW = H * W;
+    const int nplanes = p.N * p.C;
+    const bool vec = W % 4 == 0;
+    for (int plane = blockIdx.x; plane < nplanes; plane += gridDim.x) {
+        const int n = plane / p.C, c = plane % p.C;
+        const long long po = (long long)plane * HW;
+        const T* x = (const T*)p.x + po;
+        const T* lam = (const T*)p.lam + po;
+        const T* u = (const T*)p.u + po;
+        T* y = (T*)p.y + po;
+        // z = lambda * x, sum = 0
+        if (vec) {
+            for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
+                const int r = e / W, col = e - r * W;
+                float xv[4], lv[4];
+                ld_lanes<T, 4>(x + e, xv);
+                ld_lanes<T, 4>(lam + e, lv);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    z[r * Wp + col + k] = lv[k] * xv[k];
+                    acc[r * Wp + col + k] = 0.f;
+                }
+            }
+        } else {
+            for (int e = tid; e < HW; e += kPlaneThreads) {
+                const int r = e / W, col = e - r * W;
+                z[r * Wp + col] = Io<T>::ld(lam + e) * Io<T>::ld(x + e);
+                acc[r * Wp + col] = 0.f;
+            }
+        }
+        int slot = 0;
+        auto a_of = [&](int s) {
+            return (const T*)p.a + (((long long)s * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
+        };
+        if (p.mask & kTB) plane_direction<T, kTB, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
+        if (p.mask & kBT) plane_direction<T, kBT, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
+        if (p.mask & kLR) plane_direction<T, kLR, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
+        if (p.mask & kRL) plane_direction<T, kRL, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
+        // y = u * sum
+        if (vec) {
+            for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
+                const int r = e / W, col = e - r * W;
+                float uv[4];
+                ld_lanes<T, 4>(u + e, uv);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) uv[k] *= acc[r * Wp + col + k];
+                st_lanes<T, 4>(y + e, uv);
+            }
+        } else {
+            for (int e = tid; e < HW; e += kPlaneThreads) {
+                const int r = e / W, col = e - r * W;
+                Io<T>::st(y + e, Io<T>::ld(u + e) * acc[r * Wp + col]);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ================================================================== backward (per-channel)
+struct PlaneBwdArgs {
+    const void* x;
+    const void* lam;
+    const void* u;
+    const void* a;
+    const void* dy;
+    void* dx;
+    void* da;
+    void* dlam;
+    void* du;
+    int N, C, H, W, Wp;
+    unsigned mask;
+};
+
+// Forward recompute of direction D by one warp: hb = h^D (plane layout), acc += h^D.
+template <unsigned D, int LPT>
+__device__ __forceinline__ void plane_recompute(const float* z, const float* w0b, const float* w2b, float* hb,
+                                                float* acc, int H, int W, int Wp, int lane) {
+    constexpr bool V = D == kTB || D == kBT;
+    const int L = V ? H : W, M = V ? W : H;
+    float h[LPT];
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+    for (int i = 0; i < L; ++i) {
+        float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
+        float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
+        if (lane == 0) hl = 0.f;
+        if (lane == 31) hr = 0.f;
+        float hn[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            const int j = lane * LPT + e;
+            hn[e] = 0.f;
+            if (j < M) {
+                const int q = plane_pix<D>(H, W, Wp, i, j);
+                float v = z[q];
+                if (i > 0) {
+                    const float w0 = w0b[q], w2 = w2b[q];
+                    v = fmaf(w0, e == 0 ? hl : h[e - 1], fmaf(1.f - w0 - w2, h[e], fmaf(w2, e == LPT - 1 ? hr : h[e + 1], v)));
+                }
+                hb[q] = v;
+                acc[q] += v;
+                hn[e] = v;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+    }
+}
+
+// Reverse scan of direction D by one warp:
+//   delta_i[j] = g_i[j] + w_{i+1}[j-1][2] delta_{i+1}[j-1] + w_{i+1}[j][1] delta_{i+1}[j] + w_{i+1}[j+1][0] delta_{i+1}[j+1]
+// dz += delta; da_k = w_k sigmoid(-a_k) (dw_k - sum_k' w_k' dw_k') with dw_k = delta_i[j] h_{i-1}[j+k-1].
+template <typename T, unsigned D, int LPT>
+__device__ __forceinline__ void plane_reverse(const T* a3, T* da3, const float* g, const float* w0b, const float* w2b,
+                                             const float* hb, float* dz, int H, int W, int Wp, int lane) {
+    constexpr bool V = D == kTB || D == kBT;
+    const int L = V ? H : W, M = V ? W : H;
+    const int HW = H * W;
+    float del[LPT], pw0[LPT], pw1[LPT], pw2[LPT];   // delta and weights of step i+1
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) del[e] = pw0[e] = pw1[e] = pw2[e] = 0.f;
+    for (int i = L - 1; i >= 0; --i) {
+        // neighbour terms of w_{i+1}^T delta_{i+1}: lane j-1's (w2 delta) and lane j+1's (w0 delta)
+        float fromL = __shfl_up_sync(0xffffffffu, pw2[LPT - 1] * del[LPT - 1], 1);
+        float fromR = __shfl_down_sync(0xffffffffu, pw0[0] * del[0], 1);
+        if (lane == 0) fromL = 0.f;
+        if (lane == 31) fromR = 0.f;
+        float dn[LPT], nw0[LPT], nw1[LPT], nw2[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            const int j = lane * LPT + e;
+            dn[e] = nw0[e] = nw1[e] = nw2[e] = 0.f;
+            if (j < M) {
+                const int q = plane_pix<D>(H, W, Wp, i, j);
+                float d = g[q];
+                if (i < L - 1) {
+                    const float l = e == 0 ? fromL : pw2[e - 1] * del[e - 1];
+                    const float r = e == LPT - 1 ? fromR : pw0[e + 1] * del[e + 1];
+                    d = fmaf(pw1[e], del[e], d) + l + r;
+                }
+                dz[q] += d;
+                dn[e] = d;
+                // image offset of (i, j) for the logits / da
+                const int r0 = q / Wp, c0 = q - r0 * Wp;
+                const int gq = r0 * W + c0;
+                if (i > 0) {
+                    const float w0 = w0b[q], w2 = w2b[q], w1 = 1.f - w0 - w2;
+                    const bool hasl = j > 0, hasr = j < M - 1;
+                    const float h0 = hasl ? hb[plane_pix<D>(H, W, Wp, i - 1, j - 1)] : 0.f;
+                    const float h1 = hb[plane_pix<D>(H, W, Wp, i - 1, j)];
+                    const float h2 = hasr ? hb[plane_pix<D>(H, W, Wp, i - 1, j + 1)] : 0.f;
+                    const float dw0 = d * h0, dw1 = d * h1, dw2 = d * h2;
+                    const float sdw = w0 * dw0 + w1 * dw1 + w2 * dw2;
+                    const float a0 = Io<T>::ld(a3 + gq), a1 = Io<T>::ld(a3 + HW + gq), a2 = Io<T>::ld(a3 + 2 * HW + gq);
+                    Io<T>::st(da3 + gq, hasl ? w0 * sigmoidf_(-a0) * (dw0 - sdw) : 0.f);
+                    Io<T>::st(da3 + HW + gq, w1 * sigmoidf_(-a1) * (dw1 - sdw));
+                    Io<T>::st(da3 + 2 * HW + gq, hasr ? w2 * sigmoidf_(-a2) * (dw2 - sdw) : 0.f);
+                    nw0[e] = w0;
+                    nw1[e] = w1;
+                    nw2[e] = w2;
+                } else {
+                    Io<T>::st(da3 + gq, 0.f);
+                    Io<T>::st(da3 + HW + gq, 0.f);
+                    Io<T>::st(da3 + 2 * HW + gq, 0.f);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            del[e] = dn[e];
+            pw0[e] = nw0[e];
+            pw1[e] = nw1[e];
+            pw2[e] = nw2[e];
+        }
+    }
+}
+
+template <typename T, unsigned D, int LPT>
+__device__ __forceinline__ void plane_bwd_direction(const T* a3, T* da3, const float* z, const float* g, float* w0b,
+                                                    float* w2b, float* hb, float* acc, float* dz, int H, int W, int Wp,
+                                                    int tid) {
+    plane_weights<T, D>(a3, w0b, w2b, H, W, Wp, tid);
+    __syncthreads();
+    if (tid < 32) {
+        plane_recompute<D, LPT>(z, w0b, w2b, hb, acc, H, W, Wp, tid);
+        __syncwarp();
+        plane_reverse<T, D, LPT>(a3, da3, g, w0b, w2b, hb, dz, H, W, Wp, tid);
+    }
+    __syncthreads();
+}
+
+template <typename T, int LPT>
+__global__ void __launch_bounds__(kPlaneThreads) k_plane_bwd(PlaneBwdArgs p) {
+    extern __shared__ float sm[];
+    const int H = p.H, W = p.W, Wp = p.Wp;
+    const int HWs = H * Wp;
+    float* z = sm;
+    float* g = z + HWs;
+    float* acc = g + HWs;
+    float* dz = acc + HWs;
+    float* hb = dz + HWs;
+    float* w0b = hb + HWs;
+    float* w2b = w0b + HWs;
+    const int tid = threadIdx.x;
+    const int HW = H * W;
+    const int nplanes = p.N * p.C;
+    for (int plane = blockIdx.x; plane < nplanes; plane += gridDim.x) {
+        const int n = plane / p.C, c = plane % p.C;
+        const long long po = (long long)plane * HW;
+        const T *x = (const T*)p.x + po, *lam = (const T*)p.lam + po, *u = (const T*)p.u + po, *dy = (const T*)p.dy + po;
+        for (int e = tid; e < HW; e += kPlaneThreads) {
+            const int q = (e / W) * Wp + e % W;
+            z[q] = Io<T>::ld(lam + e) * Io<T>::ld(x + e);
+            g[q] = Io<T>::ld(u + e) * Io<T>::ld(dy + e);
+            acc[q] = 0.f;
+            dz[q] = 0.f;
+        }
+        int slot = 0;
+        auto aoff = [&](int s) { return (((long long)s * p.N + n) * p.C + c) * 3 * HW; };
+        if (p.mask & kTB) { const long long o = aoff(slot++); plane_bwd_direction<T, kTB, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
+        for (int e = tid; e < HW; e += kPlaneThreads) {
+            const int q = (e / W) * Wp + e % W;
+            Io<T>::st((T*)p.dx + po + e, Io<T>::ld(lam + e) * dz[q]);
+            Io<T>::st((T*)p.dlam + po + e, Io<T>::ld(x + e) * dz[q]);
+            Io<T>::st((T*)p.du + po + e, Io<T>::ld(dy + e) * acc[q]);
+        }
+        __syncthreads();
+    }
+}
+
+int plane_wp(const Problem& P) { return P.W % 2 == 0 ? P.W + 1 : P.W; }
+size_t plane_smem(const Problem& P) { return 4 * (size_t)P.H * plane_wp(P) * sizeof(float); }
+int plane_lanes(const Problem& P) {
+    const int M = std::max(P.H, P.W);
+    return M <= 32 ? 1 : (M <= 64 ? 2 : 4);
+}
+
+size_t plane_bwd_smem(const Problem& P) { return 7 * (size_t)P.H * plane_wp(P) * sizeof(float); }
+
+template <typename T, int LPT>
+cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
+    const size_t smem = plane_bwd_smem(P);
+    cudaError_t e = cudaFuncSetAttribute(k_plane_bwd<T, LPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(k_plane_bwd<T, LPT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int per_sm = 1;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_bwd<T, LPT>, kPlaneThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long want = (long long)std::max(1, per_sm) * device_sm_count();
+    const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
+    launch_begin(st);
+    k_plane_bwd<T, LPT><<<grid, kPlaneThreads, smem, st>>>(a);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+template <typename T, int LPT>
+cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
+    const size_t smem = plane_smem(P);
+    cudaError_t e = cudaFuncSetAttribute(k_plane_fwd<T, LPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(k_plane_fwd<T, LPT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int per_sm = 1;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_fwd<T, LPT>, kPlaneThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long want = (long long)std::max(1, per_sm) * device_sm_count();
+    const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
+    launch_begin(st);
+    k_plane_fwd<T, LPT><<<grid, kPlaneThreads, smem, st>>>(a);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t plane_forward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
+                            cudaStream_t st) {
+    PlaneArgs args{x, lam, u, a, y, P.N, P.C, P.H, P.W, P.Cw, plane_wp(P), P.mask};
+    switch (plane_lanes(P)) {
+    case 1: return plane_fwd_launch<T, 1>(P, args, st);
+    case 2: return plane_fwd_launch<T, 2>(P, args, st);
+    default: return plane_fwd_launch<T, 4>(P, args, st);
+    }
+}
+
+}  // namespace
+
+bool plane_supports(const Problem& P, bool bwd) {
+    if (std::max(P.H, P.W) > kPlaneMaxLanes) return false;
+    if ((long long)P.H * P.W > (1LL << 20)) return false;
+    if (bwd) return P.wmode == GSPN_W_PER_CHANNEL && plane_bwd_smem(P) <= kPlaneSmemBudget;
+    return plane_smem(P) <= kPlaneSmemBudget;
+}
+
+size_t plane_ws_bytes(const Problem&, bool) { return 256; }
+
+cudaError_t plane_forward(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
+                          void*, cudaStream_t st) {
+    if (P.dtype == GSPN_F32) return plane_forward_t<float>(P, x, a, lam, u, y, st);
+    return plane_forward_t<__nv_bfloat16>(P, x, a, lam, u, y, st);
+}
+
+cudaError_t plane_backward(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
+                           const void* dy, void* dx, void* da, void* dlam, void* du, void*, cudaStream_t st) {
+    PlaneBwdArgs args{x, lam, u, a, dy, dx, da, dlam, du, P.N, P.C, P.H, P.W, plane_wp(P), P.mask};
+    const int lpt = plane_lanes(P);
+    if (P.dtype == GSPN_F32)
+        return lpt == 1 ? plane_bwd_launch<float, 1>(P, args, st)
+                        : (lpt == 2 ? plane_bwd_launch<float, 2>(P, args, st) : plane_bwd_launch<float, 4>(P, args, st));
+    return lpt == 1 ? plane_bwd_launch<__nv_bfloat16, 1>(P, args, st)
+                    : (lpt == 2 ? plane_bwd_launch<__nv_bfloat16, 2>(P, args, st)
+                                : plane_bwd_launch<__nv_bfloat16, 4>(P, args, st));
+}
+
 }  // namespace gspn

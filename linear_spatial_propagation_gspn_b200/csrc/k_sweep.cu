@@ -122,85 +122,6 @@ __device__ __forceinline__ unsigned char* align128(unsigned char* ptr) {
     return (unsigned char*)(((uintptr_t)ptr + 127) & ~(uintptr_t)127);
 }
 
-// L consecutive lanes of storage type T (aligned to L elements).
-template <typename T, int L>
-__device__ __forceinline__ void ld_lanes(const void* ptr, float (&v)[L]) {
-    if constexpr (L == 8) {
-        if constexpr (std::is_same<T, float>::value) {
-            const float4 q0 = *(const float4*)ptr, q1 = *((const float4*)ptr + 1);
-            v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
-            v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
-        } else {
-            const uint4 q = *(const uint4*)ptr;
-            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&w[k]);
-                v[2 * k] = f.x;
-                v[2 * k + 1] = f.y;
-            }
-        }
-    } else if constexpr (std::is_same<T, float>::value) {
-        if constexpr (L == 1) {
-            v[0] = *(const float*)ptr;
-        } else if constexpr (L == 2) {
-            const float2 q = *(const float2*)ptr;
-            v[0] = q.x; v[1] = q.y;
-        } else {
-            const float4 q = *(const float4*)ptr;
-            v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-        }
-    } else {
-        if constexpr (L == 1) {
-            v[0] = __bfloat162float(*(const __nv_bfloat16*)ptr);
-        } else if constexpr (L == 2) {
-            const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)ptr);
-            v[0] = f.x; v[1] = f.y;
-        } else {
-            const uint2 q = *(const uint2*)ptr;
-            const float2 f0 = __bfloat1622float2(*(const __nv_bfloat162*)&q.x);
-            const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&q.y);
-            v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
-        }
-    }
-}
-
-template <typename T, int L>
-__device__ __forceinline__ void st_lanes(void* ptr, const float (&v)[L]) {
-    if constexpr (L == 8) {
-        if constexpr (std::is_same<T, float>::value) {
-            *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
-            *((float4*)ptr + 1) = make_float4(v[4], v[5], v[6], v[7]);
-        } else {
-            uint4 q;
-            uint32_t* w = &q.x;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-                w[k] = *(const uint32_t*)&b;
-            }
-            *(uint4*)ptr = q;
-        }
-    } else if constexpr (std::is_same<T, float>::value) {
-        if constexpr (L == 1) *(float*)ptr = v[0];
-        else if constexpr (L == 2) *(float2*)ptr = make_float2(v[0], v[1]);
-        else *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
-    } else {
-        if constexpr (L == 1) {
-            *(__nv_bfloat16*)ptr = __float2bfloat16_rn(v[0]);
-        } else if constexpr (L == 2) {
-            *(__nv_bfloat162*)ptr = __floats2bfloat162_rn(v[0], v[1]);
-        } else {
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
-            uint2 q;
-            q.x = *(const uint32_t*)&b0;
-            q.y = *(const uint32_t*)&b1;
-            *(uint2*)ptr = q;
-        }
-    }
-}
-
 // A thread's LPT lanes of one row in shared memory. With fp32 and LPT = 8 a thread owns 32
 // bytes, and threads t and t+4 would hit the same banks in a 16-byte load phase; the thread
 // therefore stores its two 16-byte chunks in swapped order when bit 2 of its index is set
@@ -322,14 +243,15 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
     const int wrowB = W * 4;
     const int stageB = 2 * wrowB + NTEN * rowB;
     float* halo = (float*)(smem + (size_t)NS * stageB);   // [2 parity][2 lo/hi][32 warps]
-    // TOUT staging: Md::NSTG blocks of [kTB_STEPS][R] fp32, row stride R = 4 (mod 32) so the
-    // column reads of the flush hit at most two lanes per bank.
-    float* stg = halo + 128;
-    const int R = ((W + 31) / 32) * 32 + 4;
+    // TOUT staging: Md::NSTG blocks of [kTB_STEPS][R] in the storage dtype (the values are
+    // stored in that dtype anyway). R is W rounded up to 32 plus 16 bytes, so every staging row
+    // starts 16-byte aligned (vector stores) and consecutive rows shift the bank pattern.
+    T* stg = (T*)(halo + 128);
+    const int R = ((W + 31) / 32) * 32 + 16 / (int)sizeof(T);
     // TOUT final: u of the next staging block, prefetched lane-major, 16 bytes per chunk id
     constexpr int CH = 16 / (int)sizeof(T);          // steps per 16-byte chunk
     constexpr int CPL = kTB_STEPS / CH;              // chunks per lane segment
-    uint4* ubuf = (uint4*)(stg + (size_t)Md::NSTG * kTB_STEPS * R);
+    uint4* ubuf = (uint4*)align128((unsigned char*)(stg + (size_t)Md::NSTG * kTB_STEPS * R));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const int j0 = tid * LPT;
     const bool active = j0 < W;
@@ -481,12 +403,12 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
                 if (Md::URING) o[e] *= cu[e];
             }
             if constexpr (TOUT) {
-                float* srow = stg + (size_t)(r % kTB_STEPS) * R + j0;
+                T* srow = stg + (size_t)(r % kTB_STEPS) * R + j0;
                 if constexpr (Md::FINAL) {
-                    st_lanes<float, LPT>(srow, o);
+                    st_lanes<T, LPT>(srow, o);
                 } else {
-                    st_lanes<float, LPT>(srow, cz);
-                    st_lanes<float, LPT>(srow + kTB_STEPS * R, o);
+                    st_lanes<T, LPT>(srow, cz);
+                    st_lanes<T, LPT>(srow + kTB_STEPS * R, o);
                 }
             } else {
                 st_lanes<T, LPT>((T*)(Md::FINAL ? p.y : p.acc) + off, o);
@@ -517,7 +439,7 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
                 const int q = tid % CPL, jstep = (int)blockDim.x / CPL;
                 if (q * CH < nvalid) {
                     const long long gstep = (long long)jstep * H;
-                    const float* sp = stg + (size_t)(q * CH) * R + tid / CPL;
+                    const T* sp = stg + (size_t)(q * CH) * R + tid / CPL;
                     const long long g0 = poff + (long long)(tid / CPL) * H + s_base + q * CH;
                     if constexpr (Md::FINAL) {
                         T* gp = (T*)p.y + g0;
@@ -527,7 +449,7 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
                             float v[CH], uu[CH];
                             ld_lanes<T, CH>(up, uu);
 #pragma unroll
-                            for (int k = 0; k < CH; ++k) v[k] = sp[k * R] * uu[k];
+                            for (int k = 0; k < CH; ++k) v[k] = Io<T>::ld(sp + k * R) * uu[k];
                             st_lanes<T, CH>(gp, v);
                         }
                     } else {
@@ -539,8 +461,8 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
                             float v[CH], va[CH];
 #pragma unroll
                             for (int k = 0; k < CH; ++k) {
-                                v[k] = sp[k * R];
-                                va[k] = sp[second + k * R];
+                                v[k] = Io<T>::ld(sp + k * R);
+                                va[k] = Io<T>::ld(sp + second + k * R);
                             }
                             st_lanes<T, CH>(gz, v);
                             st_lanes<T, CH>(ga, va);
@@ -780,15 +702,21 @@ int v_lanes(const Problem& P) {
 }
 int v_threads(const Problem& P) { return std::max(32, ((P.W / v_lanes(P) + 31) / 32) * 32); }
 size_t v_smem(const Problem& P, int mode, int ns, bool tout) {
-    const size_t R = ((size_t)(P.W + 31) / 32) * 32 + 4;
+    const size_t R = ((size_t)(P.W + 31) / 32) * 32 + 16 / P.esize();
     const bool ubuf = tout && (mode == M_LAST || mode == M_ONLY);
     return 128 + (size_t)ns * (2 * (size_t)P.W * 4 + (size_t)ntensors(mode, tout) * P.W * P.esize()) + 512 +
-           (size_t)nstaged(mode, tout) * kTB_STEPS * R * sizeof(float) +
+           (size_t)nstaged(mode, tout) * kTB_STEPS * R * P.esize() + 128 +
            (ubuf ? (size_t)P.W * kTB_STEPS * P.esize() : 0);
 }
+// 4 stages when they fit; 2 when there are more planes than SMs and the shorter ring lets twice
+// as many CTAs (planes) share an SM, which hides more of the per-step latency.
 int v_stages(const Problem& P, int mode, bool tout = false) {
-    if (v_smem(P, mode, 4, tout) <= kSmemBudget) return 4;
-    return v_smem(P, mode, 2, tout) <= kSmemBudget ? 2 : 0;
+    const size_t s4 = v_smem(P, mode, 4, tout), s2 = v_smem(P, mode, 2, tout);
+    if (s2 > kSmemBudget) return 0;
+    if (s4 > kSmemBudget) return 2;
+    const bool many = (long long)P.N * P.C > device_sm_count();
+    if (many && kSmemBudget / s2 >= 2 * (kSmemBudget / s4)) return 2;
+    return 4;
 }
 
 // ---- horizontal geometry: threads, rows per thread (as instantiated), padded rows, ring depth
@@ -819,13 +747,25 @@ int h_stages(const Problem& P, int mode) {
     return h_smem(P, mode, 2) <= kSmemBudget ? 2 : 0;
 }
 
+// Persistent grid: as many CTAs as fit on the device at once, but never more than planes. Each
+// CTA runs one plane's scan at a time, so several CTAs per SM hide the per-step latency when
+// there are more planes than SMs.
+template <typename K>
+int sweep_grid(const Problem& P, K kern, int threads, size_t smem) {
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    return (int)std::min<long long>((long long)per_sm * device_sm_count(), (long long)P.N * P.C);
+}
+
 template <typename T, unsigned DIR, int MODE, bool TOUT, int LPT, int NS>
 cudaError_t launch_v4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
     const size_t smem = v_smem(P, MODE, NS, TOUT);
-    const int grid = std::min(P.N * P.C, device_sm_count());
-    cudaError_t e = cudaFuncSetAttribute(k_vsweep<T, DIR, MODE, LPT, NS, TOUT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = k_vsweep<T, DIR, MODE, LPT, NS, TOUT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    const int grid = sweep_grid(P, kern, v_threads(P), smem);
     launch_begin(st);
     k_vsweep<T, DIR, MODE, LPT, NS, TOUT><<<grid, v_threads(P), smem, st>>>(a);
     launch_end(st);
@@ -847,10 +787,11 @@ cudaError_t launch_v(const Problem& P, const SweepArgs& a, cudaStream_t st) {
 template <typename T, unsigned DIR, int MODE, int G, int NS>
 cudaError_t launch_h4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
     const size_t smem = h_smem(P, MODE, NS);
-    const int grid = std::min(P.N * P.C, device_sm_count());
-    cudaError_t e = cudaFuncSetAttribute(k_hsweep<T, DIR, MODE, G, NS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = k_hsweep<T, DIR, MODE, G, NS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    const int grid = sweep_grid(P, kern, h_threads(P), smem);
     launch_begin(st);
     k_hsweep<T, DIR, MODE, G, NS><<<grid, h_threads(P), smem, st>>>(a, h_pad(P));
     launch_end(st);
