@@ -10,16 +10,20 @@
 // costs about 285 ns per operation per SM whatever its size up to 32 KB, and the operations of
 // one SM are serialised; a sweep needs 5-7 row-sized copies per step, which capped it near
 // 1.2-1.9 us per step. Per-thread copies have no such per-operation cost.)
-//   - vertical sweeps (TB, BT): thread t owns LPT consecutive lanes of a row; its copies are
-//     contiguous across the warp (fully coalesced);
-//   - horizontal sweeps (LR, RL): column tiles of 16 bytes per row (4 fp32 or 8 bf16 steps, a
-//     staged transpose); thread t owns rows t, t+T, ..., copies and reads 16 bytes per row per
-//     tensor (conflict-free), and writes its outputs back as 16-byte row segments.
-// No direction issues strided per-element HBM traffic. The first sweep reads x and lambda and
-// writes z = lambda * x and the partial sum; later sweeps read z and the partial sum (both in the
-// storage dtype); the last one reads u and writes y = u * (partial + h). ("GSPN-2: Efficient
-// Parallel Sequence Modeling" paper notes, section "Optimisation 3: efficient CUDA extension":
-// coalesced access and on-chip reuse of h_{i-1} were the decisive optimisations on A100.)
+//
+// Horizontal directions. When both image axes give 16-byte rows, the vertical sweeps also write
+// z and the partial sum lane-major (transposed), and the horizontal scans run on the vertical
+// kernel over those buffers; the last one writes y back in the image layout. A lane-major output
+// leaves through a double-buffered shared-memory staging block of KST steps that dedicated
+// writer warps drain as one 32- or 64-byte segment per lane while the scan warps go on (hand-off
+// by mbarriers), so the scattered segment writes stay off the scan's critical path. Otherwise
+// the horizontal scans read column tiles of 16 bytes per row (k_hsweep).
+//
+// The first sweep reads x and lambda (z = lambda * x); later sweeps read z or recompute it, and
+// the partial sum (both in the storage dtype); the last one applies u and writes y. No direction
+// issues strided per-element HBM traffic. ("GSPN-2: Efficient Parallel Sequence Modeling" paper
+// notes, section "Optimisation 3: efficient CUDA extension": coalesced access and on-chip reuse
+// of h_{i-1} were the decisive optimisations on A100.)
 #include <stdlib.h>
 
 #include <algorithm>
@@ -33,35 +37,30 @@ namespace {
 
 enum { M_FIRST = 0, M_ONLY = 1, M_MID = 2, M_LAST = 3 };
 
-// TOUT: outputs leave through a shared-memory staging block and are written lane-major
-// (transposed); a final sweep then applies u while flushing, so u is not in the ring.
-template <int MODE, bool TOUT = false> struct ModeT {
+// Column-tile sweep modes (k_hsweep).
+template <int MODE> struct ModeT {
     static constexpr bool XL = MODE == M_FIRST || MODE == M_ONLY;     // read x, lam (else z)
     static constexpr bool ACCIN = MODE == M_MID || MODE == M_LAST;    // read the partial sum
     static constexpr bool FINAL = MODE == M_ONLY || MODE == M_LAST;   // read u, write y
-    static constexpr bool ZOUT = MODE == M_FIRST || (TOUT && !FINAL); // write z (z^T when TOUT)
-    static constexpr bool URING = FINAL && !TOUT;                     // u comes through the ring
+    static constexpr bool ZOUT = MODE == M_FIRST;                     // write z
+    static constexpr bool URING = FINAL;                              // u comes through the ring
     // storage-dtype tensors per stage: x lam | z, [acc], [u]  (plus the two fp32 weight rows)
     static constexpr int NTEN = (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (URING ? 1 : 0);
-    // staged outputs when TOUT: z and acc, or the unscaled sum for a final sweep
-    static constexpr int NSTG = TOUT ? (FINAL ? 1 : 2) : 0;
 };
-
-// Steps per staging block of a transposed-output sweep (64 bytes of fp32 per lane).
-constexpr int kTB_STEPS = 16;
 
 // Sweep arguments in scan coordinates: H = scan length (steps), W = lanes. A horizontal scan
 // over transposed buffers passes (H, W) = (image width, image height).
 struct SweepArgs {
     const void* x;
     const void* lam;
-    const void* u;    // scan-major, or lane-major (image layout) for a transposed-output final sweep
+    const void* u;    // scan-major, or lane-major (image layout) for a lane-major final sweep
     const float* wt;  // weight table of this direction's slot: [N][Cw][2][H][W] fp32 (w0, w2)
     void* z;          // workspace, storage dtype, scan-major
     void* acc;        // workspace, storage dtype, scan-major
-    void* y;          // output (scan-major, or lane-major when TOUT)
-    void* zt;         // lane-major z   (TOUT, non-final)
-    void* acct;       // lane-major acc (TOUT, non-final)
+    void* y;          // output (scan-major, or lane-major for a lane-major final sweep)
+    void* zt;         // lane-major z
+    void* acct;       // lane-major partial sum
+    unsigned* status; // device status word (hand-off timeouts)
     int N, C, H, W, Cw;
 };
 
@@ -227,256 +226,608 @@ __global__ void __launch_bounds__(256) k_sweep_weights_t(WeightArgs p) {
 }
 
 // ================================================================== vertical sweep
-// CTA = one plane at a time (persistent over planes b, b + grid, ...); thread t owns lanes
-// [LPT t, LPT t + LPT). Ring of NS stages; a stage is one image row of the two fp32 weight
-// rows and of each storage-dtype input. Every thread keeps NS rows of its own lanes in flight.
-// The loop is software-pipelined by one step: while step g's new line is exchanged at the
-// barrier, every thread has already pulled step g+1's inputs out of the ring.
-template <typename T, unsigned DIR, int MODE, int LPT, int NS, bool TOUT>
+// Roles of a vertical sweep. On the transposed path (a vertical and a horizontal direction in the
+// mask, 16-byte rows on both axes) the vertical sweeps hand z and the partial sum over
+// lane-major, the horizontal scans run as vertical sweeps over those buffers with H and W
+// swapped, and the last of them writes y back in the image layout.
+enum {
+    R_FIRST = 0,   // x, lam -> z, partial                          (scan-major)
+    R_ONLY = 1,    // x, lam, u -> y                                (scan-major)
+    R_MID = 2,     // z, partial -> partial                         (scan-major)
+    R_LAST = 3,    // z, partial, u -> y                            (scan-major)
+    R_SZ = 4,      // x, lam -> partial (scan-major), z (lane-major)
+    R_SA = 5,      // x, lam, partial -> partial (lane-major)
+    R_SZA = 6,     // x, lam -> z and partial (lane-major)
+    R_SY = 7,      // z, partial -> y (lane-major, u applied while writing)
+    R_ZSA = 8,     // z, partial -> z and partial (lane-major)
+};
+template <int ROLE> struct RoleT {
+    static constexpr bool XL = ROLE == R_FIRST || ROLE == R_ONLY || ROLE == R_SZ || ROLE == R_SA || ROLE == R_SZA;
+    static constexpr bool ACCIN = ROLE == R_MID || ROLE == R_LAST || ROLE == R_SA || ROLE == R_SY || ROLE == R_ZSA;
+    static constexpr bool URING = ROLE == R_ONLY || ROLE == R_LAST;   // u through the ring
+    static constexpr bool ZNAT = ROLE == R_FIRST;
+    static constexpr bool ANAT = ROLE == R_FIRST || ROLE == R_MID || ROLE == R_SZ;
+    static constexpr bool YNAT = ROLE == R_ONLY || ROLE == R_LAST;
+    static constexpr bool ZSTG = ROLE == R_SZ || ROLE == R_SZA || ROLE == R_ZSA;
+    static constexpr bool ASTG = ROLE == R_SA || ROLE == R_SZA || ROLE == R_SY || ROLE == R_ZSA;
+    static constexpr bool YSTG = ROLE == R_SY;
+    // storage-dtype tensors per ring stage: x lam | z, [partial], [u]  (plus two fp32 weight rows)
+    static constexpr int NTEN = (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (URING ? 1 : 0);
+    static constexpr int NSTG = (ZSTG ? 1 : 0) + (ASTG ? 1 : 0);   // staged (lane-major) outputs
+    // (ring stages, lane-major segment bytes) of the two launch configurations: A, and B with a
+    // shorter ring for more CTAs per SM. A final lane-major sweep also keeps u of two blocks.
+    static constexpr int NS_A = 4, SEG_A = (NSTG == 1 && !YSTG) ? 64 : 32;
+    static constexpr int NS_B = 2, SEG_B = 32;
+};
+
+// ---- mbarrier hand-off between the scan warps and the writer warps of a lane-major sweep
+constexpr unsigned long long kHandoffLimitNs = 1000000000ull;   // 1 s: far above any block's time
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
+    unsigned ok;
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0u;
+}
+// Waits for the phase of `bar` with this parity. Gives up after kHandoffLimitNs: the timeout is
+// recorded in the status word and the caller carries on as if the phase had completed (its
+// outputs are then garbage, but every thread still reaches every barrier, so the kernel ends).
+// SLEEP: back off between polls (the writer warps, which wait most of the time and would
+// otherwise take issue slots from the scan warps on the same scheduler).
+template <bool SLEEP>
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned* status) {
+    if (mbar_test(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_test(bar, parity)) {
+        if (globaltimer_ns() - t0 > kHandoffLimitNs) {
+            report_timeout(status);
+            return false;
+        }
+        if (SLEEP) __nanosleep(128);
+    }
+    return true;
+}
+
+// Writer warps of a lane-major sweep. The scan warps fill staging block k (KST steps of every
+// lane, [step][lane]) in buffer k % 2 and arrive on full[k % 2]; the writers wait for it, write
+// each lane's KST steps as one segment of KST * sizeof(T) bytes of the lane-major output, and
+// arrive on free[k % 2], which the scan warps wait for before refilling that buffer two blocks
+// later. Writer thread f handles chunk q = f % CPL (16 bytes) of lanes f / CPL, f / CPL + nfl /
+// CPL, ...: a warp store covers 32 / CPL whole segments. For y, the writers multiply by u, which
+// they copy (cp.async, the same chunks) into ubuf[(k + 1) % 2] one block ahead: scattered
+// segment reads are latency-bound, so they must be in flight long before they are needed.
+template <typename T, unsigned DIR, int ROLE, int KST>
+__device__ __forceinline__ void write_blocks(const SweepArgs& p, const T* stg, size_t stg_buf, int R, uint64_t* bars,
+                                             T* ubuf, int f, int nfl, int my_planes) {
+    using Rl = RoleT<ROLE>;
+    constexpr int CH = 16 / (int)sizeof(T);   // steps per 16-byte chunk
+    constexpr int CPL = KST / CH;             // chunks per lane segment
+    const int H = p.H, W = p.W;
+    const long long HW = (long long)H * W;
+    const int nbp = (H + KST - 1) / KST;
+    const int nblk = my_planes * nbp;
+    const int q = f % CPL, j1 = f / CPL, jstep = nfl / CPL;
+    // block k -> (plane offset, first step, valid steps)
+    auto block_at = [&](int k, long long& poff, int& s_base, int& nvalid) {
+        const int pl = k / nbp, bi = k - pl * nbp;
+        poff = (long long)((int)blockIdx.x + pl * (int)gridDim.x) * HW;
+        s_base = (DIR == kTB ? bi : nbp - 1 - bi) * KST;
+        nvalid = min(KST, H - s_base);
+    };
+    // y only: copy u of block k into ubuf[k % 2] (this thread's chunks), one commit group
+    auto prefetch_u = [&](int k) {
+        if constexpr (Rl::YSTG) {
+            if (k < nblk) {
+                long long poff;
+                int s_base, nvalid;
+                block_at(k, poff, s_base, nvalid);
+                if (q * CH < nvalid) {
+                    const T* src = (const T*)p.u + poff + s_base + q * CH;
+                    T* dst = ubuf + (size_t)(k & 1) * W * KST + q * CH;
+                    for (int j = j1; j < W; j += jstep) cp_async<16>(dst + (size_t)j * KST, src + (long long)j * H);
+                }
+            }
+            cp_async_commit();
+        }
+    };
+    prefetch_u(0);
+    bool dead = false;
+    for (int k = 0; k < nblk; ++k) {
+        prefetch_u(k + 1);
+        const int b = k & 1;
+        if (!dead) dead = !mbar_wait_bounded<true>(&bars[b], (unsigned)(k >> 1) & 1u, p.status);
+        long long poff;
+        int s_base, nvalid;
+        block_at(k, poff, s_base, nvalid);
+        if (q * CH < nvalid) {   // H is a multiple of CH: a chunk is either all valid or absent
+            const T* sb = stg + (size_t)b * stg_buf + (size_t)(q * CH) * R;
+            const long long g0 = poff + s_base + q * CH;
+#pragma unroll
+            for (int s = 0; s < Rl::NSTG; ++s) {
+                const T* ss = sb + (size_t)s * KST * R;
+                T* dst = (T*)(Rl::YSTG ? p.y : ((Rl::ZSTG && s == 0) ? p.zt : p.acct));
+                if constexpr (Rl::YSTG) {
+                    cp_async_wait<1>();   // block k's u has landed (block k + 1's may be in flight)
+                    const T* ub = ubuf + (size_t)b * W * KST + q * CH;
+#pragma unroll 4
+                    for (int j = j1; j < W; j += jstep) {
+                        const uint4 uu = *(const uint4*)(ub + (size_t)j * KST);
+                        float v[CH];
+#pragma unroll
+                        for (int kk = 0; kk < CH; ++kk) v[kk] = Io<T>::ld(ss + kk * R + j) * Seg<T>::get(uu, kk);
+                        st_lanes<T, CH>(dst + g0 + (long long)j * H, v);
+                    }
+                } else {
+#pragma unroll 4
+                    for (int j = j1; j < W; j += jstep) {
+                        float v[CH];
+#pragma unroll
+                        for (int kk = 0; kk < CH; ++kk) v[kk] = Io<T>::ld(ss + kk * R + j);
+                        st_lanes<T, CH>(dst + g0 + (long long)j * H, v);
+                    }
+                }
+            }
+        }
+        mbar_arrive(&bars[2 + b]);
+    }
+    if constexpr (Rl::YSTG) cp_async_wait<0>();
+}
+
+// CTA = one plane at a time (persistent over planes b, b + grid, ...). Scan thread t owns lanes
+// [LPT t, LPT t + LPT). Ring of NS stages; a stage is one image row of the two fp32 weight rows
+// and of each storage-dtype input, and every scan thread keeps NS rows of its own lanes in
+// flight. The loop is software-pipelined by one step (while step g's new line is exchanged at
+// the barrier, every thread has already pulled step g+1's inputs out of the ring) and unrolled by
+// NS, so ring stages and halo buffers are compile-time. Bookkeeping is incremental: 32-bit row
+// offsets within the plane, plane base pointers set once per plane. A plane starts from h = 0 and
+// a zero halo, so its first step needs no special case (h_0 = z exactly). Lane-major roles
+// (NSTG > 0) launch as many writer threads as scan threads (write_blocks above); the scan warps
+// then synchronise among themselves with named barrier 1.
+template <typename T, unsigned DIR, int ROLE, int LPT, int NS, int SEGB>
 __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p) {
-    using Md = ModeT<MODE, TOUT>;
-    constexpr int NTEN = Md::NTEN;
+    using Rl = RoleT<ROLE>;
+    constexpr int NTEN = Rl::NTEN;
+    constexpr int NSTG = Rl::NSTG;
+    constexpr int KST = SEGB / (int)sizeof(T);   // steps per staging block (a power of two)
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align128(smem_raw);
     const int H = p.H, W = p.W;
     const int rowB = W * (int)sizeof(T);
     const int wrowB = W * 4;
     const int stageB = 2 * wrowB + NTEN * rowB;
-    float* halo = (float*)(smem + (size_t)NS * stageB);   // [2 parity][2 lo/hi][32 warps]
-    // TOUT staging: Md::NSTG blocks of [kTB_STEPS][R] in the storage dtype (the values are
-    // stored in that dtype anyway). R is W rounded up to 32 plus 16 bytes, so every staging row
-    // starts 16-byte aligned (vector stores) and consecutive rows shift the bank pattern.
-    T* stg = (T*)(halo + 128);
+    // halo, per step parity: lo[0..32] (lane 0 of warp w writes lo[w]) and hi[0..32] (lane 31 of
+    // warp w writes hi[w + 1]); hi[0] and lo[nw] are never written and stay zero, so the first
+    // lane's left and the last lane's right neighbour read zero without a test.
+    float* halo = (float*)(smem + (size_t)NS * stageB);   // [2 parity][lo 33 | pad | hi 33 | pad] = 2 x 68
+    uint64_t* bars = (uint64_t*)(halo + 136);             // full[2], free[2]
+    // Staging: two buffers of NSTG blocks [KST][R] in the storage dtype (the values are stored in
+    // that dtype anyway). R is W rounded up to 32 plus 16 bytes: every staging row starts 16-byte
+    // aligned and consecutive rows shift the bank pattern.
+    T* stg = (T*)(bars + 4);
     const int R = ((W + 31) / 32) * 32 + 16 / (int)sizeof(T);
-    // TOUT final: u of the next staging block, prefetched lane-major, 16 bytes per chunk id
-    constexpr int CH = 16 / (int)sizeof(T);          // steps per 16-byte chunk
-    constexpr int CPL = kTB_STEPS / CH;              // chunks per lane segment
-    uint4* ubuf = (uint4*)align128((unsigned char*)(stg + (size_t)Md::NSTG * kTB_STEPS * R));
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    const int j0 = tid * LPT;
-    const bool active = j0 < W;
-    const int sw = (tid >> 2) & 1;
+    const size_t stg_buf = (size_t)NSTG * KST * R;
+    T* ubuf = stg + 2 * stg_buf;   // final lane-major sweep: u of two blocks, [2][W][KST]
+    const int nsc = NSTG > 0 ? (int)blockDim.x / 2 : (int)blockDim.x;
+    const int tid = threadIdx.x;
     const long long HW = (long long)H * W;
     const int nplanes = p.N * p.C;
     const int my_planes = (nplanes - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const long long total = (long long)my_planes * H;
-    const size_t wofs = (size_t)j0 * 4;                                  // this thread in a weight row
-    const size_t tofs = 2 * (size_t)wrowB + (size_t)j0 * sizeof(T);      // ... in the first T row
 
-    // Issue cursor: rows are requested strictly in step order, so plane, row and stage advance
-    // incrementally (no division inside the loop).
-    long long iss_left = total;
-    int iss_i = 0, iss_s = 0, iss_plane = (int)blockIdx.x;
-    const float* iss_wt = nullptr;
-    long long iss_poff = 0;
-    auto iss_plane_setup = [&]() {
-        const int n = iss_plane / p.C, c = iss_plane % p.C;
-        iss_wt = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
-        iss_poff = (long long)iss_plane * HW;
+    for (int k = tid; k < 2 * 68; k += blockDim.x) halo[k] = 0.f;
+    if constexpr (NSTG > 0) {
+        if (tid == 0) {
+            mbar_init(&bars[0], (unsigned)nsc);
+            mbar_init(&bars[1], (unsigned)nsc);
+            mbar_init(&bars[2], blockDim.x - (unsigned)nsc);
+            mbar_init(&bars[3], blockDim.x - (unsigned)nsc);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+    }
+    __syncthreads();
+    if constexpr (NSTG > 0) {
+        if (tid >= nsc) {
+            write_blocks<T, DIR, ROLE, KST>(p, stg, stg_buf, R, bars, ubuf, tid - nsc, (int)blockDim.x - nsc, my_planes);
+            return;
+        }
+    }
+
+    const int lane = tid & 31, warp = tid >> 5;
+    const int j0 = tid * LPT;
+    const bool active = j0 < W;
+    const int sw = (tid >> 2) & 1;
+    const int total = my_planes * H;                               // rows this CTA scans
+    const int dstep = DIR == kTB ? W : -W;                         // row-offset step in scan order
+    const int off0 = (DIR == kTB ? 0 : (H - 1) * W) + j0;          // first row offset of a plane
+    const int r0 = DIR == kTB ? 0 : H - 1;                         // first row of a plane
+    const int rstep = DIR == kTB ? 1 : -1;
+    unsigned char* const wdst = smem + (size_t)j0 * 4;                                 // + stage
+    unsigned char* const tdst = smem + 2 * (size_t)wrowB + (size_t)j0 * sizeof(T);    // + stage
+
+    // ---- issue cursor (rows requested strictly in scan order, NS rows ahead of the consumer)
+    int iss_left = total, iss_rows = H, iss_off = off0, iss_plane = (int)blockIdx.x;
+    const float* iw0 = nullptr;
+    const float* iw2 = nullptr;
+    const T* isrc[NTEN];
+    auto iss_setup = [&]() {
+        const int n = iss_plane / p.C, c = iss_plane - n * p.C;
+        iw0 = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
+        iw2 = iw0 + HW;
+        const long long po = (long long)iss_plane * HW;
+        int t = 0;
+        if (Rl::XL) {
+            isrc[t++] = (const T*)p.x + po;
+            isrc[t++] = (const T*)p.lam + po;
+        } else {
+            isrc[t++] = (const T*)p.z + po;
+        }
+        if (Rl::ACCIN) isrc[t++] = (const T*)p.acc + po;
+        if (Rl::URING) isrc[t++] = (const T*)p.u + po;
     };
-    auto issue = [&]() {
+    auto issue = [&](int s) {   // s: compile-time after unrolling
         if (iss_left > 0) {
             if (active) {
-                const int r = DIR == kTB ? iss_i : H - 1 - iss_i;
-                unsigned char* st = smem + (size_t)iss_s * stageB;
-                const long long ro = (long long)r * W + j0;
-                copy_lanes<float, LPT>(st + wofs, iss_wt + ro, sw);
-                copy_lanes<float, LPT>(st + wrowB + wofs, iss_wt + HW + ro, sw);
-                const long long off = iss_poff + ro;
-                unsigned char* sd = st + tofs;
-                int t = 0;
-                if (Md::XL) {
-                    copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.x + off, sw);
-                    copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.lam + off, sw);
-                } else {
-                    copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.z + off, sw);
-                }
-                if (Md::ACCIN) copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.acc + off, sw);
-                if (Md::URING) copy_lanes<T, LPT>(sd + (t++) * rowB, (const T*)p.u + off, sw);
+                unsigned char* ws = wdst + (size_t)s * stageB;
+                copy_lanes<float, LPT>(ws, iw0 + iss_off, sw);
+                copy_lanes<float, LPT>(ws + wrowB, iw2 + iss_off, sw);
+                unsigned char* ts = tdst + (size_t)s * stageB;
+#pragma unroll
+                for (int t = 0; t < NTEN; ++t) copy_lanes<T, LPT>(ts + t * rowB, isrc[t] + iss_off, sw);
             }
             --iss_left;
-            if (++iss_s == NS) iss_s = 0;
-            if (++iss_i == H) {
-                iss_i = 0;
+            iss_off += dstep;
+            if (--iss_rows == 0) {
+                iss_rows = H;
+                iss_off = off0;
                 iss_plane += (int)gridDim.x;
-                if (iss_plane < nplanes) iss_plane_setup();
+                if (iss_plane < nplanes) iss_setup();
             }
         }
         cp_async_commit();   // always one group per call, so the wait counts stay uniform
     };
-    // Final transposed-output sweep: copy u of the staging block that contains scan row `row`
-    // of plane offset `po` into ubuf (same chunk ids as the flush). The copies join the ring's
-    // next commit group, which is complete at least kTB_STEPS - NS steps before the flush.
-    auto prefetch_u = [&](int row, long long po) {
-        if constexpr (TOUT && Md::FINAL) {
-            const int s_base = row - row % kTB_STEPS;
-            const int nvalid = min(kTB_STEPS, H - s_base);
-            const int q = tid % CPL, jstep = (int)blockDim.x / CPL;
-            if (q * CH < nvalid) {
-                const T* src = (const T*)p.u + po + (long long)(tid / CPL) * H + s_base + q * CH;
-                for (int j = tid / CPL; j < W; j += jstep, src += (long long)jstep * H)
-                    cp_async<16>(ubuf + j * CPL + q, src);
-            }
-        }
-    };
-    prefetch_u(DIR == kTB ? 0 : H - 1, (long long)blockIdx.x * HW);
-    iss_plane_setup();
+    iss_setup();
 #pragma unroll
-    for (int q = 0; q < NS; ++q) issue();
+    for (int s = 0; s < NS; ++s) issue(s);
 
-    // inputs of the next step, already out of shared memory
+    // ---- inputs of the next step, already out of shared memory (inactive threads keep zeros,
+    //      which make their lanes compute h = 0)
     float nz[LPT], nacc[LPT], nu[LPT], nw0[LPT], nw2[LPT];
 #pragma unroll
     for (int e = 0; e < LPT; ++e) nz[e] = nacc[e] = nu[e] = nw0[e] = nw2[e] = 0.f;
-    int fs = 0;   // consumer stage
-    auto fetch = [&]() {
+    auto fetch = [&](int s) {   // s: compile-time after unrolling
         cp_async_wait<NS - 1>();
         if (active) {
-            const unsigned char* st = smem + (size_t)fs * stageB;
-            read_lanes<float, LPT>(st + wofs, nw0, sw);
-            read_lanes<float, LPT>(st + wrowB + wofs, nw2, sw);
-            const unsigned char* sd = st + tofs;
-            read_lanes<T, LPT>(sd, nz, sw);
-            if (Md::XL) {
+            const unsigned char* ws = wdst + (size_t)s * stageB;
+            read_lanes<float, LPT>(ws, nw0, sw);
+            read_lanes<float, LPT>(ws + wrowB, nw2, sw);
+            const unsigned char* ts = tdst + (size_t)s * stageB;
+            read_lanes<T, LPT>(ts, nz, sw);
+            if (Rl::XL) {
                 float l2[LPT];
-                read_lanes<T, LPT>(sd + rowB, l2, sw);
+                read_lanes<T, LPT>(ts + rowB, l2, sw);
 #pragma unroll
                 for (int e = 0; e < LPT; ++e) nz[e] *= l2[e];     // z = x * lam
             }
-            int t = Md::XL ? 2 : 1;
-            if (Md::ACCIN) read_lanes<T, LPT>(sd + (t++) * rowB, nacc, sw);
-            if (Md::URING) read_lanes<T, LPT>(sd + (t++) * rowB, nu, sw);
+            int t = Rl::XL ? 2 : 1;
+            if (Rl::ACCIN) read_lanes<T, LPT>(ts + (t++) * rowB, nacc, sw);
+            if (Rl::URING) read_lanes<T, LPT>(ts + (t++) * rowB, nu, sw);
         }
-        if (++fs == NS) fs = 0;
-        issue();   // this thread has consumed its lanes of the stage: refill it NS steps ahead
+        issue(s);   // this thread has consumed its lanes of the stage: refill it NS rows ahead
     };
+    fetch(0);
 
-    fetch();
+    // ---- consumer cursor
+    int c_rows = H, c_off = off0, c_r = r0, c_plane = (int)blockIdx.x;
+    T* oacc = nullptr;
+    T* oy = nullptr;
+    T* oz = nullptr;
+    auto out_setup = [&]() {
+        const long long po = (long long)c_plane * HW;
+        if (Rl::ANAT) oacc = (T*)p.acc + po;
+        if (Rl::YNAT) oy = (T*)p.y + po;
+        if (Rl::ZNAT) oz = (T*)p.z + po;
+    };
+    out_setup();
+    int kblk = 0;        // staging blocks completed by this CTA
+    bool dead = false;   // a hand-off wait timed out: stop waiting
     float h[LPT];
 #pragma unroll
     for (int e = 0; e < LPT; ++e) h[e] = 0.f;
-    int i = 0;                                   // step within the plane
-    long long poff = (long long)blockIdx.x * HW;
-    int plane = (int)blockIdx.x;
-    for (long long g = 0; g < total; ++g) {
-        float cz[LPT], cacc[LPT], cu[LPT], cw0[LPT], cw2[LPT];
-#pragma unroll
-        for (int e = 0; e < LPT; ++e) {
-            cz[e] = nz[e]; cacc[e] = nacc[e]; cu[e] = nu[e]; cw0[e] = nw0[e]; cw2[e] = nw2[e];
-            if (i == 0) h[e] = 0.f;
-        }
-        if constexpr (TOUT && Md::FINAL) {
-            // first step of a staging block (after the first): the previous block was flushed
-            // behind a barrier at the end of the last iteration, so ubuf is free. The copies
-            // join the commit group of this iteration's fetch.
-            const int rc = DIR == kTB ? i : H - 1 - i;
-            const bool starts = DIR == kTB ? rc % kTB_STEPS == 0 : (rc % kTB_STEPS == kTB_STEPS - 1 || rc == H - 1);
-            if (g > 0 && starts) prefetch_u(rc, poff);
-        }
-        // neighbours from the previous step: lane j0-1 and lane j0+LPT
-        const float* hprev = halo + ((g + 1) & 1) * 64;
+
+    auto step = [&](int u) {   // u: position in the unrolled group (compile-time)
+        const float* lo_prev = halo + ((u + 1) & 1) * 68;
+        float* lo_cur = halo + (u & 1) * 68;
         float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
         float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
-        const float edge = lane == 0 ? hprev[32 + warp - 1 + (warp == 0)] : hprev[warp + 1 - (warp == nw - 1)];
-        if (lane == 0) hl = warp > 0 ? edge : 0.f;
-        if (lane == 31) hr = warp < nw - 1 ? edge : 0.f;
+        if (lane == 0) hl = lo_prev[34 + warp];          // hi of the warp to the left (0 for warp 0)
+        if (lane == 31) hr = lo_prev[warp + 1];          // lo of the warp to the right (0 for the last)
         float hn[LPT];
 #pragma unroll
-        for (int e = 0; e < LPT; ++e) hn[e] = 0.f;
+        for (int e = 0; e < LPT; ++e) {
+            const float left = e == 0 ? hl : h[e - 1];
+            const float right = e == LPT - 1 ? hr : h[e + 1];
+            const float w1 = 1.f - nw0[e] - nw2[e];
+            hn[e] = fmaf(nw0[e], left, fmaf(w1, h[e], fmaf(nw2[e], right, nz[e])));
+        }
+        float o[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            o[e] = Rl::ACCIN ? nacc[e] + hn[e] : hn[e];
+            if (Rl::URING) o[e] *= nu[e];
+        }
         if (active) {
-#pragma unroll
-            for (int e = 0; e < LPT; ++e) {
-                hn[e] = cz[e];
-                if (i > 0) {
-                    const float left = e == 0 ? hl : h[e - 1];
-                    const float right = e == LPT - 1 ? hr : h[e + 1];
-                    const float w1 = 1.f - cw0[e] - cw2[e];
-                    hn[e] = fmaf(cw0[e], left, fmaf(w1, h[e], fmaf(cw2[e], right, hn[e])));
-                }
+            if (Rl::ANAT) st_lanes<T, LPT>(oacc + c_off, o);
+            if (Rl::YNAT) st_lanes<T, LPT>(oy + c_off, o);
+            if (Rl::ZNAT) st_lanes<T, LPT>(oz + c_off, nz);
+        }
+        if constexpr (NSTG > 0) {
+            // staging row of this step; wait for the writers to have emptied the buffer (used
+            // two blocks ago) before the block's first row, hand the block over after its last
+            const int rb = c_r & (KST - 1);
+            const bool bstart = DIR == kTB ? rb == 0 : (rb == KST - 1 || c_r == H - 1);
+            const bool bend = DIR == kTB ? (rb == KST - 1 || c_r == H - 1) : rb == 0;
+            const int b = kblk & 1;
+            if (bstart && kblk >= 2 && !dead)
+                dead = !mbar_wait_bounded<false>(&bars[2 + b], (unsigned)((kblk >> 1) - 1) & 1u, p.status);
+            if (active) {
+                T* srow = stg + (size_t)b * stg_buf + (size_t)rb * R + j0;
+                if (Rl::ZSTG) st_lanes<T, LPT>(srow, nz);
+                if (Rl::ASTG) st_lanes<T, LPT>(srow + (Rl::ZSTG ? (size_t)KST * R : 0), o);
             }
-            const int r = DIR == kTB ? i : H - 1 - i;
-            const long long off = poff + (long long)r * W + j0;
-            float o[LPT];
-#pragma unroll
-            for (int e = 0; e < LPT; ++e) {
-                o[e] = Md::ACCIN ? cacc[e] + hn[e] : hn[e];
-                if (Md::URING) o[e] *= cu[e];
-            }
-            if constexpr (TOUT) {
-                T* srow = stg + (size_t)(r % kTB_STEPS) * R + j0;
-                if constexpr (Md::FINAL) {
-                    st_lanes<T, LPT>(srow, o);
-                } else {
-                    st_lanes<T, LPT>(srow, cz);
-                    st_lanes<T, LPT>(srow + kTB_STEPS * R, o);
-                }
-            } else {
-                st_lanes<T, LPT>((T*)(Md::FINAL ? p.y : p.acc) + off, o);
-                if (Md::ZOUT) st_lanes<T, LPT>((T*)p.z + off, cz);
+            if (bend) {
+                mbar_arrive(&bars[b]);
+                ++kblk;
             }
         }
-        float* hcur = halo + (g & 1) * 64;
-        if (lane == 0) hcur[warp] = hn[0];
-        if (lane == 31) hcur[32 + warp] = hn[LPT - 1];
-        if (g + 1 < total) fetch();
-        __syncthreads();
+        // the last row of a plane hands zeros to the next plane's first step
+        const bool last = c_rows == 1;
+        if (lane == 0) lo_cur[warp] = last ? 0.f : hn[0];
+        if (lane == 31) lo_cur[34 + warp + 1] = last ? 0.f : hn[LPT - 1];
+        fetch((u + 1) % NS);
+        if constexpr (NSTG > 0)
+            asm volatile("bar.sync 1, %0;" ::"r"(nsc) : "memory");
+        else
+            __syncthreads();
 #pragma unroll
         for (int e = 0; e < LPT; ++e) h[e] = hn[e];
-        if constexpr (TOUT) {
-            // a staging block is complete: write it lane-major, 16 bytes per chunk
-            const int r = DIR == kTB ? i : H - 1 - i;
-            const bool flush = DIR == kTB ? (r % kTB_STEPS == kTB_STEPS - 1 || r == H - 1) : (r % kTB_STEPS == 0);
-            if (flush) {
-                const int s_base = r - r % kTB_STEPS;
-                const int nvalid = min(kTB_STEPS, H - s_base);
-                // The ring's waits already cover the u copies of a block longer than NS steps
-                // (issued with the block's first step); short blocks and the last step wait here.
-                if constexpr (Md::FINAL)
-                    if (nvalid <= NS || g + 1 >= total) cp_async_wait<0>();
-                // Thread t writes chunk q = t % CPL of lanes t / CPL, t / CPL + T / CPL, ...: a warp
-                // covers 32 / CPL whole lane segments per store; its shared reads are runs of
-                // consecutive lanes in CPL staging rows (R = 4 mod 32: at most two threads per bank).
-                const int q = tid % CPL, jstep = (int)blockDim.x / CPL;
-                if (q * CH < nvalid) {
-                    const long long gstep = (long long)jstep * H;
-                    const T* sp = stg + (size_t)(q * CH) * R + tid / CPL;
-                    const long long g0 = poff + (long long)(tid / CPL) * H + s_base + q * CH;
-                    if constexpr (Md::FINAL) {
-                        T* gp = (T*)p.y + g0;
-                        const uint4* up = ubuf + (tid / CPL) * CPL + q;
-#pragma unroll 4
-                        for (int j = tid / CPL; j < W; j += jstep, sp += jstep, gp += gstep, up += jstep * CPL) {
-                            float v[CH], uu[CH];
-                            ld_lanes<T, CH>(up, uu);
+        c_off += dstep;
+        c_r += rstep;
+        if (--c_rows == 0) {
 #pragma unroll
-                            for (int k = 0; k < CH; ++k) v[k] = Io<T>::ld(sp + k * R) * uu[k];
-                            st_lanes<T, CH>(gp, v);
-                        }
-                    } else {
-                        T* gz = (T*)p.zt + g0;
-                        T* ga = (T*)p.acct + g0;
-                        const size_t second = (size_t)kTB_STEPS * R;
-#pragma unroll 4
-                        for (int j = tid / CPL; j < W; j += jstep, sp += jstep, gz += gstep, ga += gstep) {
-                            float v[CH], va[CH];
+            for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+            c_rows = H;
+            c_off = off0;
+            c_r = r0;
+            c_plane += (int)gridDim.x;
+            if (c_plane < nplanes) out_setup();
+        }
+    };
+    for (int g = 0; g < total; g += NS) {
 #pragma unroll
-                            for (int k = 0; k < CH; ++k) {
-                                v[k] = Io<T>::ld(sp + k * R);
-                                va[k] = Io<T>::ld(sp + second + k * R);
-                            }
-                            st_lanes<T, CH>(gz, v);
-                            st_lanes<T, CH>(ga, va);
-                        }
-                    }
-                }
-                __syncthreads();   // the staging block is reused by the next step
+        for (int u = 0; u < NS; ++u)
+            if (g + u < total) step(u);
+    }
+    cp_async_wait<0>();
+}
+
+// Fixed-width variant of k_vsweep for lines of WL lanes (WL a multiple of 32 * LPT) and scan
+// lengths that are a multiple of 32 (so of NS and of every staging block). With the line width
+// known at compile time every ring, halo and staging address is a per-thread base plus an
+// immediate, and the plane loop is split so that neither cursor tests for a plane change inside
+// the step: per step a scan warp executes little more than its loads, its 6-7 floating-point
+// operations per lane, the neighbour exchange and the barrier. Same roles, layouts and
+// hand-off protocol as k_vsweep.
+template <typename T, unsigned DIR, int ROLE, int LPT, int NS, int SEGB, int WL>
+__global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
+    using Rl = RoleT<ROLE>;
+    constexpr int NTEN = Rl::NTEN;
+    constexpr int NSTG = Rl::NSTG;
+    constexpr int KST = SEGB / (int)sizeof(T);
+    constexpr int NSC = WL / LPT;                         // scan threads
+    constexpr int ROWB = WL * (int)sizeof(T);
+    constexpr int WROWB = WL * 4;
+    constexpr int STAGEB = 2 * WROWB + NTEN * ROWB;
+    constexpr int R = ((WL + 31) / 32) * 32 + 16 / (int)sizeof(T);
+    constexpr int STG_BUF = NSTG * KST * R;               // elements per staging buffer
+    static_assert(WL % (32 * LPT) == 0, "whole warps of active lanes");
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = align128(smem_raw);
+    const int H = p.H;
+    float* halo = (float*)(smem + (size_t)NS * STAGEB);   // [2 parity][lo 33 | pad | hi 33 | pad]
+    uint64_t* bars = (uint64_t*)(halo + 136);
+    T* stg = (T*)(bars + 4);
+    T* ubuf = stg + 2 * STG_BUF;
+    const int tid = threadIdx.x;
+    const long long HW = (long long)H * WL;
+    const int nplanes = p.N * p.C;
+    const int my_planes = (nplanes - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+
+    for (int k = tid; k < 2 * 68; k += blockDim.x) halo[k] = 0.f;
+    if constexpr (NSTG > 0) {
+        if (tid == 0) {
+            mbar_init(&bars[0], (unsigned)NSC);
+            mbar_init(&bars[1], (unsigned)NSC);
+            mbar_init(&bars[2], blockDim.x - (unsigned)NSC);
+            mbar_init(&bars[3], blockDim.x - (unsigned)NSC);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+    }
+    __syncthreads();
+    if constexpr (NSTG > 0) {
+        if (tid >= NSC) {
+            write_blocks<T, DIR, ROLE, KST>(p, stg, (size_t)STG_BUF, R, bars, ubuf, tid - NSC, (int)blockDim.x - NSC,
+                                            my_planes);
+            return;
+        }
+    }
+
+    const int lane = tid & 31, warp = tid >> 5;
+    const int j0 = tid * LPT;
+    const int sw = (tid >> 2) & 1;
+    constexpr int DSTEP = DIR == kTB ? WL : -WL;
+    const int off0 = (DIR == kTB ? 0 : (H - 1) * WL) + j0;
+    unsigned char* const wdst = smem + (size_t)j0 * 4;
+    unsigned char* const tdst = smem + 2 * (size_t)WROWB + (size_t)j0 * sizeof(T);
+
+    // ---- issue cursor: plane bases and a 32-bit row offset
+    int iss_off = off0;
+    const float* iw0 = nullptr;
+    const float* iw2 = nullptr;
+    const T* isrc[NTEN];
+    auto iss_setup = [&](int plane) {
+        const int n = plane / p.C, c = plane - n * p.C;
+        iw0 = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
+        iw2 = iw0 + HW;
+        const long long po = (long long)plane * HW;
+        int t = 0;
+        if (Rl::XL) {
+            isrc[t++] = (const T*)p.x + po;
+            isrc[t++] = (const T*)p.lam + po;
+        } else {
+            isrc[t++] = (const T*)p.z + po;
+        }
+        if (Rl::ACCIN) isrc[t++] = (const T*)p.acc + po;
+        if (Rl::URING) isrc[t++] = (const T*)p.u + po;
+        iss_off = off0;
+    };
+    auto issue = [&](int s, bool live) {   // s compile-time; live: uniform
+        if (live) {
+            unsigned char* ws = wdst + s * STAGEB;
+            copy_lanes<float, LPT>(ws, iw0 + iss_off, sw);
+            copy_lanes<float, LPT>(ws + WROWB, iw2 + iss_off, sw);
+            unsigned char* ts = tdst + s * STAGEB;
+#pragma unroll
+            for (int t = 0; t < NTEN; ++t) copy_lanes<T, LPT>(ts + t * ROWB, isrc[t] + iss_off, sw);
+            iss_off += DSTEP;
+        }
+        cp_async_commit();
+    };
+    float nz[LPT], nacc[LPT], nu[LPT], nw0[LPT], nw2[LPT];
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) nz[e] = nacc[e] = nu[e] = nw0[e] = nw2[e] = 0.f;
+    auto fetch = [&](int s, bool live) {
+        cp_async_wait<NS - 1>();
+        const unsigned char* ws = wdst + s * STAGEB;
+        read_lanes<float, LPT>(ws, nw0, sw);
+        read_lanes<float, LPT>(ws + WROWB, nw2, sw);
+        const unsigned char* ts = tdst + s * STAGEB;
+        read_lanes<T, LPT>(ts, nz, sw);
+        if (Rl::XL) {
+            float l2[LPT];
+            read_lanes<T, LPT>(ts + ROWB, l2, sw);
+#pragma unroll
+            for (int e = 0; e < LPT; ++e) nz[e] *= l2[e];
+        }
+        int t = Rl::XL ? 2 : 1;
+        if (Rl::ACCIN) read_lanes<T, LPT>(ts + (t++) * ROWB, nacc, sw);
+        if (Rl::URING) read_lanes<T, LPT>(ts + (t++) * ROWB, nu, sw);
+        issue(s, live);
+    };
+
+    // ---- consumer state
+    int c_off = off0;
+    T* oacc = nullptr;
+    T* oy = nullptr;
+    T* oz = nullptr;
+    auto out_setup = [&](int plane) {
+        const long long po = (long long)plane * HW;
+        if (Rl::ANAT) oacc = (T*)p.acc + po;
+        if (Rl::YNAT) oy = (T*)p.y + po;
+        if (Rl::ZNAT) oz = (T*)p.z + po;
+        c_off = off0;
+    };
+    int kblk = 0;
+    bool dead = false;
+    float h[LPT];
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+
+    // one step: i = step within the plane (its low bits give the staging row), u = position in
+    // the unrolled group, last = last row of the plane, live = the refill has a row to fetch
+    auto step = [&](int i, int u, bool last, bool live) {
+        const float* lo_prev = halo + ((u + 1) & 1) * 68;
+        float* lo_cur = halo + (u & 1) * 68;
+        float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
+        float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
+        if (lane == 0) hl = lo_prev[34 + warp];
+        if (lane == 31) hr = lo_prev[warp + 1];
+        float hn[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            const float left = e == 0 ? hl : h[e - 1];
+            const float right = e == LPT - 1 ? hr : h[e + 1];
+            const float w1 = 1.f - nw0[e] - nw2[e];
+            hn[e] = fmaf(nw0[e], left, fmaf(w1, h[e], fmaf(nw2[e], right, nz[e])));
+        }
+        float o[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            o[e] = Rl::ACCIN ? nacc[e] + hn[e] : hn[e];
+            if (Rl::URING) o[e] *= nu[e];
+        }
+        if (Rl::ANAT) st_lanes<T, LPT>(oacc + c_off, o);
+        if (Rl::YNAT) st_lanes<T, LPT>(oy + c_off, o);
+        if (Rl::ZNAT) st_lanes<T, LPT>(oz + c_off, nz);
+        if constexpr (NSTG > 0) {
+            const int ib = i & (KST - 1);
+            const int rb = DIR == kTB ? ib : KST - 1 - ib;
+            const int b = kblk & 1;
+            if (ib == 0 && kblk >= 2 && !dead)
+                dead = !mbar_wait_bounded<false>(&bars[2 + b], (unsigned)((kblk >> 1) - 1) & 1u, p.status);
+            T* srow = stg + b * STG_BUF + rb * R + j0;
+            if (Rl::ZSTG) st_lanes<T, LPT>(srow, nz);
+            if (Rl::ASTG) st_lanes<T, LPT>(srow + (Rl::ZSTG ? KST * R : 0), o);
+            if (ib == KST - 1) {
+                mbar_arrive(&bars[b]);
+                ++kblk;
             }
         }
-        if (++i == H) {
-            i = 0;
-            plane += (int)gridDim.x;
-            poff = (long long)plane * HW;
+        if (lane == 0) lo_cur[warp] = last ? 0.f : hn[0];
+        if (lane == 31) lo_cur[34 + warp + 1] = last ? 0.f : hn[LPT - 1];
+        fetch((u + 1) % NS, live);
+        if constexpr (NSTG > 0)
+            asm volatile("bar.sync 1, %0;" ::"n"(NSC) : "memory");
+        else
+            __syncthreads();
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+        c_off += DSTEP;
+    };
+
+    // Ring protocol: rows 0..NS-1 are issued up front; the fetch of step i (which reads row i + 1)
+    // refills the stage it frees with row i + 1 + NS. So in a plane, steps 0..H-NS-2 refill with
+    // this plane's rows and steps H-NS-1..H-1 with the next plane's rows 0..NS (the same stream
+    // the prologue starts).
+    int plane = (int)blockIdx.x;
+    iss_setup(plane);
+#pragma unroll
+    for (int s = 0; s < NS; ++s) issue(s, true);
+    fetch(0, true);
+    for (int pl = 0; pl < my_planes; ++pl, plane += (int)gridDim.x) {
+        out_setup(plane);
+        const bool more = pl + 1 < my_planes;
+        int i = 0;
+        for (; i < H - 2 * NS; i += NS) {
+#pragma unroll
+            for (int u = 0; u < NS; ++u) step(i + u, u, false, true);
         }
+#pragma unroll
+        for (int u = 0; u < NS; ++u) {
+            if (u == NS - 1 && more) iss_setup(plane + (int)gridDim.x);
+            step(i + u, u, false, u < NS - 1 || more);
+        }
+        i += NS;
+#pragma unroll
+        for (int u = 0; u < NS; ++u) step(i + u, u, u == NS - 1, more);
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) h[e] = 0.f;
     }
     cp_async_wait<0>();
 }
@@ -672,19 +1023,36 @@ __global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsw
 }
 
 // ================================================================== host side
-constexpr size_t kSmemBudget = 225 * 1024;
+constexpr size_t kSmemBudget = 225 * 1024;   // dynamic shared memory of one CTA
+constexpr size_t kSmemSM = 228 * 1024;       // shared memory of one SM (1 KB of it reserved per CTA)
 
-int ntensors(int mode, bool tout = false) {
+int ntensors(int mode) {   // horizontal column-tile sweep
     switch (mode) {
-    case M_FIRST: return tout ? ModeT<M_FIRST, true>::NTEN : ModeT<M_FIRST>::NTEN;
+    case M_FIRST: return ModeT<M_FIRST>::NTEN;
     case M_ONLY: return ModeT<M_ONLY>::NTEN;
-    case M_MID: return tout ? ModeT<M_MID, true>::NTEN : ModeT<M_MID>::NTEN;
-    default: return tout ? ModeT<M_LAST, true>::NTEN : ModeT<M_LAST>::NTEN;
+    case M_MID: return ModeT<M_MID>::NTEN;
+    default: return ModeT<M_LAST>::NTEN;
     }
 }
-int nstaged(int mode, bool tout) {
-    if (!tout) return 0;
-    return (mode == M_LAST || mode == M_ONLY) ? 1 : 2;
+struct RoleInfo {
+    int nten, nstg, ystg, ns_a, seg_a, ns_b, seg_b;
+};
+template <int ROLE> constexpr RoleInfo role_info_t() {
+    using Rl = RoleT<ROLE>;
+    return {Rl::NTEN, Rl::NSTG, Rl::YSTG ? 1 : 0, Rl::NS_A, Rl::SEG_A, Rl::NS_B, Rl::SEG_B};
+}
+RoleInfo role_info(int role) {
+    switch (role) {
+    case R_FIRST: return role_info_t<R_FIRST>();
+    case R_ONLY: return role_info_t<R_ONLY>();
+    case R_MID: return role_info_t<R_MID>();
+    case R_LAST: return role_info_t<R_LAST>();
+    case R_SZ: return role_info_t<R_SZ>();
+    case R_SA: return role_info_t<R_SA>();
+    case R_SZA: return role_info_t<R_SZA>();
+    case R_SY: return role_info_t<R_SY>();
+    default: return role_info_t<R_ZSA>();
+    }
 }
 
 int mode_of(int v, int D) {
@@ -701,22 +1069,43 @@ int v_lanes(const Problem& P) {
     return lpt;
 }
 int v_threads(const Problem& P) { return std::max(32, ((P.W / v_lanes(P) + 31) / 32) * 32); }
-size_t v_smem(const Problem& P, int mode, int ns, bool tout) {
+int v_block_threads(const Problem& P, int role) { return (role_info(role).nstg ? 2 : 1) * v_threads(P); }
+int v_max_threads(const Problem& P) { return v_lanes(P) == 8 ? 512 : 1024; }
+size_t v_smem(const Problem& P, int role, int ns, int segb) {
+    const RoleInfo ri = role_info(role);
     const size_t R = ((size_t)(P.W + 31) / 32) * 32 + 16 / P.esize();
-    const bool ubuf = tout && (mode == M_LAST || mode == M_ONLY);
-    return 128 + (size_t)ns * (2 * (size_t)P.W * 4 + (size_t)ntensors(mode, tout) * P.W * P.esize()) + 512 +
-           (size_t)nstaged(mode, tout) * kTB_STEPS * R * P.esize() + 128 +
-           (ubuf ? (size_t)P.W * kTB_STEPS * P.esize() : 0);
+    const size_t kst = (size_t)segb / P.esize();
+    return 128 + (size_t)ns * (2 * (size_t)P.W * 4 + (size_t)ri.nten * P.W * P.esize()) + 2 * 68 * 4 + 32 +
+           2 * (size_t)ri.nstg * kst * R * P.esize() + (ri.ystg ? 2 * (size_t)P.W * kst * P.esize() : 0);
 }
-// 4 stages when they fit; 2 when there are more planes than SMs and the shorter ring lets twice
-// as many CTAs (planes) share an SM, which hides more of the per-step latency.
-int v_stages(const Problem& P, int mode, bool tout = false) {
-    const size_t s4 = v_smem(P, mode, 4, tout), s2 = v_smem(P, mode, 2, tout);
-    if (s2 > kSmemBudget) return 0;
-    if (s4 > kSmemBudget) return 2;
-    const bool many = (long long)P.N * P.C > device_sm_count();
-    if (many && kSmemBudget / s2 >= 2 * (kSmemBudget / s4)) return 2;
-    return 4;
+int ctas_per_sm(size_t smem) { return smem > kSmemBudget ? 0 : (int)(kSmemSM / (smem + 1024)); }
+
+// Ring depth and staging segment of a vertical sweep; ns == 0: not supported.
+//  - no staged output: 4 stages when they fit; 2 when there are more planes than SMs and the
+//    shorter ring lets twice as many CTAs (planes) share an SM, which hides more of the per-step
+//    latency;
+//  - staged output: configuration A or B of the role, whichever runs more of the planes at once
+//    (A on a tie).
+struct VCfg {
+    int ns, segb;
+};
+VCfg v_config(const Problem& P, int role) {
+    const RoleInfo ri = role_info(role);
+    if (ri.nstg == 0) {
+        const size_t s4 = v_smem(P, role, 4, 16), s2 = v_smem(P, role, 2, 16);
+        if (s2 > kSmemBudget) return {0, 16};
+        if (s4 > kSmemBudget) return {2, 16};
+        const bool many = (long long)P.N * P.C > device_sm_count();
+        if (many && kSmemBudget / s2 >= 2 * (kSmemBudget / s4)) return {2, 16};
+        return {4, 16};
+    }
+    if (v_block_threads(P, role) > v_max_threads(P)) return {0, 0};
+    const long long planes = (long long)P.N * P.C, sms = device_sm_count();
+    const int need = (int)std::min<long long>(64, (planes + sms - 1) / sms);
+    const int ua = std::min(ctas_per_sm(v_smem(P, role, ri.ns_a, ri.seg_a)), need);
+    const int ub = std::min(ctas_per_sm(v_smem(P, role, ri.ns_b, ri.seg_b)), need);
+    if (ua == 0 && ub == 0) return {0, 0};
+    return ua >= ub ? VCfg{ri.ns_a, ri.seg_a} : VCfg{ri.ns_b, ri.seg_b};
 }
 
 // ---- horizontal geometry: threads, rows per thread (as instantiated), padded rows, ring depth
@@ -758,32 +1147,6 @@ int sweep_grid(const Problem& P, K kern, int threads, size_t smem) {
     return (int)std::min<long long>((long long)per_sm * device_sm_count(), (long long)P.N * P.C);
 }
 
-template <typename T, unsigned DIR, int MODE, bool TOUT, int LPT, int NS>
-cudaError_t launch_v4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
-    const size_t smem = v_smem(P, MODE, NS, TOUT);
-    auto kern = k_vsweep<T, DIR, MODE, LPT, NS, TOUT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    const int grid = sweep_grid(P, kern, v_threads(P), smem);
-    launch_begin(st);
-    k_vsweep<T, DIR, MODE, LPT, NS, TOUT><<<grid, v_threads(P), smem, st>>>(a);
-    launch_end(st);
-    return cudaGetLastError();
-}
-
-template <typename T, unsigned DIR, int MODE, bool TOUT, int LPT>
-cudaError_t launch_v3(const Problem& P, const SweepArgs& a, cudaStream_t st) {
-    return v_stages(P, MODE, TOUT) == 4 ? launch_v4<T, DIR, MODE, TOUT, LPT, 4>(P, a, st)
-                                        : launch_v4<T, DIR, MODE, TOUT, LPT, 2>(P, a, st);
-}
-
-template <typename T, unsigned DIR, int MODE, bool TOUT = false>
-cudaError_t launch_v(const Problem& P, const SweepArgs& a, cudaStream_t st) {
-    return v_lanes(P) == 4 ? launch_v3<T, DIR, MODE, TOUT, 4>(P, a, st)
-                           : launch_v3<T, DIR, MODE, TOUT, 8>(P, a, st);
-}
-
 template <typename T, unsigned DIR, int MODE, int G, int NS>
 cudaError_t launch_h4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
     const size_t smem = h_smem(P, MODE, NS);
@@ -813,50 +1176,153 @@ cudaError_t launch_h(const Problem& P, const SweepArgs& a, cudaStream_t st) {
     }
 }
 
-template <typename T, unsigned DIR>
-cudaError_t launch_dir(const Problem& P, const SweepArgs& a, int mode, cudaStream_t st) {
-    if constexpr (DIR == kTB || DIR == kBT) {
-        switch (mode) {
-        case M_FIRST: return launch_v<T, DIR, M_FIRST>(P, a, st);
-        case M_ONLY: return launch_v<T, DIR, M_ONLY>(P, a, st);
-        case M_MID: return launch_v<T, DIR, M_MID>(P, a, st);
-        default: return launch_v<T, DIR, M_LAST>(P, a, st);
-        }
+
+template <typename T, unsigned DIR, int ROLE, int LPT, int NS, int SEGB>
+cudaError_t launch_v4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    const size_t smem = v_smem(P, ROLE, NS, SEGB);
+    const int threads = v_block_threads(P, ROLE);
+    auto kern = k_vsweep<T, DIR, ROLE, LPT, NS, SEGB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    const int grid = sweep_grid(P, kern, threads, smem);
+    launch_begin(st);
+    k_vsweep<T, DIR, ROLE, LPT, NS, SEGB><<<grid, threads, smem, st>>>(a);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+template <typename T, unsigned DIR, int ROLE, int LPT>
+cudaError_t launch_v3(const Problem& P, const SweepArgs& a, const VCfg& c, cudaStream_t st) {
+    using Rl = RoleT<ROLE>;
+    if constexpr (Rl::NSTG == 0) {
+        return c.ns == 4 ? launch_v4<T, DIR, ROLE, LPT, 4, 16>(P, a, st) : launch_v4<T, DIR, ROLE, LPT, 2, 16>(P, a, st);
     } else {
-        switch (mode) {
-        case M_FIRST: return launch_h<T, DIR, M_FIRST>(P, a, st);
-        case M_ONLY: return launch_h<T, DIR, M_ONLY>(P, a, st);
-        case M_MID: return launch_h<T, DIR, M_MID>(P, a, st);
-        default: return launch_h<T, DIR, M_LAST>(P, a, st);
-        }
+        return (c.ns == Rl::NS_A && c.segb == Rl::SEG_A) ? launch_v4<T, DIR, ROLE, LPT, Rl::NS_A, Rl::SEG_A>(P, a, st)
+                                                         : launch_v4<T, DIR, ROLE, LPT, Rl::NS_B, Rl::SEG_B>(P, a, st);
+    }
+}
+
+// Fixed-width kernel: 1024-lane lines (the 1024 x 1024 maps in both scan orientations), scan
+// lengths a multiple of 32, 8 lanes per thread.
+constexpr int kFixedLanes = 1024;
+bool use_fixed(const Problem& P) {
+    if (const char* e = getenv("GSPN_NOFIXED"))
+        if (atoi(e) != 0) return false;
+    return P.W == kFixedLanes && P.H % 32 == 0 && P.H >= 32 && v_lanes(P) == 8;
+}
+
+template <typename T, unsigned DIR, int ROLE, int NS, int SEGB>
+cudaError_t launch_w4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    const size_t smem = v_smem(P, ROLE, NS, SEGB);
+    const int threads = v_block_threads(P, ROLE);
+    auto kern = k_vsweep_w<T, DIR, ROLE, 8, NS, SEGB, kFixedLanes>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    const int grid = sweep_grid(P, kern, threads, smem);
+    launch_begin(st);
+    k_vsweep_w<T, DIR, ROLE, 8, NS, SEGB, kFixedLanes><<<grid, threads, smem, st>>>(a);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+template <typename T, unsigned DIR, int ROLE>
+cudaError_t launch_w3(const Problem& P, const SweepArgs& a, const VCfg& c, cudaStream_t st) {
+    using Rl = RoleT<ROLE>;
+    if constexpr (Rl::NSTG == 0) {
+        return c.ns == 4 ? launch_w4<T, DIR, ROLE, 4, 16>(P, a, st) : launch_w4<T, DIR, ROLE, 2, 16>(P, a, st);
+    } else {
+        return (c.ns == Rl::NS_A && c.segb == Rl::SEG_A) ? launch_w4<T, DIR, ROLE, Rl::NS_A, Rl::SEG_A>(P, a, st)
+                                                         : launch_w4<T, DIR, ROLE, Rl::NS_B, Rl::SEG_B>(P, a, st);
+    }
+}
+
+template <typename T, unsigned DIR, int ROLE>
+cudaError_t launch_v(const Problem& P, const SweepArgs& a, cudaStream_t st) {
+    const VCfg c = v_config(P, ROLE);
+    if (c.ns == 0) return cudaErrorNotSupported;
+    if (use_fixed(P)) return launch_w3<T, DIR, ROLE>(P, a, c, st);
+    return v_lanes(P) == 4 ? launch_v3<T, DIR, ROLE, 4>(P, a, c, st) : launch_v3<T, DIR, ROLE, 8>(P, a, c, st);
+}
+
+// A vertical-kernel sweep in scan order `asc` (top->bottom / left->right) or descending.
+template <typename T>
+cudaError_t launch_role(bool asc, const Problem& P, const SweepArgs& a, int role, cudaStream_t st) {
+    switch (role) {
+    case R_FIRST: return asc ? launch_v<T, kTB, R_FIRST>(P, a, st) : launch_v<T, kBT, R_FIRST>(P, a, st);
+    case R_ONLY: return asc ? launch_v<T, kTB, R_ONLY>(P, a, st) : launch_v<T, kBT, R_ONLY>(P, a, st);
+    case R_MID: return asc ? launch_v<T, kTB, R_MID>(P, a, st) : launch_v<T, kBT, R_MID>(P, a, st);
+    case R_LAST: return asc ? launch_v<T, kTB, R_LAST>(P, a, st) : launch_v<T, kBT, R_LAST>(P, a, st);
+    case R_SZ: return asc ? launch_v<T, kTB, R_SZ>(P, a, st) : cudaErrorNotSupported;
+    case R_SA: return asc ? cudaErrorNotSupported : launch_v<T, kBT, R_SA>(P, a, st);
+    case R_SZA: return asc ? launch_v<T, kTB, R_SZA>(P, a, st) : launch_v<T, kBT, R_SZA>(P, a, st);
+    case R_SY: return asc ? launch_v<T, kTB, R_SY>(P, a, st) : launch_v<T, kBT, R_SY>(P, a, st);
+    case R_ZSA: return asc ? cudaErrorNotSupported : launch_v<T, kBT, R_ZSA>(P, a, st);
+    default: return cudaErrorNotSupported;
+    }
+}
+
+template <typename T, unsigned DIR>
+cudaError_t launch_hdir(const Problem& P, const SweepArgs& a, int mode, cudaStream_t st) {
+    switch (mode) {
+    case M_FIRST: return launch_h<T, DIR, M_FIRST>(P, a, st);
+    case M_ONLY: return launch_h<T, DIR, M_ONLY>(P, a, st);
+    case M_MID: return launch_h<T, DIR, M_MID>(P, a, st);
+    default: return launch_h<T, DIR, M_LAST>(P, a, st);
     }
 }
 
 size_t table_floats(const Problem& P) { return (size_t)P.D * P.N * P.Cw * 2 * (size_t)P.HW; }
 
-// The transposed path: when the mask has vertical and horizontal directions and both image
-// axes give 16-byte rows, the last vertical sweep writes z and the partial sum transposed and
-// the horizontal scans run as vertical-style sweeps over those transposed buffers.
+// The transposed path: when the mask has vertical and horizontal directions, both image axes
+// give 16-byte rows and a line fits a CTA with its writer warps (at most 2048 lanes), the
+// vertical sweeps hand z and the partial sum over lane-major and the horizontal scans run as
+// vertical-kernel sweeps over those buffers.
 Problem swapped(const Problem& P) {
     Problem Q = P;
     std::swap(Q.H, Q.W);
     return Q;
 }
-bool tpath(const Problem& P) {
+bool tpath_geometry(const Problem& P) {
     return (P.mask & (kTB | kBT)) && (P.mask & (kLR | kRL)) && (P.H * P.esize()) % 16 == 0 &&
-           (P.W * P.esize()) % 16 == 0 && P.H <= 4096;
+           (P.W * P.esize()) % 16 == 0 && P.H <= 2048 && P.W <= 2048;
 }
 int n_vertical(const Problem& P) { return ((P.mask & kTB) ? 1 : 0) + ((P.mask & kBT) ? 1 : 0); }
 
-template <typename T, unsigned DIR>
-cudaError_t launch_vt(const Problem& P, const SweepArgs& a, int mode, bool tout, cudaStream_t st) {
-    if (!tout) return launch_dir<T, DIR>(P, a, mode, st);
-    switch (mode) {
-    case M_FIRST: return launch_v<T, DIR, M_FIRST, true>(P, a, st);
-    case M_MID: return launch_v<T, DIR, M_MID, true>(P, a, st);
-    case M_LAST: return launch_v<T, DIR, M_LAST, true>(P, a, st);
-    default: return cudaErrorNotSupported;
+// How the vertical sweeps hand their results to the horizontal ones on the transposed path:
+//  1: TB writes the partial sum scan-major and z lane-major; BT recomputes z from x and lambda,
+//     adds its scan and writes the partial sum lane-major (one staged output each);
+//  2: TB writes z and the partial sum scan-major; BT reads both and writes both lane-major.
+// With one vertical direction it writes both lane-major.
+int tplan() {
+    if (const char* e = getenv("GSPN_TPLAN")) return atoi(e) == 2 ? 2 : 1;
+    return 1;
+}
+
+// Role of visit v (direction d).
+int visit_role(const Problem& P, unsigned d, int v, bool tp) {
+    if (!tp) return mode_of(v, P.D);   // R_FIRST..R_LAST coincide with M_FIRST..M_LAST
+    if (is_vertical(d)) {
+        if (n_vertical(P) == 1) return R_SZA;
+        if (tplan() == 2) return v == 0 ? R_FIRST : R_ZSA;
+        return v == 0 ? R_SZ : R_SA;
     }
+    return v == P.D - 1 ? R_SY : R_MID;
+}
+
+// The transposed path is taken when its geometry holds and every one of its sweeps fits a CTA;
+// otherwise the horizontal scans fall back to column tiles.
+bool tpath(const Problem& P) {
+    if (!tpath_geometry(P)) return false;
+    const Problem PS = swapped(P);
+    for (int v = 0, k = 0; k < 4; ++k) {
+        const unsigned d = 1u << k;
+        if (!(P.mask & d)) continue;
+        if (v_config(is_vertical(d) ? P : PS, visit_role(P, d, v, true)).ns == 0) return false;
+        ++v;
+    }
+    return true;
 }
 
 template <typename T>
@@ -866,10 +1332,16 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
     const int nV = n_vertical(P);
     WsCarver wc(ws);
     float* table = wc.take<float>(table_floats(P));
-    void* z = P.D > 1 ? wc.take<T>(P.U) : nullptr;
-    void* acc = P.D > 1 ? wc.take<T>(P.U) : nullptr;
-    void* zt = tp ? wc.take<T>(P.U) : nullptr;
-    void* acct = tp ? wc.take<T>(P.U) : nullptr;
+    void *z = nullptr, *acc = nullptr, *zt = nullptr, *acct = nullptr;
+    if (tp) {
+        if (nV == 2 && tplan() == 2) z = wc.take<T>(P.U);
+        if (nV == 2) acc = wc.take<T>(P.U);
+        zt = wc.take<T>(P.U);
+        acct = wc.take<T>(P.U);
+    } else if (P.D > 1) {
+        z = wc.take<T>(P.U);
+        acc = wc.take<T>(P.U);
+    }
     // A1: weight formation for every direction, once per (n, cw) plane
     WeightArgs wa{a, table, P.N, P.Cw, P.H, P.W, P.D, 0, {0u, 0u, 0u, 0u}};
     for (int v = 0, k = 0; k < 4; ++k)
@@ -899,21 +1371,21 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
     int v = 0;
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
-        const int mode = mode_of(v, P.D);
-        SweepArgs args{x, lam, u, table + v * slot_floats, z, acc, y, zt, acct, P.N, P.C, P.H, P.W, P.Cw};
+        SweepArgs args{x, lam, u, table + v * slot_floats, z, acc, y, zt, acct, (unsigned*)ws,
+                       P.N, P.C, P.H, P.W, P.Cw};
+        const int role = visit_role(P, d, v, tp);
+        const bool asc = d == kTB || d == kLR;
         if (is_vertical(d)) {
-            const bool tout = tp && v == nV - 1;
-            e = d == kTB ? launch_vt<T, kTB>(P, args, mode, tout, st) : launch_vt<T, kBT>(P, args, mode, tout, st);
+            e = launch_role<T>(asc, P, args, role, st);
         } else if (tp) {
-            // horizontal scan over the transposed buffers: scan length W, lanes H
+            // horizontal scan over the lane-major buffers: scan length W, lanes H
             args.z = zt;
             args.acc = acct;
             args.H = PS.H;
             args.W = PS.W;
-            const bool tout = v == P.D - 1;
-            e = d == kLR ? launch_vt<T, kTB>(PS, args, mode, tout, st) : launch_vt<T, kBT>(PS, args, mode, tout, st);
+            e = launch_role<T>(asc, PS, args, role, st);
         } else {
-            e = d == kLR ? launch_dir<T, kLR>(P, args, mode, st) : launch_dir<T, kRL>(P, args, mode, st);
+            e = d == kLR ? launch_hdir<T, kLR>(P, args, role, st) : launch_hdir<T, kRL>(P, args, role, st);
         }
         if (e != cudaSuccess) return e;
         ++v;
@@ -929,16 +1401,15 @@ bool sweep_supports(const Problem& P, bool bwd) {
     if (P.W > 4096) return false;
     if ((long long)P.D * P.N * P.Cw > 65535) return false;   // weight-formation grid.y / grid.z
     const bool tp = tpath(P);
-    const int nV = n_vertical(P);
     const Problem PS = swapped(P);
     for (int v = 0, k = 0; k < 4; ++k) {
         const unsigned d = 1u << k;
         if (!(P.mask & d)) continue;
-        const int mode = mode_of(v, P.D);
+        const int role = visit_role(P, d, v, tp);
         bool ok;
-        if (is_vertical(d)) ok = v_stages(P, mode, tp && v == nV - 1) > 0;
-        else if (tp) ok = v_stages(PS, mode, v == P.D - 1) > 0;
-        else ok = P.H <= 1024 && h_stages(P, mode) > 0;
+        if (is_vertical(d)) ok = v_config(P, role).ns > 0;
+        else if (tp) ok = v_config(PS, role).ns > 0;
+        else ok = P.H <= 1024 && h_stages(P, role) > 0;
         if (!ok) return false;
         ++v;
     }
@@ -948,8 +1419,9 @@ bool sweep_supports(const Problem& P, bool bwd) {
 size_t sweep_ws_bytes(const Problem& P, bool bwd) {
     if (bwd) return 0;
     size_t b = 256 + align256(table_floats(P) * sizeof(float));
-    if (P.D > 1) b += 2 * align256((size_t)P.U * P.esize());
-    if (tpath(P)) b += 2 * align256((size_t)P.U * P.esize());
+    const size_t ub = align256((size_t)P.U * P.esize());
+    if (tpath(P)) b += (n_vertical(P) == 2 ? (tplan() == 2 ? 4 : 3) : 2) * ub;
+    else if (P.D > 1) b += 2 * ub;
     return b;
 }
 
