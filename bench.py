@@ -34,7 +34,7 @@ sys.path.insert(0, ROOT)
 import gspn_inputs  # noqa: E402
 
 METRIC = "4-dir GSPN scan fwd ms & achieved HBM GB/s (frac of peak), 1024² B16 C8"
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_highres.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_highres.md")
 
 
 def parse_args():
@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--cpu-planes", type=int, default=24, help="planes of the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch N (small cases for profiler captures; not a bench line)")
     return ap.parse_args()
 
 
@@ -195,14 +197,18 @@ def kernel_source_sha():
 
 
 def committed_traffic(workload):
-    """DRAM bytes per forward from the committed ncu summary, if the kernels are unchanged."""
+    """DRAM traffic per forward from the committed ncu summary (its 'traffic-json:' line), if the
+    kernel sources are unchanged since the capture: (bytes per forward, bytes per launch)."""
     if workload != "highres" or not os.path.exists(TRAFFIC_FILE):
-        return None
+        return None, None
+    d = None
     with open(TRAFFIC_FILE) as f:
-        d = json.load(f)
-    if d.get("source_sha") != kernel_source_sha():
-        return None
-    return d.get("dram_bytes_per_forward")
+        for line in f:
+            if line.startswith("traffic-json:"):
+                d = json.loads(line[len("traffic-json:"):])
+    if not d or d.get("source_sha") != kernel_source_sha():
+        return None, None
+    return d.get("dram_bytes_per_forward"), d.get("dram_bytes_per_launch")
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -217,6 +223,8 @@ def run_libgspn(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
     wl = gspn_inputs.WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.with_(N=args.batch)
     dev = torch.device("cuda", local_rank)
     t = gspn_inputs.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
     x, a, lam, u = t["x"], t["a"], t["lam"], t["u"]
@@ -282,14 +290,18 @@ def run_libgspn(args):
     if launches == len(names) + 1:
         names = ["weights"] + names
     achieved = comp / (kern_ms * 1e-3) / 1e9
+    traffic, per_launch = committed_traffic(wl.name) if not args.batch else (None, None)
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-        "frac": round(achieved / peak, 4), "traffic": committed_traffic(wl.name),
+        "frac": round(achieved / peak, 4), "traffic": traffic,
         "peak_kind": peak_kind,
         "what": (f"whole forward = {launches} launches ({'+'.join(names)}); algorithmic bytes = compulsory "
                  f"x, lam, u, a read once + y written once = {comp} B per forward; time = sum of the launches"),
         "kernels_ms": {n: round(p, 4) for n, p in zip(names, per)} if len(names) == len(per) else [round(p, 4) for p in per],
     }
+    if per_launch and len(per_launch) == len(per):
+        # DRAM bytes each launch moves (ncu) over its event-timed duration
+        roofline["kernels_dram_gbs"] = {n: round(b / (p * 1e-3) / 1e9, 1) for n, b, p in zip(names, per_launch, per)}
 
     # ---- copy ceiling on the same byte volume
     nb = (comp // 2) // 16 * 16

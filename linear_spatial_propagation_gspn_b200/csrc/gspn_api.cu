@@ -1,5 +1,6 @@
 // gspn_api.cu -- the C ABI of libgspn: argument checks, workspace sizing, kernel-family
 // selection and the small utility kernels (copy ceiling, bounded-wait probe).
+#include <atomic>
 #include <stdint.h>
 #include <string.h>
 
@@ -96,9 +97,19 @@ void launch_end(cudaStream_t st) {
     ++g_hooks.launches;
 }
 
+// SM count of the current device, queried once per device (host-side planning asks for it
+// several times per call).
 int device_sm_count() {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (dev >= 0 && dev < 64) cache[dev].store(sms, std::memory_order_relaxed);
     return sms;
 }
 

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -27,82 +28,88 @@ template <> struct Io<__nv_bfloat16> {
     static __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 };
 
+template <> struct Io<__half> {
+    static __device__ __forceinline__ float ld(const __half* p) { return __half2float(*p); }
+    static __device__ __forceinline__ void st(__half* p, float v) { *p = __float2half_rn(v); }
+};
+
 // ------------------------------------------------------------------ vector lanes
-// L consecutive lanes of storage type T (aligned to L elements).
+// Two 16-bit values (bf16 or fp16) packed in a word, to and from floats (round to nearest even).
+template <typename T> __device__ __forceinline__ float2 unpack2(uint32_t w);
+template <> __device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t w) {
+    return __bfloat1622float2(*(const __nv_bfloat162*)&w);
+}
+template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t w) { return __half22float2(*(const __half2*)&w); }
+template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+    const __nv_bfloat162 q = __floats2bfloat162_rn(a, b);
+    return *(const uint32_t*)&q;
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+    const __half2 q = __floats2half2_rn(a, b);
+    return *(const uint32_t*)&q;
+}
+
+// L consecutive lanes of storage type T (float, bf16 or fp16; aligned to L elements).
 template <typename T, int L>
 __device__ __forceinline__ void ld_lanes(const void* ptr, float (&v)[L]) {
-    if constexpr (L == 8) {
-        if constexpr (std::is_same<T, float>::value) {
-            const float4 q0 = *(const float4*)ptr, q1 = *((const float4*)ptr + 1);
-            v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
-            v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
-        } else {
-            const uint4 q = *(const uint4*)ptr;
-            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&w[k]);
-                v[2 * k] = f.x;
-                v[2 * k + 1] = f.y;
-            }
-        }
-    } else if constexpr (std::is_same<T, float>::value) {
+    if constexpr (std::is_same<T, float>::value) {
         if constexpr (L == 1) {
             v[0] = *(const float*)ptr;
         } else if constexpr (L == 2) {
             const float2 q = *(const float2*)ptr;
             v[0] = q.x; v[1] = q.y;
-        } else {
+        } else if constexpr (L == 4) {
             const float4 q = *(const float4*)ptr;
             v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+        } else {
+            const float4 q0 = *(const float4*)ptr, q1 = *((const float4*)ptr + 1);
+            v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
+            v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
         }
     } else {
         if constexpr (L == 1) {
-            v[0] = __bfloat162float(*(const __nv_bfloat16*)ptr);
+            v[0] = Io<T>::ld((const T*)ptr);
         } else if constexpr (L == 2) {
-            const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)ptr);
+            const float2 f = unpack2<T>(*(const uint32_t*)ptr);
             v[0] = f.x; v[1] = f.y;
-        } else {
+        } else if constexpr (L == 4) {
             const uint2 q = *(const uint2*)ptr;
-            const float2 f0 = __bfloat1622float2(*(const __nv_bfloat162*)&q.x);
-            const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162*)&q.y);
+            const float2 f0 = unpack2<T>(q.x), f1 = unpack2<T>(q.y);
             v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+        } else {
+            const uint4 q = *(const uint4*)ptr;
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = unpack2<T>(w[k]);
+                v[2 * k] = f.x;
+                v[2 * k + 1] = f.y;
+            }
         }
     }
 }
 
 template <typename T, int L>
 __device__ __forceinline__ void st_lanes(void* ptr, const float (&v)[L]) {
-    if constexpr (L == 8) {
-        if constexpr (std::is_same<T, float>::value) {
-            *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
-            *((float4*)ptr + 1) = make_float4(v[4], v[5], v[6], v[7]);
-        } else {
-            uint4 q;
-            uint32_t* w = &q.x;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
-                w[k] = *(const uint32_t*)&b;
-            }
-            *(uint4*)ptr = q;
-        }
-    } else if constexpr (std::is_same<T, float>::value) {
+    if constexpr (std::is_same<T, float>::value) {
         if constexpr (L == 1) *(float*)ptr = v[0];
         else if constexpr (L == 2) *(float2*)ptr = make_float2(v[0], v[1]);
-        else *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
+        else if constexpr (L == 4) *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
+        else {
+            *(float4*)ptr = make_float4(v[0], v[1], v[2], v[3]);
+            *((float4*)ptr + 1) = make_float4(v[4], v[5], v[6], v[7]);
+        }
     } else {
         if constexpr (L == 1) {
-            *(__nv_bfloat16*)ptr = __float2bfloat16_rn(v[0]);
+            Io<T>::st((T*)ptr, v[0]);
         } else if constexpr (L == 2) {
-            *(__nv_bfloat162*)ptr = __floats2bfloat162_rn(v[0], v[1]);
+            *(uint32_t*)ptr = pack2<T>(v[0], v[1]);
+        } else if constexpr (L == 4) {
+            *(uint2*)ptr = make_uint2(pack2<T>(v[0], v[1]), pack2<T>(v[2], v[3]));
         } else {
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]);
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(v[2], v[3]);
-            uint2 q;
-            q.x = *(const uint32_t*)&b0;
-            q.y = *(const uint32_t*)&b1;
-            *(uint2*)ptr = q;
+            *(uint4*)ptr = make_uint4(pack2<T>(v[0], v[1]), pack2<T>(v[2], v[3]), pack2<T>(v[4], v[5]),
+                                      pack2<T>(v[6], v[7]));
         }
     }
 }

@@ -54,7 +54,7 @@ struct SweepArgs {
     const void* x;
     const void* lam;
     const void* u;    // scan-major, or lane-major (image layout) for a lane-major final sweep
-    const float* wt;  // weight table of this direction's slot: [N][Cw][2][H][W] fp32 (w0, w2)
+    const void* wt;   // weight table of this direction's slot: [N][Cw][2][H][W] of TableT (w0, w2)
     void* z;          // workspace, storage dtype, scan-major
     void* acc;        // workspace, storage dtype, scan-major
     void* y;          // output (scan-major, or lane-major for a lane-major final sweep)
@@ -66,9 +66,9 @@ struct SweepArgs {
 
 struct WeightArgs {
     const void* a;    // logits [D][N][Cw][3][H][W]
-    float* wt;        // table  [D][N][Cw][2][H][W] (transposed planes: [W][H])
+    void* wt;         // table  [D][N][Cw][2][H][W] of TableT (slots from tslot0 on: [W][H] planes)
     int N, Cw, H, W, D;
-    int plane0;       // first (slot, n, cw) plane handled by the launch
+    int tslot0;       // first slot written transposed (D: none)
     unsigned dirs[4]; // direction bit of each slot
 };
 
@@ -150,77 +150,100 @@ __device__ __forceinline__ void read_lanes(const unsigned char* srcs, float (&v)
 
 
 // ================================================================== weight formation (A1)
+// Table element type: fp32 for fp32 storage, fp16 for bf16 storage. The weights lie in [0, 1],
+// so fp16's 11-bit significand bounds their relative rounding error by 2^-12, far inside the
+// bf16 tolerance (and the sweeps re-derive w1 = 1 - w0 - w2 in fp32, so every row still sums to
+// one); it halves the table's traffic and the weight rows of a sweep's ring.
+template <typename T> struct TableT { using type = float; };
+template <> struct TableT<__nv_bfloat16> { using type = __half; };
+
 // Turns the logits of every (slot, n, cw) plane into the two outer weights w0, w2 of each
-// normalised tridiagonal row; the sweeps re-derive w1 = 1 - w0 - w2, so every row sums to one.
-// Elementwise and memory-bound: one thread per 4 consecutive pixels of a row, accurate expf and
-// IEEE reciprocal. blockIdx.y = plane, so no 64-bit division is needed.
+// normalised tridiagonal row; the sweeps re-derive w1 = 1 - w0 - w2. Elementwise and
+// memory-bound, one launch for all slots. A persistent CTA (256 threads) takes tiles of 32 rows
+// x 128 columns: thread (tx, ty) loads 4 consecutive columns (one vector per logit row) of rows
+// ty, ty + 8, ty + 16, ty + 24, forms the 16 weights (MUFU exponential and reciprocal, the
+// normalisation applied afterwards so every row still sums to one up to a few ulp; the
+// max-shifted form for logits below -40), and writes them in the image layout straight from
+// registers, or, for the transposed slots ([W][H] planes:
+// element (column c, row r) at c * H + r), through a shared-memory tile read column-wise (row
+// stride 129 words: conflict-free) so that the table writes stay coalesced. Needs W % 4 == 0.
+constexpr int kWTileR = 32, kWTileC = 128;
+
 template <typename T>
-__global__ void __launch_bounds__(256) k_sweep_weights(WeightArgs p) {
-    const long long HW = (long long)p.H * p.W;
-    const int plane = p.plane0 + (int)blockIdx.y;      // (slot, n, cw)
-    const int slot = plane / (p.N * p.Cw);
-    const unsigned d = p.dirs[slot];
-    const T* a3 = (const T*)p.a + (long long)plane * 3 * HW;
-    float* wt = p.wt + (long long)plane * 2 * HW;
-    const int quads = (int)(HW / 4);
-    for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < quads; q += gridDim.x * blockDim.x) {
-        const int pix = q * 4;
-        const int r = pix / p.W, c0 = pix - r * p.W;
-        float a0[4], a1[4], a2[4], w0[4], w2[4];
-        ld_lanes<T, 4>(a3 + pix, a0);
-        ld_lanes<T, 4>(a3 + HW + pix, a1);
-        ld_lanes<T, 4>(a3 + 2 * HW + pix, a2);
+__global__ void __launch_bounds__(256) k_weights(WeightArgs p, int tiles_x, int tiles_y, int ntiles) {
+    using WT = typename TableT<T>::type;
+    __shared__ float tile[2][kWTileR][kWTileC + 1];
+    const int H = p.H, W = p.W;
+    const long long HW = (long long)H * W;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    const int per_plane = tiles_x * tiles_y;
+    const int planes_per_slot = p.N * p.Cw;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int plane = t / per_plane, tt = t - plane * per_plane;
+        const int by = tt / tiles_x, bx = tt - by * tiles_x;
+        const int slot = plane / planes_per_slot;
+        const bool vert = is_vertical(p.dirs[slot]);
+        const T* a3 = (const T*)p.a + (long long)plane * 3 * HW;
+        WT* wt = (WT*)p.wt + (long long)plane * 2 * HW;
+        const int r0 = by * kWTileR, c0 = bx * kWTileC;
+        const int c = c0 + 4 * tx;
+        const bool cin = c < W;   // W % 4 == 0: a quad is all in or all out
+        float w0[4][4], w2[4][4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int c = c0 + k;
-            const bool hl = is_vertical(d) ? c > 0 : r > 0;
-            const bool hr = is_vertical(d) ? c < p.W - 1 : r < p.H - 1;
-            const Wts w = lane_weights_acc(a0[k], a1[k], a2[k], hl, hr);
-            w0[k] = w.w0;
-            w2[k] = w.w2;
-        }
-        st_lanes<float, 4>(wt + pix, w0);
-        st_lanes<float, 4>(wt + HW + pix, w2);
-    }
-}
-
-// Same table, written transposed ([W][H] per plane: element (column c, row r) at c*H + r) for
-// horizontal scans run over transposed buffers. 32x32 pixel tiles through shared memory keep
-// both the logit reads and the table writes coalesced.
-template <typename T>
-__global__ void __launch_bounds__(256) k_sweep_weights_t(WeightArgs p) {
-    __shared__ float tile[2][32][33];
-    const long long HW = (long long)p.H * p.W;
-    const int plane = p.plane0 + (int)blockIdx.z;
-    const int slot = plane / (p.N * p.Cw);
-    const unsigned d = p.dirs[slot];
-    const T* a3 = (const T*)p.a + (long long)plane * 3 * HW;
-    float* wt = p.wt + (long long)plane * 2 * HW;
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8
+            const int r = r0 + ty + 8 * k;
+            float l0[4] = {0.f, 0.f, 0.f, 0.f}, l1[4] = {0.f, 0.f, 0.f, 0.f}, l2[4] = {0.f, 0.f, 0.f, 0.f};
+            const bool in = cin && r < H;
+            if (in) {
+                const long long q = (long long)r * W + c;
+                ld_lanes<T, 4>(a3 + q, l0);
+                ld_lanes<T, 4>(a3 + HW + q, l1);
+                ld_lanes<T, 4>(a3 + 2 * HW + q, l2);
+            }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int r = r0 + ty + 8 * k, c = c0 + tx;
-        float w0 = 0.f, w2 = 0.f;
-        if (r < p.H && c < p.W) {
-            const long long q = (long long)r * p.W + c;
-            const bool hl = is_vertical(d) ? c > 0 : r > 0;
-            const bool hr = is_vertical(d) ? c < p.W - 1 : r < p.H - 1;
-            const Wts w = lane_weights_acc(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q), Io<T>::ld(a3 + 2 * HW + q), hl, hr);
-            w0 = w.w0;
-            w2 = w.w2;
+            for (int e = 0; e < 4; ++e) {
+                const int cc = c + e;
+                const bool hl = vert ? cc > 0 : r > 0;
+                const bool hr = vert ? cc < W - 1 : r < H - 1;
+                Wts w = lane_weights_fast_nocheck(l0[e], l1[e], l2[e], hl, hr);
+                if (weights_need_shift(l0[e], l1[e], l2[e], hl, hr)) w = weights_shifted(l0[e], l1[e], l2[e], hl, hr);
+                w0[k][e] = in ? w.w0 : 0.f;
+                w2[k][e] = in ? w.w2 : 0.f;
+            }
         }
-        tile[0][ty + 8 * k][tx] = w0;
-        tile[1][ty + 8 * k][tx] = w2;
-    }
-    __syncthreads();
+        if (slot < p.tslot0) {   // image layout, straight from registers
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int c = c0 + ty + 8 * k, r = r0 + tx;
-        if (r < p.H && c < p.W) {
-            const long long q = (long long)c * p.H + r;
-            wt[q] = tile[0][tx][ty + 8 * k];
-            wt[HW + q] = tile[1][tx][ty + 8 * k];
+            for (int k = 0; k < 4; ++k) {
+                const int r = r0 + ty + 8 * k;
+                if (cin && r < H) {
+                    const long long q = (long long)r * W + c;
+                    st_lanes<WT, 4>(wt + q, w0[k]);
+                    st_lanes<WT, 4>(wt + HW + q, w2[k]);
+                }
+            }
+        } else {                 // transposed planes (uniform per tile: the barriers are safe)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    tile[0][ty + 8 * k][4 * tx + e] = w0[k][e];
+                    tile[1][ty + 8 * k][4 * tx + e] = w2[k][e];
+                }
+            __syncthreads();
+            // warp ty writes columns ty, ty + 8, ...: 32 consecutive rows each (lane = row)
+            const int r = r0 + tx;
+            if (r < H) {
+#pragma unroll 4
+                for (int cc = ty; cc < kWTileC; cc += 8) {
+                    const int col = c0 + cc;
+                    if (col < W) {
+                        const long long q = (long long)col * H + r;
+                        Io<WT>::st(wt + q, tile[0][tx][cc]);
+                        Io<WT>::st(wt + HW + q, tile[1][tx][cc]);
+                    }
+                }
+            }
+            __syncthreads();
         }
     }
 }
@@ -401,7 +424,8 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
     unsigned char* smem = align128(smem_raw);
     const int H = p.H, W = p.W;
     const int rowB = W * (int)sizeof(T);
-    const int wrowB = W * 4;
+    using WT = typename TableT<T>::type;
+    const int wrowB = W * (int)sizeof(WT);
     const int stageB = 2 * wrowB + NTEN * rowB;
     // halo, per step parity: lo[0..32] (lane 0 of warp w writes lo[w]) and hi[0..32] (lane 31 of
     // warp w writes hi[w + 1]); hi[0] and lo[nw] are never written and stay zero, so the first
@@ -448,17 +472,17 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
     const int off0 = (DIR == kTB ? 0 : (H - 1) * W) + j0;          // first row offset of a plane
     const int r0 = DIR == kTB ? 0 : H - 1;                         // first row of a plane
     const int rstep = DIR == kTB ? 1 : -1;
-    unsigned char* const wdst = smem + (size_t)j0 * 4;                                 // + stage
+    unsigned char* const wdst = smem + (size_t)j0 * sizeof(WT);                        // + stage
     unsigned char* const tdst = smem + 2 * (size_t)wrowB + (size_t)j0 * sizeof(T);    // + stage
 
     // ---- issue cursor (rows requested strictly in scan order, NS rows ahead of the consumer)
     int iss_left = total, iss_rows = H, iss_off = off0, iss_plane = (int)blockIdx.x;
-    const float* iw0 = nullptr;
-    const float* iw2 = nullptr;
+    const WT* iw0 = nullptr;
+    const WT* iw2 = nullptr;
     const T* isrc[NTEN];
     auto iss_setup = [&]() {
         const int n = iss_plane / p.C, c = iss_plane - n * p.C;
-        iw0 = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
+        iw0 = (const WT*)p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
         iw2 = iw0 + HW;
         const long long po = (long long)iss_plane * HW;
         int t = 0;
@@ -475,8 +499,8 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
         if (iss_left > 0) {
             if (active) {
                 unsigned char* ws = wdst + (size_t)s * stageB;
-                copy_lanes<float, LPT>(ws, iw0 + iss_off, sw);
-                copy_lanes<float, LPT>(ws + wrowB, iw2 + iss_off, sw);
+                copy_lanes<WT, LPT>(ws, iw0 + iss_off, sw);
+                copy_lanes<WT, LPT>(ws + wrowB, iw2 + iss_off, sw);
                 unsigned char* ts = tdst + (size_t)s * stageB;
 #pragma unroll
                 for (int t = 0; t < NTEN; ++t) copy_lanes<T, LPT>(ts + t * rowB, isrc[t] + iss_off, sw);
@@ -505,8 +529,8 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
         cp_async_wait<NS - 1>();
         if (active) {
             const unsigned char* ws = wdst + (size_t)s * stageB;
-            read_lanes<float, LPT>(ws, nw0, sw);
-            read_lanes<float, LPT>(ws + wrowB, nw2, sw);
+            read_lanes<WT, LPT>(ws, nw0, sw);
+            read_lanes<WT, LPT>(ws + wrowB, nw2, sw);
             const unsigned char* ts = tdst + (size_t)s * stageB;
             read_lanes<T, LPT>(ts, nz, sw);
             if (Rl::XL) {
@@ -632,7 +656,8 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     constexpr int KST = SEGB / (int)sizeof(T);
     constexpr int NSC = WL / LPT;                         // scan threads
     constexpr int ROWB = WL * (int)sizeof(T);
-    constexpr int WROWB = WL * 4;
+    using WT = typename TableT<T>::type;
+    constexpr int WROWB = WL * (int)sizeof(WT);
     constexpr int STAGEB = 2 * WROWB + NTEN * ROWB;
     constexpr int R = ((WL + 31) / 32) * 32 + 16 / (int)sizeof(T);
     constexpr int STG_BUF = NSTG * KST * R;               // elements per staging buffer
@@ -640,7 +665,10 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align128(smem_raw);
     const int H = p.H;
-    float* halo = (float*)(smem + (size_t)NS * STAGEB);   // [2 parity][lo 33 | pad | hi 33 | pad]
+    // [2 parity][lo 33 | pad | hi 33 | pad | sink]: every lane loads and stores one halo word per
+    // step at a precomputed address (lanes other than 0 and 31 use a sink word), so the
+    // exchange has no branches
+    float* halo = (float*)(smem + (size_t)NS * STAGEB);
     uint64_t* bars = (uint64_t*)(halo + 136);
     T* stg = (T*)(bars + 4);
     T* ubuf = stg + 2 * STG_BUF;
@@ -671,19 +699,24 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     const int lane = tid & 31, warp = tid >> 5;
     const int j0 = tid * LPT;
     const int sw = (tid >> 2) & 1;
+    const bool first = lane == 0, lastl = lane == 31;
+    // halo word this lane reads (lane 0: hi of the warp to the left; lane 31: lo of the warp to
+    // the right) and writes (lane 0: its lo; lane 31: its hi), per parity offset 0 / 68
+    const int hread = first ? 34 + warp : (lastl ? warp + 1 : 67);
+    const int hwrite = first ? warp : (lastl ? 34 + warp + 1 : 67);
     constexpr int DSTEP = DIR == kTB ? WL : -WL;
     const int off0 = (DIR == kTB ? 0 : (H - 1) * WL) + j0;
-    unsigned char* const wdst = smem + (size_t)j0 * 4;
+    unsigned char* const wdst = smem + (size_t)j0 * sizeof(WT);
     unsigned char* const tdst = smem + 2 * (size_t)WROWB + (size_t)j0 * sizeof(T);
 
     // ---- issue cursor: plane bases and a 32-bit row offset
     int iss_off = off0;
-    const float* iw0 = nullptr;
-    const float* iw2 = nullptr;
+    const WT* iw0 = nullptr;
+    const WT* iw2 = nullptr;
     const T* isrc[NTEN];
     auto iss_setup = [&](int plane) {
         const int n = plane / p.C, c = plane - n * p.C;
-        iw0 = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
+        iw0 = (const WT*)p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
         iw2 = iw0 + HW;
         const long long po = (long long)plane * HW;
         int t = 0;
@@ -700,8 +733,8 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     auto issue = [&](int s, bool live) {   // s compile-time; live: uniform
         if (live) {
             unsigned char* ws = wdst + s * STAGEB;
-            copy_lanes<float, LPT>(ws, iw0 + iss_off, sw);
-            copy_lanes<float, LPT>(ws + WROWB, iw2 + iss_off, sw);
+            copy_lanes<WT, LPT>(ws, iw0 + iss_off, sw);
+            copy_lanes<WT, LPT>(ws + WROWB, iw2 + iss_off, sw);
             unsigned char* ts = tdst + s * STAGEB;
 #pragma unroll
             for (int t = 0; t < NTEN; ++t) copy_lanes<T, LPT>(ts + t * ROWB, isrc[t] + iss_off, sw);
@@ -715,8 +748,8 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     auto fetch = [&](int s, bool live) {
         cp_async_wait<NS - 1>();
         const unsigned char* ws = wdst + s * STAGEB;
-        read_lanes<float, LPT>(ws, nw0, sw);
-        read_lanes<float, LPT>(ws + WROWB, nw2, sw);
+        read_lanes<WT, LPT>(ws, nw0, sw);
+        read_lanes<WT, LPT>(ws + WROWB, nw2, sw);
         const unsigned char* ts = tdst + s * STAGEB;
         read_lanes<T, LPT>(ts, nz, sw);
         if (Rl::XL) {
@@ -754,10 +787,11 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     auto step = [&](int i, int u, bool last, bool live) {
         const float* lo_prev = halo + ((u + 1) & 1) * 68;
         float* lo_cur = halo + (u & 1) * 68;
+        const float hx = lo_prev[hread];
         float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
         float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
-        if (lane == 0) hl = lo_prev[34 + warp];
-        if (lane == 31) hr = lo_prev[warp + 1];
+        hl = first ? hx : hl;
+        hr = lastl ? hx : hr;
         float hn[LPT];
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
@@ -789,8 +823,7 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
                 ++kblk;
             }
         }
-        if (lane == 0) lo_cur[warp] = last ? 0.f : hn[0];
-        if (lane == 31) lo_cur[34 + warp + 1] = last ? 0.f : hn[LPT - 1];
+        lo_cur[hwrite] = last ? 0.f : (lastl ? hn[LPT - 1] : hn[0]);
         fetch((u + 1) % NS, live);
         if constexpr (NSTG > 0)
             asm volatile("bar.sync 1, %0;" ::"n"(NSC) : "memory");
@@ -836,6 +869,19 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
 __device__ __forceinline__ float u4_get(const uint4& r, int c) {
     return __uint_as_float(c == 0 ? r.x : c == 1 ? r.y : c == 2 ? r.z : r.w);
 }
+// Weight sl of a row segment held as WC 16-byte chunks of table elements.
+template <typename WT, int WC>
+__device__ __forceinline__ float wt_get(const uint4 (&r)[WC], int sl) {
+    if constexpr (std::is_same<WT, float>::value) {
+        return u4_get(r[sl >> 2], sl & 3);
+    } else {
+        const uint4& q = r[sl >> 3];
+        const int e = sl & 7;
+        const uint32_t w = (e >> 1) == 0 ? q.x : (e >> 1) == 1 ? q.y : (e >> 1) == 2 ? q.z : q.w;
+        const float2 f = unpack2<WT>(w);
+        return (e & 1) ? f.y : f.x;
+    }
+}
 
 // CTA = one plane at a time. Thread t owns rows t + T*g for g < G. Ring of NS column tiles; a
 // tile holds, for every row, S steps: 16 bytes of each storage-dtype input and S*4 bytes of each
@@ -847,7 +893,9 @@ __global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsw
     using SG = Seg<T>;
     constexpr int NTEN = Md::NTEN;
     constexpr int S = SG::S;
-    constexpr int WC = S / 4;                             // 16-byte chunks per weight row segment
+    using WT = typename TableT<T>::type;
+    constexpr int WC = S * (int)sizeof(WT) / 16;          // 16-byte chunks per weight row segment
+    constexpr int WPC = 16 / (int)sizeof(WT);             // weights per chunk
     constexpr int NSLOT = 2 * WC + NTEN;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align128(smem_raw);
@@ -866,11 +914,11 @@ __global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsw
     // Issue cursor (per thread): tiles are requested strictly in order.
     long long iss_left = total;
     int iss_bt = 0, iss_s = 0, iss_plane = (int)blockIdx.x;
-    const float* iss_wt = nullptr;
+    const WT* iss_wt = nullptr;
     long long iss_poff = 0;
     auto iss_plane_setup = [&]() {
         const int n = iss_plane / p.C, c = iss_plane % p.C;
-        iss_wt = p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
+        iss_wt = (const WT*)p.wt + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 2 * HW;
         iss_poff = (long long)iss_plane * HW;
     };
     auto issue = [&]() {
@@ -885,8 +933,8 @@ __global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsw
                     unsigned char* d = st + (size_t)row * 16;
 #pragma unroll
                     for (int k = 0; k < WC; ++k) {
-                        cp_async<16>(d + k * slotB, iss_wt + ro + 4 * k);
-                        cp_async<16>(d + (WC + k) * slotB, iss_wt + HW + ro + 4 * k);
+                        cp_async<16>(d + k * slotB, iss_wt + ro + WPC * k);
+                        cp_async<16>(d + (WC + k) * slotB, iss_wt + HW + ro + WPC * k);
                     }
                     const long long off = iss_poff + ro;
                     unsigned char* dt = d + 2 * WC * slotB;
@@ -981,8 +1029,8 @@ __global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsw
                     if (Md::XL) zz *= SG::get(rs1[gg], sl);
                     v = zz;
                     if (i > 0) {
-                        const float w0 = u4_get(rw0[gg][sl >> 2], sl & 3);
-                        const float w2 = u4_get(rw2[gg][sl >> 2], sl & 3);
+                        const float w0 = wt_get<WT, WC>(rw0[gg], sl);
+                        const float w2 = wt_get<WT, WC>(rw2[gg], sl);
                         v = fmaf(w0, hl, fmaf(1.f - w0 - w2, h[gg], fmaf(w2, hr, v)));
                     }
                     float accv = v;
@@ -1061,21 +1109,30 @@ int mode_of(int v, int D) {
     return v == D - 1 ? M_LAST : M_MID;
 }
 
-// ---- vertical geometry: lanes per thread (8, or 4 when W is not a multiple of 8), ring depth
+// ---- vertical geometry: lanes per thread, ring depth
+// 8 lanes per thread, or 4: when W is not a multiple of 8 (every thread's lanes must lie in the
+// row), and for 1024-lane lines when every plane has an SM to itself (one CTA per SM: twice the
+// warps per scheduler hide the per-step latency; with more planes than SMs, the smaller blocks
+// of 8 lanes per thread let more CTAs share an SM instead).
+constexpr int kFixedLanes = 1024;
 int v_lanes(const Problem& P) {
-    int lpt = 8;
-    if (const char* e = getenv("GSPN_VLPT")) lpt = atoi(e) == 4 ? 4 : 8;
-    if (P.W % 8 != 0) lpt = 4;   // 8 lanes per thread only when every thread's lanes lie in the row
-    return lpt;
+    if (P.W % 8 != 0) return 4;
+    if (const char* e = getenv("GSPN_VLPT")) return atoi(e) == 4 ? 4 : 8;
+    if (P.W == kFixedLanes && P.H % 32 == 0 && (long long)P.N * P.C <= device_sm_count()) return 4;
+    return 8;
 }
 int v_threads(const Problem& P) { return std::max(32, ((P.W / v_lanes(P) + 31) / 32) * 32); }
+// Weight-table element bytes (TableT): 4 for fp32 storage, 2 (fp16) for bf16 storage.
+size_t table_esize(const Problem& P) { return P.dtype == GSPN_F32 ? 4 : 2; }
+size_t table_elems(const Problem& P) { return (size_t)P.D * P.N * P.Cw * 2 * (size_t)P.HW; }
+
 int v_block_threads(const Problem& P, int role) { return (role_info(role).nstg ? 2 : 1) * v_threads(P); }
 int v_max_threads(const Problem& P) { return v_lanes(P) == 8 ? 512 : 1024; }
 size_t v_smem(const Problem& P, int role, int ns, int segb) {
     const RoleInfo ri = role_info(role);
     const size_t R = ((size_t)(P.W + 31) / 32) * 32 + 16 / P.esize();
     const size_t kst = (size_t)segb / P.esize();
-    return 128 + (size_t)ns * (2 * (size_t)P.W * 4 + (size_t)ri.nten * P.W * P.esize()) + 2 * 68 * 4 + 32 +
+    return 128 + (size_t)ns * (2 * (size_t)P.W * table_esize(P) + (size_t)ri.nten * P.W * P.esize()) + 2 * 68 * 4 + 32 +
            2 * (size_t)ri.nstg * kst * R * P.esize() + (ri.ystg ? 2 * (size_t)P.W * kst * P.esize() : 0);
 }
 int ctas_per_sm(size_t smem) { return smem > kSmemBudget ? 0 : (int)(kSmemSM / (smem + 1024)); }
@@ -1127,7 +1184,9 @@ int h_rows(const Problem& P) {
     return g <= 1 ? 1 : (g <= 2 ? 2 : 4);
 }
 int h_pad(const Problem& P) { return ((P.H + 7) / 8) * 8; }
-int h_slots(const Problem& P, int mode) { return 2 * ((16 / P.esize()) / 4) + ntensors(mode); }
+// One 16-byte chunk per weight row segment: 4 fp32 or 8 fp16 weights, as many as storage
+// elements in a 16-byte segment.
+int h_slots(const Problem&, int mode) { return 2 + ntensors(mode); }
 size_t h_smem(const Problem& P, int mode, int ns) {
     return 128 + (size_t)ns * h_slots(P, mode) * h_pad(P) * 16 + 2 * 2 * h_rows(P) * 32 * sizeof(float);
 }
@@ -1204,37 +1263,37 @@ cudaError_t launch_v3(const Problem& P, const SweepArgs& a, const VCfg& c, cudaS
 }
 
 // Fixed-width kernel: 1024-lane lines (the 1024 x 1024 maps in both scan orientations), scan
-// lengths a multiple of 32, 8 lanes per thread.
-constexpr int kFixedLanes = 1024;
+// lengths a multiple of 32.
 bool use_fixed(const Problem& P) {
     if (const char* e = getenv("GSPN_NOFIXED"))
         if (atoi(e) != 0) return false;
-    return P.W == kFixedLanes && P.H % 32 == 0 && P.H >= 32 && v_lanes(P) == 8;
+    return P.W == kFixedLanes && P.H % 32 == 0 && P.H >= 32;
 }
 
-template <typename T, unsigned DIR, int ROLE, int NS, int SEGB>
+template <typename T, unsigned DIR, int ROLE, int LPT, int NS, int SEGB>
 cudaError_t launch_w4(const Problem& P, const SweepArgs& a, cudaStream_t st) {
     const size_t smem = v_smem(P, ROLE, NS, SEGB);
     const int threads = v_block_threads(P, ROLE);
-    auto kern = k_vsweep_w<T, DIR, ROLE, 8, NS, SEGB, kFixedLanes>;
+    auto kern = k_vsweep_w<T, DIR, ROLE, LPT, NS, SEGB, kFixedLanes>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     const int grid = sweep_grid(P, kern, threads, smem);
     launch_begin(st);
-    k_vsweep_w<T, DIR, ROLE, 8, NS, SEGB, kFixedLanes><<<grid, threads, smem, st>>>(a);
+    k_vsweep_w<T, DIR, ROLE, LPT, NS, SEGB, kFixedLanes><<<grid, threads, smem, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
 }
 
-template <typename T, unsigned DIR, int ROLE>
+template <typename T, unsigned DIR, int ROLE, int LPT>
 cudaError_t launch_w3(const Problem& P, const SweepArgs& a, const VCfg& c, cudaStream_t st) {
     using Rl = RoleT<ROLE>;
     if constexpr (Rl::NSTG == 0) {
-        return c.ns == 4 ? launch_w4<T, DIR, ROLE, 4, 16>(P, a, st) : launch_w4<T, DIR, ROLE, 2, 16>(P, a, st);
+        return c.ns == 4 ? launch_w4<T, DIR, ROLE, LPT, 4, 16>(P, a, st) : launch_w4<T, DIR, ROLE, LPT, 2, 16>(P, a, st);
     } else {
-        return (c.ns == Rl::NS_A && c.segb == Rl::SEG_A) ? launch_w4<T, DIR, ROLE, Rl::NS_A, Rl::SEG_A>(P, a, st)
-                                                         : launch_w4<T, DIR, ROLE, Rl::NS_B, Rl::SEG_B>(P, a, st);
+        return (c.ns == Rl::NS_A && c.segb == Rl::SEG_A)
+                   ? launch_w4<T, DIR, ROLE, LPT, Rl::NS_A, Rl::SEG_A>(P, a, st)
+                   : launch_w4<T, DIR, ROLE, LPT, Rl::NS_B, Rl::SEG_B>(P, a, st);
     }
 }
 
@@ -1242,7 +1301,8 @@ template <typename T, unsigned DIR, int ROLE>
 cudaError_t launch_v(const Problem& P, const SweepArgs& a, cudaStream_t st) {
     const VCfg c = v_config(P, ROLE);
     if (c.ns == 0) return cudaErrorNotSupported;
-    if (use_fixed(P)) return launch_w3<T, DIR, ROLE>(P, a, c, st);
+    if (use_fixed(P))
+        return v_lanes(P) == 4 ? launch_w3<T, DIR, ROLE, 4>(P, a, c, st) : launch_w3<T, DIR, ROLE, 8>(P, a, c, st);
     return v_lanes(P) == 4 ? launch_v3<T, DIR, ROLE, 4>(P, a, c, st) : launch_v3<T, DIR, ROLE, 8>(P, a, c, st);
 }
 
@@ -1273,7 +1333,6 @@ cudaError_t launch_hdir(const Problem& P, const SweepArgs& a, int mode, cudaStre
     }
 }
 
-size_t table_floats(const Problem& P) { return (size_t)P.D * P.N * P.Cw * 2 * (size_t)P.HW; }
 
 // The transposed path: when the mask has vertical and horizontal directions, both image axes
 // give 16-byte rows and a line fits a CTA with its writer warps (at most 2048 lanes), the
@@ -1330,8 +1389,9 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
                             void* ws, cudaStream_t st) {
     const bool tp = tpath(P);
     const int nV = n_vertical(P);
+    using WT = typename TableT<T>::type;
     WsCarver wc(ws);
-    float* table = wc.take<float>(table_floats(P));
+    WT* table = wc.take<WT>(table_elems(P));
     void *z = nullptr, *acc = nullptr, *zt = nullptr, *acct = nullptr;
     if (tp) {
         if (nV == 2 && tplan() == 2) z = wc.take<T>(P.U);
@@ -1342,36 +1402,33 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
         z = wc.take<T>(P.U);
         acc = wc.take<T>(P.U);
     }
-    // A1: weight formation for every direction, once per (n, cw) plane
-    WeightArgs wa{a, table, P.N, P.Cw, P.H, P.W, P.D, 0, {0u, 0u, 0u, 0u}};
+    // A1: weight formation for every direction, once per (n, cw) plane, in one launch; on the
+    // transposed path the horizontal slots (which follow the vertical ones) are written [W][H]
+    WeightArgs wa{a, table, P.N, P.Cw, P.H, P.W, P.D, tp ? nV : P.D, {0u, 0u, 0u, 0u}};
     for (int v = 0, k = 0; k < 4; ++k)
         if (P.mask & (1u << k)) wa.dirs[v++] = 1u << k;
     const int per_slot = P.N * P.Cw;
-    const int row_planes = (tp ? nV : P.D) * per_slot;
+    {
+        const int tiles_x = (P.W + kWTileC - 1) / kWTileC, tiles_y = (P.H + kWTileR - 1) / kWTileR;
+        const long long ntiles = (long long)P.D * per_slot * tiles_x * tiles_y;
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_weights<T>, 256, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        const int grid = (int)std::min<long long>(ntiles, (long long)per_sm * device_sm_count());
+        launch_begin(st);
+        k_weights<T><<<grid, 256, 0, st>>>(wa, tiles_x, tiles_y, (int)ntiles);
+        launch_end(st);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     cudaError_t e;
-    if (row_planes > 0) {
-        const int quads = (int)(P.HW / 4);
-        const dim3 wgrid((unsigned)std::max(1, std::min((quads + 255) / 256, 64)), (unsigned)row_planes);
-        launch_begin(st);
-        k_sweep_weights<T><<<wgrid, 256, 0, st>>>(wa);
-        launch_end(st);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    if (tp) {
-        wa.plane0 = nV * per_slot;
-        const dim3 tgrid((unsigned)((P.W + 31) / 32), (unsigned)((P.H + 31) / 32), (unsigned)((P.D - nV) * per_slot));
-        launch_begin(st);
-        k_sweep_weights_t<T><<<tgrid, 256, 0, st>>>(wa);
-        launch_end(st);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
     // A2-A6: one sweep per direction
-    const size_t slot_floats = (size_t)per_slot * 2 * (size_t)P.HW;
+    const size_t slot_elems = (size_t)per_slot * 2 * (size_t)P.HW;
     const Problem PS = swapped(P);
     int v = 0;
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
-        SweepArgs args{x, lam, u, table + v * slot_floats, z, acc, y, zt, acct, (unsigned*)ws,
+        SweepArgs args{x, lam, u, table + v * slot_elems, z, acc, y, zt, acct, (unsigned*)ws,
                        P.N, P.C, P.H, P.W, P.Cw};
         const int role = visit_role(P, d, v, tp);
         const bool asc = d == kTB || d == kLR;
@@ -1399,7 +1456,8 @@ bool sweep_supports(const Problem& P, bool bwd) {
     if (bwd) return false;
     if ((P.W * P.esize()) % 16 != 0) return false;   // 16-byte rows and column tiles
     if (P.W > 4096) return false;
-    if ((long long)P.D * P.N * P.Cw > 65535) return false;   // weight-formation grid.y / grid.z
+    if ((long long)P.D * P.N * P.Cw * ((P.H + kWTileR - 1) / kWTileR) * ((P.W + kWTileC - 1) / kWTileC) > 0x7fffffffLL)
+        return false;   // weight-formation tile count
     const bool tp = tpath(P);
     const Problem PS = swapped(P);
     for (int v = 0, k = 0; k < 4; ++k) {
@@ -1418,7 +1476,7 @@ bool sweep_supports(const Problem& P, bool bwd) {
 
 size_t sweep_ws_bytes(const Problem& P, bool bwd) {
     if (bwd) return 0;
-    size_t b = 256 + align256(table_floats(P) * sizeof(float));
+    size_t b = 256 + align256(table_elems(P) * table_esize(P));
     const size_t ub = align256((size_t)P.U * P.esize());
     if (tpath(P)) b += (n_vertical(P) == 2 ? (tplan() == 2 ? 4 : 3) : 2) * ub;
     else if (P.D > 1) b += 2 * ub;
