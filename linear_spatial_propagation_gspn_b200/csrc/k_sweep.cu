@@ -159,23 +159,25 @@ template <> struct TableT<__nv_bfloat16> { using type = __half; };
 
 // Turns the logits of every (slot, n, cw) plane into the two outer weights w0, w2 of each
 // normalised tridiagonal row; the sweeps re-derive w1 = 1 - w0 - w2. Elementwise and
-// memory-bound, one launch for all slots. A persistent CTA (256 threads) takes tiles of 32 rows
+// memory-bound, one launch for all slots. A persistent CTA (512 threads) takes tiles of 32 rows
 // x 128 columns: thread (tx, ty) loads 4 consecutive columns (one vector per logit row) of rows
-// ty, ty + 8, ty + 16, ty + 24, forms the 16 weights (MUFU exponential and reciprocal, the
-// normalisation applied afterwards so every row still sums to one up to a few ulp; the
-// max-shifted form for logits below -40), and writes them in the image layout straight from
-// registers, or, for the transposed slots ([W][H] planes:
-// element (column c, row r) at c * H + r), through a shared-memory tile read column-wise (row
-// stride 129 words: conflict-free) so that the table writes stay coalesced. Needs W % 4 == 0.
-constexpr int kWTileR = 32, kWTileC = 128;
+// ty and ty + 16, forms the 8 weights (MUFU exponential and reciprocal, the normalisation
+// applied afterwards so every row still sums to one up to a few ulp; the max-shifted form for
+// logits below -40), and writes them in the image layout straight from registers, or, for the
+// transposed slots ([W][H] planes: element (column c, row r) at c * H + r), through a
+// shared-memory tile read column-wise (row stride 129 words: conflict-free) so that the table
+// writes stay coalesced. Needs W % 4 == 0.
+constexpr int kWTileR = 32, kWTileC = 128, kWThreads = 512;
 
 template <typename T>
-__global__ void __launch_bounds__(256) k_weights(WeightArgs p, int tiles_x, int tiles_y, int ntiles) {
+__global__ void __launch_bounds__(kWThreads) k_weights(WeightArgs p, int tiles_x, int tiles_y, int ntiles) {
     using WT = typename TableT<T>::type;
+    constexpr int RPT = kWTileR * 32 / kWThreads;   // rows per thread (2)
+    constexpr int RSTEP = kWThreads / 32;           // 16
     __shared__ float tile[2][kWTileR][kWTileC + 1];
     const int H = p.H, W = p.W;
     const long long HW = (long long)H * W;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
     const int per_plane = tiles_x * tiles_y;
     const int planes_per_slot = p.N * p.Cw;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -188,33 +190,40 @@ __global__ void __launch_bounds__(256) k_weights(WeightArgs p, int tiles_x, int 
         const int r0 = by * kWTileR, c0 = bx * kWTileC;
         const int c = c0 + 4 * tx;
         const bool cin = c < W;   // W % 4 == 0: a quad is all in or all out
-        float w0[4][4], w2[4][4];
+        float l0[RPT][4], l1[RPT][4], l2[RPT][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int r = r0 + ty + 8 * k;
-            float l0[4] = {0.f, 0.f, 0.f, 0.f}, l1[4] = {0.f, 0.f, 0.f, 0.f}, l2[4] = {0.f, 0.f, 0.f, 0.f};
-            const bool in = cin && r < H;
-            if (in) {
+        for (int k = 0; k < RPT; ++k) {
+            const int r = r0 + ty + RSTEP * k;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) l0[k][e] = l1[k][e] = l2[k][e] = 0.f;
+            if (cin && r < H) {
                 const long long q = (long long)r * W + c;
-                ld_lanes<T, 4>(a3 + q, l0);
-                ld_lanes<T, 4>(a3 + HW + q, l1);
-                ld_lanes<T, 4>(a3 + 2 * HW + q, l2);
+                ld_lanes<T, 4>(a3 + q, l0[k]);
+                ld_lanes<T, 4>(a3 + HW + q, l1[k]);
+                ld_lanes<T, 4>(a3 + 2 * HW + q, l2[k]);
             }
+        }
+        float w0[RPT][4], w2[RPT][4];
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int r = r0 + ty + RSTEP * k;
+            const bool in = cin && r < H;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int cc = c + e;
                 const bool hl = vert ? cc > 0 : r > 0;
                 const bool hr = vert ? cc < W - 1 : r < H - 1;
-                Wts w = lane_weights_fast_nocheck(l0[e], l1[e], l2[e], hl, hr);
-                if (weights_need_shift(l0[e], l1[e], l2[e], hl, hr)) w = weights_shifted(l0[e], l1[e], l2[e], hl, hr);
+                Wts w = lane_weights_fast_nocheck(l0[k][e], l1[k][e], l2[k][e], hl, hr);
+                if (weights_need_shift(l0[k][e], l1[k][e], l2[k][e], hl, hr))
+                    w = weights_shifted(l0[k][e], l1[k][e], l2[k][e], hl, hr);
                 w0[k][e] = in ? w.w0 : 0.f;
                 w2[k][e] = in ? w.w2 : 0.f;
             }
         }
         if (slot < p.tslot0) {   // image layout, straight from registers
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int r = r0 + ty + 8 * k;
+            for (int k = 0; k < RPT; ++k) {
+                const int r = r0 + ty + RSTEP * k;
                 if (cin && r < H) {
                     const long long q = (long long)r * W + c;
                     st_lanes<WT, 4>(wt + q, w0[k]);
@@ -223,18 +232,18 @@ __global__ void __launch_bounds__(256) k_weights(WeightArgs p, int tiles_x, int 
             }
         } else {                 // transposed planes (uniform per tile: the barriers are safe)
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < RPT; ++k)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    tile[0][ty + 8 * k][4 * tx + e] = w0[k][e];
-                    tile[1][ty + 8 * k][4 * tx + e] = w2[k][e];
+                    tile[0][ty + RSTEP * k][4 * tx + e] = w0[k][e];
+                    tile[1][ty + RSTEP * k][4 * tx + e] = w2[k][e];
                 }
             __syncthreads();
-            // warp ty writes columns ty, ty + 8, ...: 32 consecutive rows each (lane = row)
+            // warp ty writes columns ty, ty + 16, ...: 32 consecutive rows each (lane = row)
             const int r = r0 + tx;
             if (r < H) {
 #pragma unroll 4
-                for (int cc = ty; cc < kWTileC; cc += 8) {
+                for (int cc = ty; cc < kWTileC; cc += RSTEP) {
                     const int col = c0 + cc;
                     if (col < W) {
                         const long long q = (long long)col * H + r;
@@ -277,10 +286,12 @@ template <int ROLE> struct RoleT {
     // storage-dtype tensors per ring stage: x lam | z, [partial], [u]  (plus two fp32 weight rows)
     static constexpr int NTEN = (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (URING ? 1 : 0);
     static constexpr int NSTG = (ZSTG ? 1 : 0) + (ASTG ? 1 : 0);   // staged (lane-major) outputs
-    // (ring stages, lane-major segment bytes) of the two launch configurations: A, and B with a
-    // shorter ring for more CTAs per SM. A final lane-major sweep also keeps u of two blocks.
+    // (ring stages, lane-major segment bytes) of the two launch configurations: A, and B with
+    // less shared memory for more CTAs per SM (a shorter ring at 4-byte storage; at 2-byte
+    // storage the halved staging suffices). A final lane-major sweep also keeps u of two blocks.
     static constexpr int NS_A = 4, SEG_A = (NSTG == 1 && !YSTG) ? 64 : 32;
-    static constexpr int NS_B = 2, SEG_B = 32;
+    static constexpr int SEG_B = 32;
+    template <typename T> static constexpr int ns_b() { return sizeof(T) == 2 ? 4 : 2; }
 };
 
 // ---- mbarrier hand-off between the scan warps and the writer warps of a lane-major sweep
@@ -1083,11 +1094,12 @@ int ntensors(int mode) {   // horizontal column-tile sweep
     }
 }
 struct RoleInfo {
-    int nten, nstg, ystg, ns_a, seg_a, ns_b, seg_b;
+    int nten, nstg, ystg, ns_a, seg_a, ns_b2, ns_b4, seg_b;   // ns_b2 / ns_b4: 2- / 4-byte storage
 };
 template <int ROLE> constexpr RoleInfo role_info_t() {
     using Rl = RoleT<ROLE>;
-    return {Rl::NTEN, Rl::NSTG, Rl::YSTG ? 1 : 0, Rl::NS_A, Rl::SEG_A, Rl::NS_B, Rl::SEG_B};
+    return {Rl::NTEN, Rl::NSTG, Rl::YSTG ? 1 : 0, Rl::NS_A, Rl::SEG_A,
+            Rl::template ns_b<__nv_bfloat16>(), Rl::template ns_b<float>(), Rl::SEG_B};
 }
 RoleInfo role_info(int role) {
     switch (role) {
@@ -1135,12 +1147,18 @@ size_t v_smem(const Problem& P, int role, int ns, int segb) {
     return 128 + (size_t)ns * (2 * (size_t)P.W * table_esize(P) + (size_t)ri.nten * P.W * P.esize()) + 2 * 68 * 4 + 32 +
            2 * (size_t)ri.nstg * kst * R * P.esize() + (ri.ystg ? 2 * (size_t)P.W * kst * P.esize() : 0);
 }
-int ctas_per_sm(size_t smem) { return smem > kSmemBudget ? 0 : (int)(kSmemSM / (smem + 1024)); }
+// Resident CTAs per SM by shared memory and, assuming the 128-register cap of the 8-lane
+// kernels (the largest of them use about that many), by registers.
+int ctas_per_sm(size_t smem, int threads) {
+    if (smem > kSmemBudget) return 0;
+    const int by_smem = (int)(kSmemSM / (smem + 1024));
+    const int by_regs = 65536 / (threads * 128);
+    return std::max(0, std::min(by_smem, by_regs));
+}
 
 // Ring depth and staging segment of a vertical sweep; ns == 0: not supported.
-//  - no staged output: 4 stages when they fit; 2 when there are more planes than SMs and the
-//    shorter ring lets twice as many CTAs (planes) share an SM, which hides more of the per-step
-//    latency;
+//  - no staged output: 4 stages, or 2 when there are more planes than SMs and the shorter ring
+//    lets more CTAs (planes) share an SM, which hides more of the per-step latency;
 //  - staged output: configuration A or B of the role, whichever runs more of the planes at once
 //    (A on a tie).
 struct VCfg {
@@ -1148,21 +1166,23 @@ struct VCfg {
 };
 VCfg v_config(const Problem& P, int role) {
     const RoleInfo ri = role_info(role);
+    const int threads = v_block_threads(P, role);
     if (ri.nstg == 0) {
         const size_t s4 = v_smem(P, role, 4, 16), s2 = v_smem(P, role, 2, 16);
         if (s2 > kSmemBudget) return {0, 16};
         if (s4 > kSmemBudget) return {2, 16};
         const bool many = (long long)P.N * P.C > device_sm_count();
-        if (many && kSmemBudget / s2 >= 2 * (kSmemBudget / s4)) return {2, 16};
+        if (many && ctas_per_sm(s2, threads) > ctas_per_sm(s4, threads)) return {2, 16};
         return {4, 16};
     }
-    if (v_block_threads(P, role) > v_max_threads(P)) return {0, 0};
+    if (threads > v_max_threads(P)) return {0, 0};
     const long long planes = (long long)P.N * P.C, sms = device_sm_count();
     const int need = (int)std::min<long long>(64, (planes + sms - 1) / sms);
-    const int ua = std::min(ctas_per_sm(v_smem(P, role, ri.ns_a, ri.seg_a)), need);
-    const int ub = std::min(ctas_per_sm(v_smem(P, role, ri.ns_b, ri.seg_b)), need);
+    const int ns_b = P.esize() == 2 ? ri.ns_b2 : ri.ns_b4;
+    const int ua = std::min(ctas_per_sm(v_smem(P, role, ri.ns_a, ri.seg_a), threads), need);
+    const int ub = std::min(ctas_per_sm(v_smem(P, role, ns_b, ri.seg_b), threads), need);
     if (ua == 0 && ub == 0) return {0, 0};
-    return ua >= ub ? VCfg{ri.ns_a, ri.seg_a} : VCfg{ri.ns_b, ri.seg_b};
+    return ua >= ub ? VCfg{ri.ns_a, ri.seg_a} : VCfg{ns_b, ri.seg_b};
 }
 
 // ---- horizontal geometry: threads, rows per thread (as instantiated), padded rows, ring depth
@@ -1257,8 +1277,9 @@ cudaError_t launch_v3(const Problem& P, const SweepArgs& a, const VCfg& c, cudaS
     if constexpr (Rl::NSTG == 0) {
         return c.ns == 4 ? launch_v4<T, DIR, ROLE, LPT, 4, 16>(P, a, st) : launch_v4<T, DIR, ROLE, LPT, 2, 16>(P, a, st);
     } else {
+        constexpr int NSB = Rl::template ns_b<T>();
         return (c.ns == Rl::NS_A && c.segb == Rl::SEG_A) ? launch_v4<T, DIR, ROLE, LPT, Rl::NS_A, Rl::SEG_A>(P, a, st)
-                                                         : launch_v4<T, DIR, ROLE, LPT, Rl::NS_B, Rl::SEG_B>(P, a, st);
+                                                         : launch_v4<T, DIR, ROLE, LPT, NSB, Rl::SEG_B>(P, a, st);
     }
 }
 
@@ -1291,9 +1312,9 @@ cudaError_t launch_w3(const Problem& P, const SweepArgs& a, const VCfg& c, cudaS
     if constexpr (Rl::NSTG == 0) {
         return c.ns == 4 ? launch_w4<T, DIR, ROLE, LPT, 4, 16>(P, a, st) : launch_w4<T, DIR, ROLE, LPT, 2, 16>(P, a, st);
     } else {
-        return (c.ns == Rl::NS_A && c.segb == Rl::SEG_A)
-                   ? launch_w4<T, DIR, ROLE, LPT, Rl::NS_A, Rl::SEG_A>(P, a, st)
-                   : launch_w4<T, DIR, ROLE, LPT, Rl::NS_B, Rl::SEG_B>(P, a, st);
+        constexpr int NSB = Rl::template ns_b<T>();
+        return (c.ns == Rl::NS_A && c.segb == Rl::SEG_A) ? launch_w4<T, DIR, ROLE, LPT, Rl::NS_A, Rl::SEG_A>(P, a, st)
+                                                         : launch_w4<T, DIR, ROLE, LPT, NSB, Rl::SEG_B>(P, a, st);
     }
 }
 
@@ -1412,11 +1433,12 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
         const int tiles_x = (P.W + kWTileC - 1) / kWTileC, tiles_y = (P.H + kWTileR - 1) / kWTileR;
         const long long ntiles = (long long)P.D * per_slot * tiles_x * tiles_y;
         int per_sm = 1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_weights<T>, 256, 0) != cudaSuccess || per_sm < 1)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_weights<T>, kWThreads, 0) != cudaSuccess ||
+            per_sm < 1)
             per_sm = 1;
         const int grid = (int)std::min<long long>(ntiles, (long long)per_sm * device_sm_count());
         launch_begin(st);
-        k_weights<T><<<grid, 256, 0, st>>>(wa, tiles_x, tiles_y, (int)ntiles);
+        k_weights<T><<<grid, kWThreads, 0, st>>>(wa, tiles_x, tiles_y, (int)ntiles);
         launch_end(st);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
