@@ -59,16 +59,42 @@ __device__ __forceinline__ int plane_pix(int H, int W, int Wp, int i, int j) {
     return j * Wp + (W - 1 - i);
 }
 
-// One warp scans the whole plane for direction D; lane j is held by thread j / LPT.
+// One warp scans the whole plane for direction D; lane j is held by thread j / LPT. Software
+// pipelined: the shared-memory operands of step i + 1 (z, w0, w2 and the running sum) are
+// loaded while step i's new line is formed, so a step waits only for the shuffles and FMAs of
+// the recurrence. Lanes past the line (j >= M) read index 0 and contribute nothing.
 template <unsigned D, int LPT>
 __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, const float* w2b, float* acc, int H,
                                            int W, int Wp, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
-    float h[LPT];
+    float h[LPT], cz[LPT], cw0[LPT], cw2[LPT], ca[LPT];
+    int cq[LPT];
+    bool on[LPT];
 #pragma unroll
-    for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+    for (int e = 0; e < LPT; ++e) {
+        h[e] = 0.f;
+        const int j = lane * LPT + e;
+        on[e] = j < M;
+        cq[e] = on[e] ? plane_pix<D>(H, W, Wp, 0, j) : 0;
+        cz[e] = z[cq[e]];
+        cw0[e] = 0.f;   // step 0 has no predecessor: h_0 = z
+        cw2[e] = 0.f;
+        ca[e] = acc[cq[e]];
+    }
     for (int i = 0; i < L; ++i) {
+        // operands of step i + 1
+        float nz[LPT], nw0[LPT], nw2[LPT], na[LPT];
+        int nq[LPT];
+        const bool more = i + 1 < L;
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            const int j = lane * LPT + e;
+            nq[e] = (more && on[e]) ? plane_pix<D>(H, W, Wp, i + 1, j) : 0;
+            nz[e] = z[nq[e]];
+            nw0[e] = w0b[nq[e]];
+            nw2[e] = w2b[nq[e]];
+        }
         float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
         float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
         if (lane == 0) hl = 0.f;
@@ -76,23 +102,24 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
         float hn[LPT];
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
-            const int j = lane * LPT + e;
-            hn[e] = 0.f;
-            if (j < M) {
-                const int q = plane_pix<D>(H, W, Wp, i, j);
-                float v = z[q];
-                if (i > 0) {
-                    const float w0 = w0b[q], w2 = w2b[q];
-                    const float left = e == 0 ? hl : h[e - 1];
-                    const float right = e == LPT - 1 ? hr : h[e + 1];
-                    v = fmaf(w0, left, fmaf(1.f - w0 - w2, h[e], fmaf(w2, right, v)));
-                }
-                acc[q] += v;
-                hn[e] = v;
-            }
+            const float left = e == 0 ? hl : h[e - 1];
+            const float right = e == LPT - 1 ? hr : h[e + 1];
+            const float v = fmaf(cw0[e], left, fmaf(1.f - cw0[e] - cw2[e], h[e], fmaf(cw2[e], right, cz[e])));
+            hn[e] = on[e] ? v : 0.f;
+            if (on[e]) acc[cq[e]] = ca[e] + v;
         }
+        // the running sum of step i + 1 is read after this step's writes (different pixels
+        // except at the same lane, which this thread owns)
 #pragma unroll
-        for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+        for (int e = 0; e < LPT; ++e) {
+            na[e] = acc[nq[e]];
+            h[e] = hn[e];
+            cz[e] = nz[e];
+            cw0[e] = nw0[e];
+            cw2[e] = nw2[e];
+            ca[e] = na[e];
+            cq[e] = nq[e];
+        }
     }
 }
 
@@ -102,15 +129,33 @@ template <typename T, unsigned D>
 __device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2b, int H, int W, int Wp, int tid) {
     const int HW = H * W;
     if (W % 4 == 0) {
-        for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
-            const int r = e / W, col = e - r * W;
-            float a0[4], a1[4], a2[4];
+        // each iteration's logits are loaded one iteration ahead, so the global-load latency is
+        // paid about once per direction instead of once per iteration
+        float a0[4], a1[4], a2[4];
+        int e = tid * 4;
+        if (e < HW) {
             ld_lanes<T, 4>(a3 + e, a0);
             ld_lanes<T, 4>(a3 + HW + e, a1);
             ld_lanes<T, 4>(a3 + 2 * HW + e, a2);
+        }
+        for (; e < HW; e += kPlaneThreads * 4) {
+            float b0[4], b1[4], b2[4];
+            const int en = e + kPlaneThreads * 4;
+            if (en < HW) {
+                ld_lanes<T, 4>(a3 + en, b0);
+                ld_lanes<T, 4>(a3 + HW + en, b1);
+                ld_lanes<T, 4>(a3 + 2 * HW + en, b2);
+            }
+            const int r = e / W, col = e - r * W;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 pixel_weights<D>(a0[k], a1[k], a2[k], r, col + k, H, W, w0b[r * Wp + col + k], w2b[r * Wp + col + k]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                a0[k] = b0[k];
+                a1[k] = b1[k];
+                a2[k] = b2[k];
+            }
         }
     } else {
         for (int e = tid; e < HW; e += kPlaneThreads) {
