@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--cpu-planes", type=int, default=24, help="planes of the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward (gradients of x, logits, lambda, u); on by default for 'train'")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch N (small cases for profiler captures; not a bench line)")
     return ap.parse_args()
@@ -185,14 +187,18 @@ def measured_peak():
     return 6650.0, "fallback"
 
 
+# Sources that build the large-map forward the traffic summary describes (the sweep family,
+# its shared helpers and the entry points); other families do not affect it.
+SWEEP_SOURCES = ("gspn_api.cu", "gspn_common.cuh", "gspn_internal.h", "k_sweep.cu")
+
+
 def kernel_source_sha():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_spatial_propagation_gspn_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode())
-                h.update(f.read())
+    for fn in SWEEP_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -303,6 +309,46 @@ def run_libgspn(args):
         # DRAM bytes each launch moves (ncu) over its event-timed duration
         roofline["kernels_dram_gbs"] = {n: round(b / (p * 1e-3) / 1e9, 1) for n, b, p in zip(names, per_launch, per)}
 
+    # ---- backward (A7): gradients of sum(dy * y), timed on its own over the same number of steps
+    bwd = None
+    if args.backward or wl.name == "train":
+        dy = torch.randn(x.shape, generator=torch.Generator(device=dev).manual_seed(wl.seed + 7), device=dev,
+                         dtype=torch.float32).to(x.dtype)
+        bdesc = g.desc_for(x, wl.wmode, wl.mask)
+        bws = g.alloc_workspace(bdesc, True, dev)
+        outs = (torch.empty_like(x), torch.empty_like(a), torch.empty_like(x), torch.empty_like(x))
+
+        def bstep():
+            g.backward(x, a, lam, u, dy, wl.wmode, wl.mask, out=outs, ws=bws)
+
+        for _ in range(max(3, args.warmup // 2)):
+            bstep()
+        torch.cuda.synchronize()
+        nb_steps = max(5, args.steps // 4)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        b0 = torch.cuda.Event(enable_timing=True)
+        b1 = torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(nb_steps):
+            bstep()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        bms = b0.elapsed_time(b1) / nb_steps
+        if world > 1:
+            tt = torch.tensor([bms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            bms = float(tt.item())
+        bcomp = wl.compulsory_bwd_bytes()
+        bgbs = bcomp * world / (bms * 1e-3) / 1e9
+        bwd = {"ms_per_step": round(bms, 4), "steps": nb_steps, "compulsory_bytes": bcomp,
+               "value": round(bgbs, 2), "unit": "GB/s", "frac": round(bgbs / world / peak, 4),
+               "algo": g.ALGO_NAMES.get(g.selected_algo(bdesc, True), "?"),
+               "what": "reads dy, x, lambda, u, logits; writes dx, dlambda, du, dlogits (compulsory bytes)",
+               "train_step_ms": round(ms_step + bms, 4)}
+        del bws, outs, dy
+
     # ---- copy ceiling on the same byte volume
     nb = (comp // 2) // 16 * 16
     src = torch.empty(nb, dtype=torch.uint8, device=dev)
@@ -370,6 +416,7 @@ def run_libgspn(args):
             "copy_ceiling_gbs": round(copy_gbs, 1),
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "backward": bwd,
             "gpu_launches": launches * args.steps,
             "clocks": clocks,
         }

@@ -258,16 +258,36 @@ struct PlaneBwdArgs {
     unsigned mask;
 };
 
-// Forward recompute of direction D by one warp: hb = h^D (plane layout), acc += h^D.
+// Forward recompute of direction D by one warp: hb = h^D (plane layout), acc += h^D. Software
+// pipelined like plane_scan.
 template <unsigned D, int LPT>
 __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b, const float* w2b, float* hb,
                                                 float* acc, int H, int W, int Wp, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
-    float h[LPT];
+    float h[LPT], cz[LPT], cw0[LPT], cw2[LPT];
+    int cq[LPT];
+    bool on[LPT];
 #pragma unroll
-    for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+    for (int e = 0; e < LPT; ++e) {
+        h[e] = 0.f;
+        const int j = lane * LPT + e;
+        on[e] = j < M;
+        cq[e] = on[e] ? plane_pix<D>(H, W, Wp, 0, j) : 0;
+        cz[e] = z[cq[e]];
+        cw0[e] = cw2[e] = 0.f;   // step 0: h_0 = z
+    }
     for (int i = 0; i < L; ++i) {
+        float nz[LPT], nw0[LPT], nw2[LPT];
+        int nq[LPT];
+        const bool more = i + 1 < L;
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            nq[e] = (more && on[e]) ? plane_pix<D>(H, W, Wp, i + 1, lane * LPT + e) : 0;
+            nz[e] = z[nq[e]];
+            nw0[e] = w0b[nq[e]];
+            nw2[e] = w2b[nq[e]];
+        }
         float hl = __shfl_up_sync(0xffffffffu, h[LPT - 1], 1);
         float hr = __shfl_down_sync(0xffffffffu, h[0], 1);
         if (lane == 0) hl = 0.f;
@@ -275,104 +295,160 @@ __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b
         float hn[LPT];
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
-            const int j = lane * LPT + e;
-            hn[e] = 0.f;
-            if (j < M) {
-                const int q = plane_pix<D>(H, W, Wp, i, j);
-                float v = z[q];
-                if (i > 0) {
-                    const float w0 = w0b[q], w2 = w2b[q];
-                    v = fmaf(w0, e == 0 ? hl : h[e - 1], fmaf(1.f - w0 - w2, h[e], fmaf(w2, e == LPT - 1 ? hr : h[e + 1], v)));
-                }
-                hb[q] = v;
-                acc[q] += v;
-                hn[e] = v;
+            const float left = e == 0 ? hl : h[e - 1];
+            const float right = e == LPT - 1 ? hr : h[e + 1];
+            const float v = fmaf(cw0[e], left, fmaf(1.f - cw0[e] - cw2[e], h[e], fmaf(cw2[e], right, cz[e])));
+            hn[e] = on[e] ? v : 0.f;
+            if (on[e]) {
+                hb[cq[e]] = v;
+                acc[cq[e]] += v;
             }
         }
 #pragma unroll
-        for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+        for (int e = 0; e < LPT; ++e) {
+            h[e] = hn[e];
+            cz[e] = nz[e];
+            cw0[e] = nw0[e];
+            cw2[e] = nw2[e];
+            cq[e] = nq[e];
+        }
     }
 }
 
-// Reverse scan of direction D by one warp:
-//   delta_i[j] = g_i[j] + w_{i+1}[j-1][2] delta_{i+1}[j-1] + w_{i+1}[j][1] delta_{i+1}[j] + w_{i+1}[j+1][0] delta_{i+1}[j+1]
-// dz += delta; da_k = w_k sigmoid(-a_k) (dw_k - sum_k' w_k' dw_k') with dw_k = delta_i[j] h_{i-1}[j+k-1].
-template <typename T, unsigned D, int LPT>
-__device__ __forceinline__ void plane_reverse(const T* a3, T* da3, const float* g, const float* w0b, const float* w2b,
-                                             const float* hb, float* dz, int H, int W, int Wp, int lane) {
+// Reverse scan of direction D by one warp, delta only (no global memory):
+//   delta_i[j] = g_i[j] + w_{i+1}[j-1][2] delta_{i+1}[j-1] + w_{i+1}[j][1] delta_{i+1}[j]
+//                + w_{i+1}[j+1][0] delta_{i+1}[j+1]
+// into db (plane layout), and dz += delta. The operands of step i - 1 are loaded while step i
+// is formed.
+template <unsigned D, int LPT>
+__device__ __forceinline__ void plane_reverse(const float* g, const float* w0b, const float* w2b, float* db, float* dz,
+                                             int H, int W, int Wp, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
-    const int HW = H * W;
-    float del[LPT], pw0[LPT], pw1[LPT], pw2[LPT];   // delta and weights of step i+1
+    float del[LPT], pw0[LPT], pw1[LPT], pw2[LPT];   // delta and weights of step i + 1
+    float cg[LPT], cw0[LPT], cw2[LPT];              // g and weights of step i
+    int cq[LPT];
+    bool on[LPT];
 #pragma unroll
-    for (int e = 0; e < LPT; ++e) del[e] = pw0[e] = pw1[e] = pw2[e] = 0.f;
+    for (int e = 0; e < LPT; ++e) {
+        del[e] = pw0[e] = pw1[e] = pw2[e] = 0.f;
+        const int j = lane * LPT + e;
+        on[e] = j < M;
+        cq[e] = on[e] ? plane_pix<D>(H, W, Wp, L - 1, j) : 0;
+        cg[e] = g[cq[e]];
+        cw0[e] = w0b[cq[e]];
+        cw2[e] = w2b[cq[e]];
+    }
     for (int i = L - 1; i >= 0; --i) {
+        float ng[LPT], nw0[LPT], nw2[LPT];
+        int nq[LPT];
+#pragma unroll
+        for (int e = 0; e < LPT; ++e) {
+            nq[e] = (i > 0 && on[e]) ? plane_pix<D>(H, W, Wp, i - 1, lane * LPT + e) : 0;
+            ng[e] = g[nq[e]];
+            nw0[e] = w0b[nq[e]];
+            nw2[e] = w2b[nq[e]];
+        }
         // neighbour terms of w_{i+1}^T delta_{i+1}: lane j-1's (w2 delta) and lane j+1's (w0 delta)
         float fromL = __shfl_up_sync(0xffffffffu, pw2[LPT - 1] * del[LPT - 1], 1);
         float fromR = __shfl_down_sync(0xffffffffu, pw0[0] * del[0], 1);
         if (lane == 0) fromL = 0.f;
         if (lane == 31) fromR = 0.f;
-        float dn[LPT], nw0[LPT], nw1[LPT], nw2[LPT];
+        float dn[LPT];
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
-            const int j = lane * LPT + e;
-            dn[e] = nw0[e] = nw1[e] = nw2[e] = 0.f;
-            if (j < M) {
-                const int q = plane_pix<D>(H, W, Wp, i, j);
-                float d = g[q];
-                if (i < L - 1) {
-                    const float l = e == 0 ? fromL : pw2[e - 1] * del[e - 1];
-                    const float r = e == LPT - 1 ? fromR : pw0[e + 1] * del[e + 1];
-                    d = fmaf(pw1[e], del[e], d) + l + r;
-                }
-                dz[q] += d;
-                dn[e] = d;
-                // image offset of (i, j) for the logits / da
-                const int r0 = q / Wp, c0 = q - r0 * Wp;
-                const int gq = r0 * W + c0;
-                if (i > 0) {
-                    const float w0 = w0b[q], w2 = w2b[q], w1 = 1.f - w0 - w2;
-                    const bool hasl = j > 0, hasr = j < M - 1;
-                    const float h0 = hasl ? hb[plane_pix<D>(H, W, Wp, i - 1, j - 1)] : 0.f;
-                    const float h1 = hb[plane_pix<D>(H, W, Wp, i - 1, j)];
-                    const float h2 = hasr ? hb[plane_pix<D>(H, W, Wp, i - 1, j + 1)] : 0.f;
-                    const float dw0 = d * h0, dw1 = d * h1, dw2 = d * h2;
-                    const float sdw = w0 * dw0 + w1 * dw1 + w2 * dw2;
-                    const float a0 = Io<T>::ld(a3 + gq), a1 = Io<T>::ld(a3 + HW + gq), a2 = Io<T>::ld(a3 + 2 * HW + gq);
-                    Io<T>::st(da3 + gq, hasl ? w0 * sigmoidf_(-a0) * (dw0 - sdw) : 0.f);
-                    Io<T>::st(da3 + HW + gq, w1 * sigmoidf_(-a1) * (dw1 - sdw));
-                    Io<T>::st(da3 + 2 * HW + gq, hasr ? w2 * sigmoidf_(-a2) * (dw2 - sdw) : 0.f);
-                    nw0[e] = w0;
-                    nw1[e] = w1;
-                    nw2[e] = w2;
-                } else {
-                    Io<T>::st(da3 + gq, 0.f);
-                    Io<T>::st(da3 + HW + gq, 0.f);
-                    Io<T>::st(da3 + 2 * HW + gq, 0.f);
-                }
+            const float l = e == 0 ? fromL : pw2[e - 1] * del[e - 1];
+            const float r = e == LPT - 1 ? fromR : pw0[e + 1] * del[e + 1];
+            const float d = fmaf(pw1[e], del[e], cg[e]) + l + r;
+            dn[e] = on[e] ? d : 0.f;
+            if (on[e]) {
+                db[cq[e]] = d;
+                dz[cq[e]] += d;
             }
         }
+        // step i's weights become the "next step" weights of step i - 1 (row 0's weights are
+        // never applied: h_{-1} = 0, but w_0^T never enters delta either since it is the last)
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
             del[e] = dn[e];
-            pw0[e] = nw0[e];
-            pw1[e] = nw1[e];
-            pw2[e] = nw2[e];
+            pw0[e] = on[e] ? cw0[e] : 0.f;
+            pw2[e] = on[e] ? cw2[e] : 0.f;
+            pw1[e] = on[e] ? 1.f - cw0[e] - cw2[e] : 0.f;
+            cg[e] = ng[e];
+            cw0[e] = nw0[e];
+            cw2[e] = nw2[e];
+            cq[e] = nq[e];
+        }
+    }
+}
+
+// Logit gradients of direction D for the whole plane (all threads, image order, vector loads
+// and stores when W % 4 == 0): at scan position (i, j) with i > 0,
+//   dw_k = delta_i[j] h_{i-1}[j+k-1],  da_k = w_k sigmoid(-a_k) (dw_k - sum_k' w_k' dw_k')
+// (zero for out-of-range k); row i = 0 has zero gradient (its weights multiply h_{-1} = 0).
+template <typename T, unsigned D>
+__device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const float* w0b, const float* w2b,
+                                                  const float* hb, const float* db, int H, int W, int Wp, int tid) {
+    constexpr bool V = D == kTB || D == kBT;
+    const int M = V ? W : H;
+    const int HW = H * W;
+    auto grad = [&](float a0, float a1, float a2, int r, int c, float& g0, float& g1, float& g2) {
+        const int i = D == kTB ? r : D == kBT ? H - 1 - r : D == kLR ? c : W - 1 - c;
+        const int j = V ? c : r;
+        g0 = g1 = g2 = 0.f;
+        if (i > 0) {
+            const int q = r * Wp + c;
+            const float w0 = w0b[q], w2 = w2b[q], w1 = 1.f - w0 - w2;
+            const bool hasl = j > 0, hasr = j < M - 1;
+            const float d = db[q];
+            const float h0 = hasl ? hb[plane_pix<D>(H, W, Wp, i - 1, j - 1)] : 0.f;
+            const float h1 = hb[plane_pix<D>(H, W, Wp, i - 1, j)];
+            const float h2 = hasr ? hb[plane_pix<D>(H, W, Wp, i - 1, j + 1)] : 0.f;
+            const float dw0 = d * h0, dw1 = d * h1, dw2 = d * h2;
+            const float sdw = w0 * dw0 + w1 * dw1 + w2 * dw2;
+            g0 = hasl ? w0 * sigmoidf_(-a0) * (dw0 - sdw) : 0.f;
+            g1 = w1 * sigmoidf_(-a1) * (dw1 - sdw);
+            g2 = hasr ? w2 * sigmoidf_(-a2) * (dw2 - sdw) : 0.f;
+        }
+    };
+    if (W % 4 == 0) {
+        for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
+            const int r = e / W, c = e - r * W;
+            float a0[4], a1[4], a2[4], g0[4], g1[4], g2[4];
+            ld_lanes<T, 4>(a3 + e, a0);
+            ld_lanes<T, 4>(a3 + HW + e, a1);
+            ld_lanes<T, 4>(a3 + 2 * HW + e, a2);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) grad(a0[k], a1[k], a2[k], r, c + k, g0[k], g1[k], g2[k]);
+            st_lanes<T, 4>(da3 + e, g0);
+            st_lanes<T, 4>(da3 + HW + e, g1);
+            st_lanes<T, 4>(da3 + 2 * HW + e, g2);
+        }
+    } else {
+        for (int e = tid; e < HW; e += kPlaneThreads) {
+            const int r = e / W, c = e - r * W;
+            float g0, g1, g2;
+            grad(Io<T>::ld(a3 + e), Io<T>::ld(a3 + HW + e), Io<T>::ld(a3 + 2 * HW + e), r, c, g0, g1, g2);
+            Io<T>::st(da3 + e, g0);
+            Io<T>::st(da3 + HW + e, g1);
+            Io<T>::st(da3 + 2 * HW + e, g2);
         }
     }
 }
 
 template <typename T, unsigned D, int LPT>
 __device__ __forceinline__ void plane_bwd_direction(const T* a3, T* da3, const float* z, const float* g, float* w0b,
-                                                    float* w2b, float* hb, float* acc, float* dz, int H, int W, int Wp,
-                                                    int tid) {
+                                                    float* w2b, float* hb, float* db, float* acc, float* dz, int H,
+                                                    int W, int Wp, int tid) {
     plane_weights<T, D>(a3, w0b, w2b, H, W, Wp, tid);
     __syncthreads();
     if (tid < 32) {
         plane_recompute<D, LPT>(z, w0b, w2b, hb, acc, H, W, Wp, tid);
         __syncwarp();
-        plane_reverse<T, D, LPT>(a3, da3, g, w0b, w2b, hb, dz, H, W, Wp, tid);
+        plane_reverse<D, LPT>(g, w0b, w2b, db, dz, H, W, Wp, tid);
     }
+    __syncthreads();
+    plane_logit_grads<T, D>(a3, da3, w0b, w2b, hb, db, H, W, Wp, tid);
     __syncthreads();
 }
 
@@ -386,7 +462,8 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_bwd(PlaneBwdArgs p) {
     float* acc = g + HWs;
     float* dz = acc + HWs;
     float* hb = dz + HWs;
-    float* w0b = hb + HWs;
+    float* db = hb + HWs;
+    float* w0b = db + HWs;
     float* w2b = w0b + HWs;
     const int tid = threadIdx.x;
     const int HW = H * W;
@@ -402,12 +479,13 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_bwd(PlaneBwdArgs p) {
             acc[q] = 0.f;
             dz[q] = 0.f;
         }
+        __syncthreads();
         int slot = 0;
         auto aoff = [&](int s) { return (((long long)s * p.N + n) * p.C + c) * 3 * HW; };
-        if (p.mask & kTB) { const long long o = aoff(slot++); plane_bwd_direction<T, kTB, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
-        if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
-        if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
-        if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kTB) { const long long o = aoff(slot++); plane_bwd_direction<T, kTB, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
         for (int e = tid; e < HW; e += kPlaneThreads) {
             const int q = (e / W) * Wp + e % W;
             Io<T>::st((T*)p.dx + po + e, Io<T>::ld(lam + e) * dz[q]);
@@ -425,7 +503,7 @@ int plane_lanes(const Problem& P) {
     return M <= 32 ? 1 : (M <= 64 ? 2 : 4);
 }
 
-size_t plane_bwd_smem(const Problem& P) { return 7 * (size_t)P.H * plane_wp(P) * sizeof(float); }
+size_t plane_bwd_smem(const Problem& P) { return 8 * (size_t)P.H * plane_wp(P) * sizeof(float); }
 
 template <typename T, int LPT>
 cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
