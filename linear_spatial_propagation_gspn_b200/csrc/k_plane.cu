@@ -22,6 +22,8 @@ namespace gspn {
 namespace {
 
 constexpr int kPlaneThreads = 128;
+constexpr int kPlaneBwdThreads = 256;          // the backward runs one or two CTAs per SM: more warps
+                                               // for its parallel phases
 constexpr int kPlaneMaxLanes = 128;            // scan lanes held by one warp (4 per thread)
 constexpr size_t kPlaneSmemBudget = 225 * 1024;
 
@@ -125,7 +127,7 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
 
 // Weights of direction D for the whole plane into w0b / w2b (all threads; 4 pixels per
 // iteration when a row is a multiple of 4 long).
-template <typename T, unsigned D>
+template <typename T, unsigned D, int NT = kPlaneThreads>
 __device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2b, int H, int W, int Wp, int tid) {
     const int HW = H * W;
     if (W % 4 == 0) {
@@ -138,9 +140,9 @@ __device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2
             ld_lanes<T, 4>(a3 + HW + e, a1);
             ld_lanes<T, 4>(a3 + 2 * HW + e, a2);
         }
-        for (; e < HW; e += kPlaneThreads * 4) {
+        for (; e < HW; e += NT * 4) {
             float b0[4], b1[4], b2[4];
-            const int en = e + kPlaneThreads * 4;
+            const int en = e + NT * 4;
             if (en < HW) {
                 ld_lanes<T, 4>(a3 + en, b0);
                 ld_lanes<T, 4>(a3 + HW + en, b1);
@@ -158,7 +160,7 @@ __device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2
             }
         }
     } else {
-        for (int e = tid; e < HW; e += kPlaneThreads) {
+        for (int e = tid; e < HW; e += NT) {
             const int r = e / W, col = e - r * W;
             pixel_weights<D>(Io<T>::ld(a3 + e), Io<T>::ld(a3 + HW + e), Io<T>::ld(a3 + 2 * HW + e), r, col, H, W,
                              w0b[r * Wp + col], w2b[r * Wp + col]);
@@ -386,7 +388,7 @@ __device__ __forceinline__ void plane_reverse(const float* g, const float* w0b, 
 // and stores when W % 4 == 0): at scan position (i, j) with i > 0,
 //   dw_k = delta_i[j] h_{i-1}[j+k-1],  da_k = w_k sigmoid(-a_k) (dw_k - sum_k' w_k' dw_k')
 // (zero for out-of-range k); row i = 0 has zero gradient (its weights multiply h_{-1} = 0).
-template <typename T, unsigned D>
+template <typename T, unsigned D, int NT>
 __device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const float* w0b, const float* w2b,
                                                   const float* hb, const float* db, int H, int W, int Wp, int tid) {
     constexpr bool V = D == kTB || D == kBT;
@@ -406,13 +408,17 @@ __device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const flo
             const float h2 = hasr ? hb[plane_pix<D>(H, W, Wp, i - 1, j + 1)] : 0.f;
             const float dw0 = d * h0, dw1 = d * h1, dw2 = d * h2;
             const float sdw = w0 * dw0 + w1 * dw1 + w2 * dw2;
-            g0 = hasl ? w0 * sigmoidf_(-a0) * (dw0 - sdw) : 0.f;
-            g1 = w1 * sigmoidf_(-a1) * (dw1 - sdw);
-            g2 = hasr ? w2 * sigmoidf_(-a2) * (dw2 - sdw) : 0.f;
+            // sigmoid(-a) = 1 / (1 + exp(a)) from the MUFU exponential (relative error a few ulp,
+            // far inside the gradient tolerance); the argument is clamped at 80 so exp stays
+            // finite (sigmoid(-80) is 2e-35, indistinguishable from the limit 0 here)
+            auto sgm = [](float a) { return __fdividef(1.f, 1.f + __expf(fminf(a, 80.f))); };
+            g0 = hasl ? w0 * sgm(a0) * (dw0 - sdw) : 0.f;
+            g1 = w1 * sgm(a1) * (dw1 - sdw);
+            g2 = hasr ? w2 * sgm(a2) * (dw2 - sdw) : 0.f;
         }
     };
     if (W % 4 == 0) {
-        for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
+        for (int e = tid * 4; e < HW; e += NT * 4) {
             const int r = e / W, c = e - r * W;
             float a0[4], a1[4], a2[4], g0[4], g1[4], g2[4];
             ld_lanes<T, 4>(a3 + e, a0);
@@ -425,7 +431,7 @@ __device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const flo
             st_lanes<T, 4>(da3 + 2 * HW + e, g2);
         }
     } else {
-        for (int e = tid; e < HW; e += kPlaneThreads) {
+        for (int e = tid; e < HW; e += NT) {
             const int r = e / W, c = e - r * W;
             float g0, g1, g2;
             grad(Io<T>::ld(a3 + e), Io<T>::ld(a3 + HW + e), Io<T>::ld(a3 + 2 * HW + e), r, c, g0, g1, g2);
@@ -440,7 +446,7 @@ template <typename T, unsigned D, int LPT>
 __device__ __forceinline__ void plane_bwd_direction(const T* a3, T* da3, const float* z, const float* g, float* w0b,
                                                     float* w2b, float* hb, float* db, float* acc, float* dz, int H,
                                                     int W, int Wp, int tid) {
-    plane_weights<T, D>(a3, w0b, w2b, H, W, Wp, tid);
+    plane_weights<T, D, kPlaneBwdThreads>(a3, w0b, w2b, H, W, Wp, tid);
     __syncthreads();
     if (tid < 32) {
         plane_recompute<D, LPT>(z, w0b, w2b, hb, acc, H, W, Wp, tid);
@@ -448,12 +454,12 @@ __device__ __forceinline__ void plane_bwd_direction(const T* a3, T* da3, const f
         plane_reverse<D, LPT>(g, w0b, w2b, db, dz, H, W, Wp, tid);
     }
     __syncthreads();
-    plane_logit_grads<T, D>(a3, da3, w0b, w2b, hb, db, H, W, Wp, tid);
+    plane_logit_grads<T, D, kPlaneBwdThreads>(a3, da3, w0b, w2b, hb, db, H, W, Wp, tid);
     __syncthreads();
 }
 
 template <typename T, int LPT>
-__global__ void __launch_bounds__(kPlaneThreads) k_plane_bwd(PlaneBwdArgs p) {
+__global__ void __launch_bounds__(kPlaneBwdThreads) k_plane_bwd(PlaneBwdArgs p) {
     extern __shared__ float sm[];
     const int H = p.H, W = p.W, Wp = p.Wp;
     const int HWs = H * Wp;
@@ -472,7 +478,7 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_bwd(PlaneBwdArgs p) {
         const int n = plane / p.C, c = plane % p.C;
         const long long po = (long long)plane * HW;
         const T *x = (const T*)p.x + po, *lam = (const T*)p.lam + po, *u = (const T*)p.u + po, *dy = (const T*)p.dy + po;
-        for (int e = tid; e < HW; e += kPlaneThreads) {
+        for (int e = tid; e < HW; e += kPlaneBwdThreads) {
             const int q = (e / W) * Wp + e % W;
             z[q] = Io<T>::ld(lam + e) * Io<T>::ld(x + e);
             g[q] = Io<T>::ld(u + e) * Io<T>::ld(dy + e);
@@ -486,7 +492,7 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_bwd(PlaneBwdArgs p) {
         if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
         if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
         if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
-        for (int e = tid; e < HW; e += kPlaneThreads) {
+        for (int e = tid; e < HW; e += kPlaneBwdThreads) {
             const int q = (e / W) * Wp + e % W;
             Io<T>::st((T*)p.dx + po + e, Io<T>::ld(lam + e) * dz[q]);
             Io<T>::st((T*)p.dlam + po + e, Io<T>::ld(x + e) * dz[q]);
@@ -512,12 +518,12 @@ cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream
     if (e != cudaSuccess) return e;
     cudaFuncSetAttribute(k_plane_bwd<T, LPT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int per_sm = 1;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_bwd<T, LPT>, kPlaneThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_bwd<T, LPT>, kPlaneBwdThreads, smem);
     if (e != cudaSuccess) return e;
     const long long want = (long long)std::max(1, per_sm) * device_sm_count();
     const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
     launch_begin(st);
-    k_plane_bwd<T, LPT><<<grid, kPlaneThreads, smem, st>>>(a);
+    k_plane_bwd<T, LPT><<<grid, kPlaneBwdThreads, smem, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
 }
