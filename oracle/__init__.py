@@ -56,6 +56,12 @@ def _load():
         lib.gspn_ref_forward.restype = ctypes.c_int
         lib.gspn_ref_backward.argtypes = args + [dp] * 9
         lib.gspn_ref_backward.restype = ctypes.c_int
+        lib.gspn_ref_forward_chunked.argtypes = args + [ctypes.c_int] + [dp] * 5
+        lib.gspn_ref_forward_chunked.restype = ctypes.c_int
+        lib.gspn_ref_backward_chunked.argtypes = args + [ctypes.c_int] + [dp] * 9
+        lib.gspn_ref_backward_chunked.restype = ctypes.c_int
+        if lib.gspn_ref_abi_version() != 2:
+            raise RuntimeError("stale oracle build; rebuild with oracle.build(force=True)")
         _lib = lib
     return _lib
 
@@ -83,18 +89,20 @@ def _check_shapes(x, a, lam, u, wmode, mask):
     return N, C, H, W
 
 
-def forward(x, a, lam, u, wmode: int = 0, mask: int = 15) -> np.ndarray:
-    """y = u * sum_{d in mask} h^d, float64. ``wmode`` 0 = per-channel, 1 = shared."""
+def forward(x, a, lam, u, wmode: int = 0, mask: int = 15, chunk: int = 0) -> np.ndarray:
+    """y = u * sum_{d in mask} h^d, float64. ``wmode`` 0 = per-channel, 1 = shared; ``chunk``
+    > 0: local propagation within image-aligned chunks of that many lines (0 = global)."""
     x, a, lam, u = _f64(x), _f64(a), _f64(lam), _f64(u)
     N, C, H, W = _check_shapes(x, a, lam, u, wmode, mask)
     y = np.empty_like(x)
-    rc = _load().gspn_ref_forward(N, C, H, W, int(wmode), int(mask), _ptr(x), _ptr(a), _ptr(lam), _ptr(u), _ptr(y))
+    rc = _load().gspn_ref_forward_chunked(N, C, H, W, int(wmode), int(mask), int(chunk), _ptr(x), _ptr(a),
+                                          _ptr(lam), _ptr(u), _ptr(y))
     if rc:
         raise RuntimeError(f"gspn_ref_forward failed ({rc})")
     return y
 
 
-def backward(x, a, lam, u, dy, wmode: int = 0, mask: int = 15):
+def backward(x, a, lam, u, dy, wmode: int = 0, mask: int = 15, chunk: int = 0):
     """Returns (dx, da, dlam, du), float64, for the loss sum(dy * y)."""
     x, a, lam, u, dy = _f64(x), _f64(a), _f64(lam), _f64(u), _f64(dy)
     N, C, H, W = _check_shapes(x, a, lam, u, wmode, mask)
@@ -102,8 +110,8 @@ def backward(x, a, lam, u, dy, wmode: int = 0, mask: int = 15):
         raise ValueError("dy must have the shape of x")
     dx, dlam, du = np.empty_like(x), np.empty_like(x), np.empty_like(x)
     da = np.empty_like(a)
-    rc = _load().gspn_ref_backward(N, C, H, W, int(wmode), int(mask), _ptr(x), _ptr(a), _ptr(lam), _ptr(u),
-                                   _ptr(dy), _ptr(dx), _ptr(da), _ptr(dlam), _ptr(du))
+    rc = _load().gspn_ref_backward_chunked(N, C, H, W, int(wmode), int(mask), int(chunk), _ptr(x), _ptr(a),
+                                           _ptr(lam), _ptr(u), _ptr(dy), _ptr(dx), _ptr(da), _ptr(dlam), _ptr(du))
     if rc:
         raise RuntimeError(f"gspn_ref_backward failed ({rc})")
     return dx, da, dlam, du

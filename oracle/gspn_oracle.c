@@ -39,6 +39,16 @@
  *  - Neighbour k in {0,1,2} is lane j+k-1, i.e. ordered by increasing image coordinate
  *    on the axis across the scan. The 3 logits of hidden pixel (r,c) are stored at
  *    image position (r,c).
+ *
+ * Local (chunked) propagation. The pages contrast local and global GSPN ("Parallel
+ * Sequence Modeling via Generalized Spatial Propagation Network" summary, section
+ * "Measured effects": a hybrid of local and global layers beats all-local ones) and give
+ * the fused kernel a chunk grid axis ("GSPN-2 ..." paper notes, "Optimisation 1"), but do
+ * not spell the local rule out. Reading used here: with chunk length K > 0 the image is cut
+ * along each direction's scan axis into chunks of K lines aligned to line 0 (rows for
+ * TB/BT, columns for LR/RL) and propagation does not cross a chunk boundary: the scan
+ * restarts from h = 0 at the first line of every chunk in scan order. K = 0 is the global
+ * scan. The *_chunked entry points take K; the plain ones are K = 0.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -83,17 +93,32 @@ static void row_weights(const double av[3], int j, int M, double w[3], double s[
     *S = sum;
 }
 
+/* Whether scan step i of direction d starts a chunk (h restarts from 0 there). */
+static int chunk_start(unsigned d, int H, int W, int chunk, int i) {
+    if (i == 0) return 1;
+    if (chunk <= 0) return 0;
+    int line; /* image row (TB, BT) or column (LR, RL) of step i */
+    switch (d) {
+    case DIR_TB: line = i;         break;
+    case DIR_BT: line = H - 1 - i; break;
+    case DIR_LR: line = i;         break;
+    default:     line = W - 1 - i; break; /* RL */
+    }
+    if (d == DIR_TB || d == DIR_LR) return line % chunk == 0;  /* first line of its chunk */
+    return (line + 1) % chunk == 0;                            /* last line of its chunk */
+}
+
 static int popcount4(unsigned m) { int n = 0; for (int b = 0; b < 4; ++b) n += (m >> b) & 1u; return n; }
 
-static int check_args(int N, int C, int H, int W, int wmode, unsigned mask) {
-    if (N < 1 || C < 1 || H < 1 || W < 1) return 1;
+static int check_args(int N, int C, int H, int W, int wmode, unsigned mask, int chunk) {
+    if (N < 1 || C < 1 || H < 1 || W < 1 || chunk < 0) return 1;
     if (wmode != 0 && wmode != 1) return 1;
     if (mask < 1u || mask > 15u) return 1;
     return 0;
 }
 
 /* Forward scan of one (n, c, d): fills hbuf[i*M + j] (scan coordinates). */
-static void scan_forward(unsigned d, int H, int W, const double *x, const double *lam,
+static void scan_forward(unsigned d, int H, int W, int chunk, const double *x, const double *lam,
                          const double *a3 /* 3 planes of H*W */, double *hbuf) {
     int L, M;
     geom(d, H, W, &L, &M);
@@ -103,7 +128,7 @@ static void scan_forward(unsigned d, int H, int W, const double *x, const double
             long p = pix(d, H, W, i, j);
             double z = lam[p] * x[p];
             double acc = z;
-            if (i > 0) {
+            if (!chunk_start(d, H, W, chunk, i)) {
                 double av[3] = {a3[p], a3[HW + p], a3[2 * HW + p]}, w[3], s[3], S;
                 row_weights(av, j, M, w, s, &S);
                 for (int k = 0; k < 3; ++k) {
@@ -120,10 +145,10 @@ static long logit_base(int slot, int n, int cw, int N, int Cw, long HW) {
     return (((long)slot * N + n) * Cw + cw) * 3 * HW;
 }
 
-int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
-                     const double *x, const double *a, const double *lam, const double *u,
-                     double *y) {
-    if (check_args(N, C, H, W, wmode, mask)) return 1;
+int gspn_ref_forward_chunked(int N, int C, int H, int W, int wmode, unsigned mask, int chunk,
+                             const double *x, const double *a, const double *lam, const double *u,
+                             double *y) {
+    if (check_args(N, C, H, W, wmode, mask, chunk)) return 1;
     const long HW = (long)H * W;
     const int Cw = wmode ? 1 : C;
     const int Lmax = H > W ? H : W;
@@ -138,7 +163,7 @@ int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
             for (unsigned d = DIR_TB; d <= DIR_RL; d <<= 1) {
                 if (!(mask & d)) continue;
                 const double *a3 = a + logit_base(slot, n, wmode ? 0 : c, N, Cw, HW);
-                scan_forward(d, H, W, x + off, lam + off, a3, hbuf);
+                scan_forward(d, H, W, chunk, x + off, lam + off, a3, hbuf);
                 int L, M;
                 geom(d, H, W, &L, &M);
                 for (int i = 0; i < L; ++i)
@@ -153,6 +178,12 @@ int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
     return 0;
 }
 
+int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
+                     const double *x, const double *a, const double *lam, const double *u,
+                     double *y) {
+    return gspn_ref_forward_chunked(N, C, H, W, wmode, mask, 0, x, a, lam, u, y);
+}
+
 /*
  * Backward (the adjoint of the forward above, written from the chain rule):
  *   acc = sum_d h^d,  du = dy (.) acc,  g = dy (.) u.
@@ -165,11 +196,13 @@ int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
  *   w_k = s_k / S with s_k = sigmoid(a_k):
  *     da_k = s_k (1 - s_k) (dw_k - sum_{k' in range} w_k' dw_k') / S  for in-range k,
  *     da_k = 0 for out-of-range k. In the shared mode da is summed over channels.
+ *   With chunks, a step that starts a chunk behaves like step 0: its weights multiply
+ *   h = 0 (zero logit gradient) and no delta flows back through them.
  */
-int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
-                      const double *x, const double *a, const double *lam, const double *u,
-                      const double *dy, double *dx, double *da, double *dlam, double *du) {
-    if (check_args(N, C, H, W, wmode, mask)) return 1;
+int gspn_ref_backward_chunked(int N, int C, int H, int W, int wmode, unsigned mask, int chunk,
+                              const double *x, const double *a, const double *lam, const double *u,
+                              const double *dy, double *dx, double *da, double *dlam, double *du) {
+    if (check_args(N, C, H, W, wmode, mask, chunk)) return 1;
     const long HW = (long)H * W;
     const int Cw = wmode ? 1 : C;
     const int D = popcount4(mask);
@@ -200,7 +233,7 @@ int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
                 double *da3 = da + ab;
                 int L, M;
                 geom(d, H, W, &L, &M);
-                scan_forward(d, H, W, xp, lp, a3, hbuf);
+                scan_forward(d, H, W, chunk, xp, lp, a3, hbuf);
                 for (int i = 0; i < L; ++i)
                     for (int j = 0; j < M; ++j) acc[pix(d, H, W, i, j)] += hbuf[(long)i * M + j];
                 /* reverse scan */
@@ -224,7 +257,7 @@ int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
                         long p = pix(d, H, W, i, j);
                         double av[3] = {a3[p], a3[HW + p], a3[2 * HW + p]}, w[3], s[3], S;
                         row_weights(av, j, M, w, s, &S);
-                        if (i > 0) {
+                        if (!chunk_start(d, H, W, chunk, i)) {
                             double dw[3] = {0.0, 0.0, 0.0}, wdw = 0.0;
                             for (int k = 0; k < 3; ++k) {
                                 int jj = j + k - 1;
@@ -239,7 +272,7 @@ int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
                                     da3[k * HW + p] += s[k] * (1.0 - s[k]) * (dw[k] - wdw) / S;
                             }
                         } else {
-                            /* w_0 multiplies h_{-1} = 0: no effect on the output */
+                            /* w_0 (and a chunk's first w) multiplies h = 0: no effect on the output */
                             for (int k = 0; k < 3; ++k) w[k] = 0.0;
                         }
                         for (int k = 0; k < 3; ++k) wnext[3 * (long)j + k] = w[k];
@@ -259,5 +292,11 @@ int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
     return 0;
 }
 
+int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
+                      const double *x, const double *a, const double *lam, const double *u,
+                      const double *dy, double *dx, double *da, double *dlam, double *du) {
+    return gspn_ref_backward_chunked(N, C, H, W, wmode, mask, 0, x, a, lam, u, dy, dx, da, dlam, du);
+}
+
 /* Version tag so that a loader can check it got this file's build. */
-int gspn_ref_abi_version(void) { return 1; }
+int gspn_ref_abi_version(void) { return 2; }

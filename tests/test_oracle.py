@@ -319,3 +319,106 @@ def test_mutation_is_detected():
     good = brute.forward(x, a, lam, u, 0, 1)
     wrong = oracle.forward(x, a[:, :, :, ::-1].copy(), lam, u, 0, 1)
     assert np.abs(good - wrong).max() > 1e-3
+
+
+# ----------------------------------------------------------------------------- local (chunked) scans
+# Reading: with chunk length K the image is cut into K-line chunks along each direction's scan
+# axis, aligned to image line 0, and propagation never crosses a chunk boundary.
+
+def _slot_of(mask, d):
+    return bin(mask & (d - 1)).count("1")
+
+
+@pytest.mark.parametrize("wmode", [0, 1])
+def test_chunk_at_least_the_map_is_global(wmode):
+    rng = np.random.default_rng(70 + wmode)
+    x, a, lam, u = rand_case(rng, 1, 2, 6, 5, 15, wmode)
+    y0 = oracle.forward(x, a, lam, u, wmode, 15)
+    for k in (6, 7, 100):
+        assert np.array_equal(oracle.forward(x, a, lam, u, wmode, 15, chunk=k), y0)
+
+
+@pytest.mark.parametrize("mask", [1, 2, 4, 8, 15, 6])
+def test_chunk_of_one_line_is_pure_injection(mask):
+    """K = 1: every line starts a chunk, h = z everywhere, y = u * D * lambda * x."""
+    rng = np.random.default_rng(80 + mask)
+    x, a, lam, u = rand_case(rng, 2, 2, 5, 7, mask, 0)
+    y = oracle.forward(x, a, lam, u, 0, mask, chunk=1)
+    D = bin(mask).count("1")
+    assert np.abs(y - u * D * lam * x).max() <= 1e-12
+
+
+@pytest.mark.parametrize("d", [1, 2, 4, 8])
+@pytest.mark.parametrize("K", [2, 3, 4])
+def test_chunked_scan_is_the_global_scan_of_each_block(d, K):
+    """A chunked single-direction scan equals the global scan run separately on each
+    image-aligned block of K lines (rows for TB/BT, columns for LR/RL), including the short
+    last block; this pins the block alignment for the descending scans too."""
+    rng = np.random.default_rng(90 + d + 10 * K)
+    H, W = 7, 8
+    x, a, lam, u = rand_case(rng, 1, 2, H, W, d, 0)
+    y = oracle.forward(x, a, lam, u, 0, d, chunk=K)
+    vertical = d in (1, 2)
+    L = H if vertical else W
+    ref = np.zeros_like(y)
+    for s0 in range(0, L, K):
+        sl = slice(s0, min(L, s0 + K))
+        if vertical:
+            blk = [t[:, :, sl, :] for t in (x, lam, u)]
+            ab = a[:, :, :, :, sl, :]
+            ref[:, :, sl, :] = oracle.forward(blk[0], ab, blk[1], blk[2], 0, d)
+        else:
+            blk = [t[:, :, :, sl] for t in (x, lam, u)]
+            ab = a[:, :, :, :, :, sl]
+            ref[:, :, :, sl] = oracle.forward(blk[0], ab, blk[1], blk[2], 0, d)
+    assert np.abs(y - ref).max() <= 1e-12
+
+
+def test_chunked_directions_add_up():
+    """The 4-direction chunked result is the sum of the single-direction chunked results."""
+    rng = np.random.default_rng(95)
+    x, a, lam, u = rand_case(rng, 1, 2, 6, 9, 15, 1)
+    y = oracle.forward(x, a, lam, u, 1, 15, chunk=4)
+    parts = sum(oracle.forward(x, a[_slot_of(15, d):_slot_of(15, d) + 1], lam, u, 1, d, chunk=4) for d in (1, 2, 4, 8))
+    assert np.abs(y - parts).max() <= 1e-12
+
+
+@pytest.mark.parametrize("wmode", [0, 1])
+@pytest.mark.parametrize("mask,K", [(15, 2), (1, 3), (2, 3), (8, 2)])
+def test_chunked_backward_finite_differences(wmode, mask, K):
+    rng = np.random.default_rng(97 + mask + 7 * K + 100 * wmode)
+    x, a, lam, u = rand_case(rng, 1, 2, 5, 5, mask, wmode)
+    dy = rng.standard_normal(x.shape)
+    grads = oracle.backward(x, a, lam, u, dy, wmode, mask, chunk=K)
+    args = [x, a, lam, u]
+    eps = 1e-6
+
+    def loss():
+        return float((dy * oracle.forward(*args, wmode, mask, chunk=K)).sum())
+
+    for gi in range(4):
+        base = args[gi]
+        fd = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = base[idx]
+            base[idx] = old + eps
+            lp = loss()
+            base[idx] = old - eps
+            lm = loss()
+            base[idx] = old
+            fd[idx] = (lp - lm) / (2 * eps)
+        scale = max(1.0, np.abs(fd).max())
+        assert np.abs(grads[gi] - fd).max() <= 1e-6 * scale, (gi, np.abs(grads[gi] - fd).max())
+
+
+def test_chunk_start_logits_have_zero_gradient():
+    """The weights of a chunk's first line multiply h = 0: their logit gradient is zero."""
+    rng = np.random.default_rng(99)
+    x, a, lam, u = rand_case(rng, 1, 1, 7, 5, 1, 0)   # TB only
+    dy = rng.standard_normal(x.shape)
+    _, da, _, _ = oracle.backward(x, a, lam, u, dy, 0, 1, chunk=3)
+    for r in (0, 3, 6):
+        assert np.all(da[0, 0, 0, :, r, :] == 0.0)
+    assert np.abs(da[0, 0, 0, :, 1, :]).max() > 0.0
