@@ -84,15 +84,25 @@ enum { GSPN_DIR_TB = 1, GSPN_DIR_BT = 2, GSPN_DIR_LR = 4, GSPN_DIR_RL = 8, GSPN_
  * on the same inputs.
  *   GENERIC: any shape; one CTA per plane and direction, hidden line in shared memory.
  *   PLANE:   small maps; the whole plane stays on chip and all directions run in one pass.
- *   SWEEP:   large maps; persistent TMA-fed line sweeps, one direction pair per kernel. */
+ *   SWEEP:   large maps (forward): persistent line sweeps fed by per-thread asynchronous copies,
+ *            one launch per direction plus one for the weights. */
 enum { GSPN_ALGO_AUTO = 0, GSPN_ALGO_GENERIC = 1, GSPN_ALGO_PLANE = 2, GSPN_ALGO_SWEEP = 3 };
 
+/* chunk: 0 = global propagation over the whole map. K > 0 = local propagation: the map is cut
+ * along each direction's scan axis into chunks of K lines aligned to image line 0 (rows for
+ * top->bottom / bottom->top, columns for left->right / right->left) and propagation does not
+ * cross a chunk boundary (the scan restarts from h = 0 at the first line of every chunk in scan
+ * order; the logits of that line get zero gradient). The pages contrast local and global GSPN
+ * ("Parallel Sequence Modeling via Generalized Spatial Propagation Network" summary, section
+ * "Measured effects") and give the fused kernel a chunk grid axis ("GSPN-2: Efficient Parallel
+ * Sequence Modeling" paper notes, "Optimisation 1"). Negative: GSPN_ERR_INVALID_ARG. */
 typedef struct {
     int N, C, H, W;
     int wmode;          /* gspn_wmode */
     unsigned dir_mask;  /* GSPN_DIR_* bits */
     int dtype;          /* gspn_dtype */
     int algo;           /* GSPN_ALGO_*, 0 = AUTO */
+    int chunk;          /* lines per local chunk; 0 = global */
 } gspn_desc;
 
 /* Bytes of device workspace that gspn_forward (for_backward = 0) or gspn_backward

@@ -19,11 +19,14 @@ bool make_problem(const gspn_desc* d, Problem* p) {
     if (d->dir_mask < 1u || d->dir_mask > 15u) return false;
     if (d->dtype != GSPN_F32 && d->dtype != GSPN_BF16) return false;
     if (d->algo < GSPN_ALGO_AUTO || d->algo > GSPN_ALGO_SWEEP) return false;
+    if (d->chunk < 0) return false;
     if ((long long)d->N * d->C > 0x7fffffffLL) return false;
     p->N = d->N; p->C = d->C; p->H = d->H; p->W = d->W;
     p->wmode = d->wmode;
     p->mask = d->dir_mask;
     p->dtype = d->dtype;
+    // a chunk at least as long as both axes is the global scan
+    p->chunk = d->chunk >= (d->H > d->W ? d->H : d->W) ? 0 : d->chunk;
     p->Cw = d->wmode == GSPN_W_SHARED ? 1 : d->C;
     p->D = __builtin_popcount(d->dir_mask);
     p->HW = (long long)d->H * d->W;
@@ -131,7 +134,7 @@ using namespace gspn;
 
 extern "C" {
 
-int gspn_version(void) { return 1; }
+int gspn_version(void) { return 2; }
 
 const char* gspn_status_string(gspn_status s) {
     switch (s) {

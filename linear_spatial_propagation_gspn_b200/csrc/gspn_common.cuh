@@ -137,6 +137,25 @@ __host__ __device__ __forceinline__ int dir_slot(unsigned mask, unsigned d) {
     return s;
 }
 
+// ------------------------------------------------------------------ local (chunked) scans
+// Local propagation restarts a scan from h = 0 at the first line, in scan order, of every chunk
+// of `chunk` image lines along the scan axis (chunks aligned to image line 0; 0 = global). In
+// scan coordinates with L steps an ascending scan (TB, LR) restarts at i % chunk == 0 and a
+// descending one (BT, RL) at i == 0 and wherever (L - i) % chunk == 0 (the step whose image line
+// is the last of its chunk).
+__host__ __device__ __forceinline__ bool chunk_start(bool asc, int L, int chunk, int i) {
+    if (i == 0) return true;
+    if (chunk <= 0) return false;
+    return asc ? (i % chunk == 0) : ((L - i) % chunk == 0);
+}
+// Steps in a scan's first chunk; every later chunk has `chunk` steps (the last may be short).
+// Scan loops count down from it instead of dividing every step. Global: L.
+__host__ __device__ __forceinline__ int first_chunk_len(bool asc, int L, int chunk) {
+    if (chunk <= 0 || chunk >= L) return L;
+    return asc ? chunk : ((L - 1) % chunk) + 1;
+}
+__host__ __device__ __forceinline__ bool scan_ascending(unsigned d) { return d == kTB || d == kLR; }
+
 // ------------------------------------------------------------------ weights
 // Normalised weights (w0, w1, w2) of one hidden lane from its logits. has_l / has_r tell
 // whether lanes j-1 / j+1 exist. With p_k = 1 + exp(-a_k) (so sigmoid = 1/p_k), multiplying

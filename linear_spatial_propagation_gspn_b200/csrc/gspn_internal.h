@@ -16,6 +16,7 @@ struct Problem {
     int wmode;
     unsigned mask;
     int dtype;       // GSPN_F32 / GSPN_BF16
+    int chunk;       // lines per local chunk (0: global)
     long long HW;    // H * W
     long long U;     // N * C * H * W
     long long A;     // D * N * Cw * 3 * H * W

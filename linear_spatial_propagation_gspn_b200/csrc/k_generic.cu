@@ -31,6 +31,7 @@ struct GenArgs {
     unsigned dir;
     int slot;
     int first, last;    // first / last direction of the mask
+    int chunk;          // lines per local chunk (0: global)
 };
 
 // Forward scan of one direction for plane blockIdx.x. Writes y (last direction), the fp32
@@ -56,7 +57,7 @@ __global__ void k_gen_fwd(GenArgs p) {
         for (int j = threadIdx.x; j < M; j += blockDim.x) {
             const long long q = scan_pixel(p.dir, p.H, p.W, i, j);
             float h = Io<T>::ld(lam + q) * Io<T>::ld(x + q);
-            if (i > 0) {
+            if (!chunk_start(scan_ascending(p.dir), L, p.chunk, i)) {
                 float w0, w1, w2;
                 lane_weights(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q), Io<T>::ld(a3 + 2 * HW + q), j > 0,
                              j < M - 1, w0, w1, w2);
@@ -96,6 +97,7 @@ struct GenBwdArgs {
     unsigned dir;
     int slot;
     int first;
+    int chunk;           // lines per local chunk (0: global)
 };
 
 // Reverse scan of one direction for plane blockIdx.x:
@@ -125,7 +127,8 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
         for (int j = threadIdx.x; j < M; j += blockDim.x) {
             const long long q = scan_pixel(p.dir, p.H, p.W, i, j);
             float del = Io<T>::ld(u + q) * Io<T>::ld(dy + q);
-            if (i < L - 1) {
+            // no delta flows back through the first line of a chunk (it does not see h_{i-1})
+            if (i < L - 1 && !chunk_start(scan_ascending(p.dir), L, p.chunk, i + 1)) {
                 // (w_{i+1}^T delta_{i+1})[j] = w[j-1][2] d[j-1] + w[j][1] d[j] + w[j+1][0] d[j+1]
                 if (j > 0) del = fmaf(wprev[2 * M + j - 1], dprev[j - 1], del);
                 del = fmaf(wprev[M + j], dprev[j], del);
@@ -134,7 +137,7 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
             dcur[j] = del;
             if (p.first) dz[q] = del;
             else dz[q] += del;
-            if (i > 0) {
+            if (!chunk_start(scan_ascending(p.dir), L, p.chunk, i)) {
                 const bool hl = j > 0, hr = j < M - 1;
                 LaneJac J = lane_jacobian(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q), Io<T>::ld(a3 + 2 * HW + q),
                                           hl, hr);
@@ -196,7 +199,8 @@ cudaError_t gen_forward_t(const Problem& P, const void* x, const void* a, const 
     int slot = 0, seen = 0;
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
-        GenArgs g{x, a, lam, u, y, acc, nullptr, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, seen == P.D - 1};
+        GenArgs g{x, a, lam, u, y, acc, nullptr, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, seen == P.D - 1,
+                  P.chunk};
         const int M = is_vertical(d) ? P.W : P.H;
         const size_t smem = 2 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -229,14 +233,16 @@ cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const
         if (!(P.mask & d)) continue;
         const int M = is_vertical(d) ? P.W : P.H;
         // 1) recompute this direction's h (image coordinates) and accumulate sum_d h for du
-        GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, false};
+        GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, false,
+                  P.chunk};
         if (P.D == 1) g.first = 1;
         size_t smem = 2 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_gen_fwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(g);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         // 2) reverse scan
-        GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, P.H, P.W, P.Cw, d, slot, seen == 0};
+        GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, P.H, P.W, P.Cw, d, slot, seen == 0,
+                     P.chunk};
         smem = 8 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_gen_bwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(b);

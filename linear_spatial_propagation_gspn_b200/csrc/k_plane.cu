@@ -35,6 +35,7 @@ struct PlaneArgs {
     void* y;
     int N, C, H, W, Cw, Wp;
     unsigned mask;
+    int chunk;   // lines per local chunk (0: global)
 };
 
 // Weights of one pixel for direction d (w1 = 1 - w0 - w2 is re-derived by the scan). Fast MUFU
@@ -67,7 +68,7 @@ __device__ __forceinline__ int plane_pix(int H, int W, int Wp, int i, int j) {
 // the recurrence. Lanes past the line (j >= M) read index 0 and contribute nothing.
 template <unsigned D, int LPT>
 __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, const float* w2b, float* acc, int H,
-                                           int W, int Wp, int lane) {
+                                           int W, int Wp, int chunk, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
     float h[LPT], cz[LPT], cw0[LPT], cw2[LPT], ca[LPT];
@@ -111,11 +112,13 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
             if (on[e]) acc[cq[e]] = ca[e] + v;
         }
         // the running sum of step i + 1 is read after this step's writes (different pixels
-        // except at the same lane, which this thread owns)
+        // except at the same lane, which this thread owns); a chunk's first step starts from
+        // h = 0 (local propagation)
+        const bool restart = more && chunk_start(scan_ascending(D), L, chunk, i + 1);
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
             na[e] = acc[nq[e]];
-            h[e] = hn[e];
+            h[e] = restart ? 0.f : hn[e];
             cz[e] = nz[e];
             cw0[e] = nw0[e];
             cw2[e] = nw2[e];
@@ -170,10 +173,10 @@ __device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2
 
 template <typename T, unsigned D, int LPT>
 __device__ __forceinline__ void plane_direction(const T* a3, const float* z, float* w0b, float* w2b, float* acc, int H,
-                                                int W, int Wp, int tid) {
+                                                int W, int Wp, int chunk, int tid) {
     plane_weights<T, D>(a3, w0b, w2b, H, W, Wp, tid);
     __syncthreads();
-    if (tid < 32) plane_scan<D, LPT>(z, w0b, w2b, acc, H, W, Wp, tid);
+    if (tid < 32) plane_scan<D, LPT>(z, w0b, w2b, acc, H, W, Wp, chunk, tid);
     __syncthreads();
 }
 
@@ -221,10 +224,10 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
         auto a_of = [&](int s) {
             return (const T*)p.a + (((long long)s * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
         };
-        if (p.mask & kTB) plane_direction<T, kTB, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
-        if (p.mask & kBT) plane_direction<T, kBT, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
-        if (p.mask & kLR) plane_direction<T, kLR, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
-        if (p.mask & kRL) plane_direction<T, kRL, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, tid);
+        if (p.mask & kTB) plane_direction<T, kTB, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
+        if (p.mask & kBT) plane_direction<T, kBT, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
+        if (p.mask & kLR) plane_direction<T, kLR, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
+        if (p.mask & kRL) plane_direction<T, kRL, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
         // y = u * sum
         if (vec) {
             for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
@@ -258,13 +261,14 @@ struct PlaneBwdArgs {
     void* du;
     int N, C, H, W, Wp;
     unsigned mask;
+    int chunk;   // lines per local chunk (0: global)
 };
 
 // Forward recompute of direction D by one warp: hb = h^D (plane layout), acc += h^D. Software
 // pipelined like plane_scan.
 template <unsigned D, int LPT>
 __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b, const float* w2b, float* hb,
-                                                float* acc, int H, int W, int Wp, int lane) {
+                                                float* acc, int H, int W, int Wp, int chunk, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
     float h[LPT], cz[LPT], cw0[LPT], cw2[LPT];
@@ -306,9 +310,10 @@ __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b
                 acc[cq[e]] += v;
             }
         }
+        const bool restart = more && chunk_start(scan_ascending(D), L, chunk, i + 1);
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
-            h[e] = hn[e];
+            h[e] = restart ? 0.f : hn[e];
             cz[e] = nz[e];
             cw0[e] = nw0[e];
             cw2[e] = nw2[e];
@@ -317,6 +322,9 @@ __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b
     }
 }
 
+// Whether step i's weights act on h_{i-1} (false at step 0 and at every chunk start).
+__device__ __forceinline__ bool on_any_weights(bool asc, int L, int chunk, int i) { return !chunk_start(asc, L, chunk, i); }
+
 // Reverse scan of direction D by one warp, delta only (no global memory):
 //   delta_i[j] = g_i[j] + w_{i+1}[j-1][2] delta_{i+1}[j-1] + w_{i+1}[j][1] delta_{i+1}[j]
 //                + w_{i+1}[j+1][0] delta_{i+1}[j+1]
@@ -324,7 +332,7 @@ __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b
 // is formed.
 template <unsigned D, int LPT>
 __device__ __forceinline__ void plane_reverse(const float* g, const float* w0b, const float* w2b, float* db, float* dz,
-                                             int H, int W, int Wp, int lane) {
+                                             int H, int W, int Wp, int chunk, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
     float del[LPT], pw0[LPT], pw1[LPT], pw2[LPT];   // delta and weights of step i + 1
@@ -368,14 +376,15 @@ __device__ __forceinline__ void plane_reverse(const float* g, const float* w0b, 
                 dz[cq[e]] += d;
             }
         }
-        // step i's weights become the "next step" weights of step i - 1 (row 0's weights are
-        // never applied: h_{-1} = 0, but w_0^T never enters delta either since it is the last)
+        // step i's weights become the "next step" weights of step i - 1; a step that starts a
+        // chunk (step 0 included) does not see h_{i-1}, so nothing flows back through it
+        const bool live = on_any_weights(scan_ascending(D), L, chunk, i);
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
             del[e] = dn[e];
-            pw0[e] = on[e] ? cw0[e] : 0.f;
-            pw2[e] = on[e] ? cw2[e] : 0.f;
-            pw1[e] = on[e] ? 1.f - cw0[e] - cw2[e] : 0.f;
+            pw0[e] = (on[e] && live) ? cw0[e] : 0.f;
+            pw2[e] = (on[e] && live) ? cw2[e] : 0.f;
+            pw1[e] = (on[e] && live) ? 1.f - cw0[e] - cw2[e] : 0.f;
             cg[e] = ng[e];
             cw0[e] = nw0[e];
             cw2[e] = nw2[e];
@@ -390,7 +399,8 @@ __device__ __forceinline__ void plane_reverse(const float* g, const float* w0b, 
 // (zero for out-of-range k); row i = 0 has zero gradient (its weights multiply h_{-1} = 0).
 template <typename T, unsigned D, int NT>
 __device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const float* w0b, const float* w2b,
-                                                  const float* hb, const float* db, int H, int W, int Wp, int tid) {
+                                                  const float* hb, const float* db, int H, int W, int Wp, int chunk,
+                                                  int tid) {
     constexpr bool V = D == kTB || D == kBT;
     const int M = V ? W : H;
     const int HW = H * W;
@@ -398,7 +408,7 @@ __device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const flo
         const int i = D == kTB ? r : D == kBT ? H - 1 - r : D == kLR ? c : W - 1 - c;
         const int j = V ? c : r;
         g0 = g1 = g2 = 0.f;
-        if (i > 0) {
+        if (!chunk_start(scan_ascending(D), V ? H : W, chunk, i)) {
             const int q = r * Wp + c;
             const float w0 = w0b[q], w2 = w2b[q], w1 = 1.f - w0 - w2;
             const bool hasl = j > 0, hasr = j < M - 1;
@@ -445,16 +455,16 @@ __device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const flo
 template <typename T, unsigned D, int LPT>
 __device__ __forceinline__ void plane_bwd_direction(const T* a3, T* da3, const float* z, const float* g, float* w0b,
                                                     float* w2b, float* hb, float* db, float* acc, float* dz, int H,
-                                                    int W, int Wp, int tid) {
+                                                    int W, int Wp, int chunk, int tid) {
     plane_weights<T, D, kPlaneBwdThreads>(a3, w0b, w2b, H, W, Wp, tid);
     __syncthreads();
     if (tid < 32) {
-        plane_recompute<D, LPT>(z, w0b, w2b, hb, acc, H, W, Wp, tid);
+        plane_recompute<D, LPT>(z, w0b, w2b, hb, acc, H, W, Wp, chunk, tid);
         __syncwarp();
-        plane_reverse<D, LPT>(g, w0b, w2b, db, dz, H, W, Wp, tid);
+        plane_reverse<D, LPT>(g, w0b, w2b, db, dz, H, W, Wp, chunk, tid);
     }
     __syncthreads();
-    plane_logit_grads<T, D, kPlaneBwdThreads>(a3, da3, w0b, w2b, hb, db, H, W, Wp, tid);
+    plane_logit_grads<T, D, kPlaneBwdThreads>(a3, da3, w0b, w2b, hb, db, H, W, Wp, chunk, tid);
     __syncthreads();
 }
 
@@ -488,10 +498,10 @@ __global__ void __launch_bounds__(kPlaneBwdThreads) k_plane_bwd(PlaneBwdArgs p) 
         __syncthreads();
         int slot = 0;
         auto aoff = [&](int s) { return (((long long)s * p.N + n) * p.C + c) * 3 * HW; };
-        if (p.mask & kTB) { const long long o = aoff(slot++); plane_bwd_direction<T, kTB, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
-        if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
-        if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
-        if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, tid); }
+        if (p.mask & kTB) { const long long o = aoff(slot++); plane_bwd_direction<T, kTB, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
+        if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
+        if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
+        if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
         for (int e = tid; e < HW; e += kPlaneBwdThreads) {
             const int q = (e / W) * Wp + e % W;
             Io<T>::st((T*)p.dx + po + e, Io<T>::ld(lam + e) * dz[q]);
@@ -548,7 +558,7 @@ cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t 
 template <typename T>
 cudaError_t plane_forward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
                             cudaStream_t st) {
-    PlaneArgs args{x, lam, u, a, y, P.N, P.C, P.H, P.W, P.Cw, plane_wp(P), P.mask};
+    PlaneArgs args{x, lam, u, a, y, P.N, P.C, P.H, P.W, P.Cw, plane_wp(P), P.mask, P.chunk};
     switch (plane_lanes(P)) {
     case 1: return plane_fwd_launch<T, 1>(P, args, st);
     case 2: return plane_fwd_launch<T, 2>(P, args, st);
@@ -575,7 +585,7 @@ cudaError_t plane_forward(const Problem& P, const void* x, const void* a, const 
 
 cudaError_t plane_backward(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
                            const void* dy, void* dx, void* da, void* dlam, void* du, void*, cudaStream_t st) {
-    PlaneBwdArgs args{x, lam, u, a, dy, dx, da, dlam, du, P.N, P.C, P.H, P.W, plane_wp(P), P.mask};
+    PlaneBwdArgs args{x, lam, u, a, dy, dx, da, dlam, du, P.N, P.C, P.H, P.W, plane_wp(P), P.mask, P.chunk};
     const int lpt = plane_lanes(P);
     if (P.dtype == GSPN_F32)
         return lpt == 1 ? plane_bwd_launch<float, 1>(P, args, st)

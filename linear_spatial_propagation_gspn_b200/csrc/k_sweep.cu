@@ -62,6 +62,7 @@ struct SweepArgs {
     void* acct;       // lane-major partial sum
     unsigned* status; // device status word (hand-off timeouts)
     int N, C, H, W, Cw;
+    int chunk;        // lines per local chunk along the scan (0: global)
 };
 
 struct WeightArgs {
@@ -572,6 +573,10 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
     out_setup();
     int kblk = 0;        // staging blocks completed by this CTA
     bool dead = false;   // a hand-off wait timed out: stop waiting
+    // local propagation: steps left in the current chunk (the plane end also ends a chunk)
+    const int cfirst = first_chunk_len(DIR == kTB, H, p.chunk);
+    const int clen = p.chunk > 0 ? p.chunk : H;
+    int crem = cfirst;
     float h[LPT];
 #pragma unroll
     for (int e = 0; e < LPT; ++e) h[e] = 0.f;
@@ -621,8 +626,9 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
                 ++kblk;
             }
         }
-        // the last row of a plane hands zeros to the next plane's first step
-        const bool last = c_rows == 1;
+        // the last row of a chunk or of the plane hands zeros to the next step (a short last
+        // chunk ends with the plane)
+        const bool last = crem == 1 || c_rows == 1;
         if (lane == 0) lo_cur[warp] = last ? 0.f : hn[0];
         if (lane == 31) lo_cur[34 + warp + 1] = last ? 0.f : hn[LPT - 1];
         fetch((u + 1) % NS);
@@ -632,9 +638,15 @@ __global__ void __launch_bounds__(LPT == 8 ? 512 : 1024, 1) k_vsweep(SweepArgs p
             __syncthreads();
 #pragma unroll
         for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+        if (--crem == 0) {
+            crem = clen;
+#pragma unroll
+            for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+        }
         c_off += dstep;
         c_r += rstep;
         if (--c_rows == 0) {
+            crem = cfirst;
 #pragma unroll
             for (int e = 0; e < LPT; ++e) h[e] = 0.f;
             c_rows = H;
@@ -789,13 +801,17 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     };
     int kblk = 0;
     bool dead = false;
+    // local propagation: steps left in the current chunk (the plane end also ends a chunk)
+    const int cfirst = first_chunk_len(DIR == kTB, H, p.chunk);
+    const int clen = p.chunk > 0 ? p.chunk : H;
+    int crem = cfirst;
     float h[LPT];
 #pragma unroll
     for (int e = 0; e < LPT; ++e) h[e] = 0.f;
 
     // one step: i = step within the plane (its low bits give the staging row), u = position in
-    // the unrolled group, last = last row of the plane, live = the refill has a row to fetch
-    auto step = [&](int i, int u, bool last, bool live) {
+    // the unrolled group, live = the refill has a row to fetch
+    auto step = [&](int i, int u, bool live) {
         const float* lo_prev = halo + ((u + 1) & 1) * 68;
         float* lo_cur = halo + (u & 1) * 68;
         const float hx = lo_prev[hread];
@@ -834,6 +850,9 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
                 ++kblk;
             }
         }
+        // the last row of a chunk or of the plane hands zeros to the next step (a short last
+        // chunk ends with the plane)
+        const bool last = crem == 1 || i == H - 1;
         lo_cur[hwrite] = last ? 0.f : (lastl ? hn[LPT - 1] : hn[0]);
         fetch((u + 1) % NS, live);
         if constexpr (NSTG > 0)
@@ -842,6 +861,11 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
             __syncthreads();
 #pragma unroll
         for (int e = 0; e < LPT; ++e) h[e] = hn[e];
+        if (--crem == 0) {
+            crem = clen;
+#pragma unroll
+            for (int e = 0; e < LPT; ++e) h[e] = 0.f;
+        }
         c_off += DSTEP;
     };
 
@@ -856,20 +880,21 @@ __global__ void __launch_bounds__(2 * WL / LPT, 1) k_vsweep_w(SweepArgs p) {
     fetch(0, true);
     for (int pl = 0; pl < my_planes; ++pl, plane += (int)gridDim.x) {
         out_setup(plane);
+        crem = cfirst;
         const bool more = pl + 1 < my_planes;
         int i = 0;
         for (; i < H - 2 * NS; i += NS) {
 #pragma unroll
-            for (int u = 0; u < NS; ++u) step(i + u, u, false, true);
+            for (int u = 0; u < NS; ++u) step(i + u, u, true);
         }
 #pragma unroll
         for (int u = 0; u < NS; ++u) {
             if (u == NS - 1 && more) iss_setup(plane + (int)gridDim.x);
-            step(i + u, u, false, u < NS - 1 || more);
+            step(i + u, u, u < NS - 1 || more);
         }
         i += NS;
 #pragma unroll
-        for (int u = 0; u < NS; ++u) step(i + u, u, u == NS - 1, more);
+        for (int u = 0; u < NS; ++u) step(i + u, u, more);
 #pragma unroll
         for (int e = 0; e < LPT; ++e) h[e] = 0.f;
     }
@@ -1039,7 +1064,7 @@ __global__ void __launch_bounds__(G == 4 ? 256 : (G == 2 ? 512 : 1024), 1) k_hsw
                     float zz = SG::get(rs0[gg], sl);
                     if (Md::XL) zz *= SG::get(rs1[gg], sl);
                     v = zz;
-                    if (i > 0) {
+                    if (!chunk_start(DIR == kLR, W, p.chunk, i)) {
                         const float w0 = wt_get<WT, WC>(rw0[gg], sl);
                         const float w2 = wt_get<WT, WC>(rw2[gg], sl);
                         v = fmaf(w0, hl, fmaf(1.f - w0 - w2, h[gg], fmaf(w2, hr, v)));
@@ -1451,7 +1476,7 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
         SweepArgs args{x, lam, u, table + v * slot_elems, z, acc, y, zt, acct, (unsigned*)ws,
-                       P.N, P.C, P.H, P.W, P.Cw};
+                       P.N, P.C, P.H, P.W, P.Cw, P.chunk};
         const int role = visit_role(P, d, v, tp);
         const bool asc = d == kTB || d == kLR;
         if (is_vertical(d)) {

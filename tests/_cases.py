@@ -37,25 +37,27 @@ def assert_close(got, ref, tol, what):
     return err
 
 
-def run_forward(wl, algo=g.ALGO_AUTO, inputs=None):
+def run_forward(wl, algo=g.ALGO_AUTO, inputs=None, chunk=0):
     t = inputs or gspn_inputs.make_inputs(wl, device="cuda")
-    y = g.forward(t["x"], t["a"], t["lam"], t["u"], wl.wmode, wl.mask, algo=algo)
+    y = g.forward(t["x"], t["a"], t["lam"], t["u"], wl.wmode, wl.mask, algo=algo, chunk=chunk)
     torch.cuda.synchronize()
     return t, y
 
 
-def check_forward(wl, algo=g.ALGO_AUTO):
-    t, y = run_forward(wl, algo)
-    ref = oracle.forward(f64(t["x"]), f64(t["a"]), f64(t["lam"]), f64(t["u"]), wl.wmode, wl.mask)
-    return assert_close(f64(y), ref, fwd_tol(wl.dtype, ref), f"forward {wl.name} algo={algo}")
+def check_forward(wl, algo=g.ALGO_AUTO, chunk=0):
+    t, y = run_forward(wl, algo, chunk=chunk)
+    ref = oracle.forward(f64(t["x"]), f64(t["a"]), f64(t["lam"]), f64(t["u"]), wl.wmode, wl.mask, chunk=chunk)
+    return assert_close(f64(y), ref, fwd_tol(wl.dtype, ref), f"forward {wl.name} algo={algo} chunk={chunk}")
 
 
-def check_backward(wl, algo=g.ALGO_AUTO):
+def check_backward(wl, algo=g.ALGO_AUTO, chunk=0):
     t = gspn_inputs.make_inputs(wl, device="cuda", with_dy=True)
-    got = g.backward(t["x"], t["a"], t["lam"], t["u"], t["dy"], wl.wmode, wl.mask, algo=algo)
+    got = g.backward(t["x"], t["a"], t["lam"], t["u"], t["dy"], wl.wmode, wl.mask, algo=algo, chunk=chunk)
     torch.cuda.synchronize()
-    ref = oracle.backward(f64(t["x"]), f64(t["a"]), f64(t["lam"]), f64(t["u"]), f64(t["dy"]), wl.wmode, wl.mask)
+    ref = oracle.backward(f64(t["x"]), f64(t["a"]), f64(t["lam"]), f64(t["u"]), f64(t["dy"]), wl.wmode, wl.mask,
+                          chunk=chunk)
     errs = []
     for name, gg, rr in zip(("dx", "da", "dlam", "du"), got, ref):
-        errs.append(assert_close(f64(gg), rr, grad_tol(wl.dtype, rr), f"backward {name} {wl.name} algo={algo}"))
+        errs.append(assert_close(f64(gg), rr, grad_tol(wl.dtype, rr),
+                                 f"backward {name} {wl.name} algo={algo} chunk={chunk}"))
     return errs
