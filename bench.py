@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="also time the backward (gradients of x, logits, lambda, u); on by default for 'train'")
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="local propagation: lines per chunk along each scan axis (0 = global, the metric's)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch N (small cases for profiler captures; not a bench line)")
     return ap.parse_args()
@@ -63,7 +65,7 @@ def dtype_name(wl):
     return "f32" if wl.dtype == "f32" else "bf16"
 
 
-def config_of(wl, world):
+def config_of(wl, world, chunk=0):
     return {
         "workload": wl.name,
         "N": wl.N, "C": wl.C, "H": wl.H, "W": wl.W,
@@ -74,11 +76,12 @@ def config_of(wl, world):
         "global_batch": wl.N * world,
         "parallelism": f"dp{world}" if world > 1 else "single",
         "l2": "inputs larger than L2 (no flush)",
+        "chunk": chunk,
     }
 
 
 # --------------------------------------------------------------------------- CPU oracle sample
-def oracle_plane_seconds_only(wl, planes):
+def oracle_plane_seconds_only(wl, planes, chunk=0):
     """Oracle time excluding input generation."""
     import numpy as np
     import oracle
@@ -90,7 +93,7 @@ def oracle_plane_seconds_only(wl, planes):
     u = rng.standard_normal((1, 1, H, W))
     t0 = time.perf_counter()
     for _ in range(planes):
-        oracle.forward(x, a, lam, u, wl.wmode, wl.mask)
+        oracle.forward(x, a, lam, u, wl.wmode, wl.mask, chunk=chunk)
     return time.perf_counter() - t0
 
 
@@ -106,7 +109,7 @@ def run_reference(args):
     planes_per_step = 2
     times = []
     for s in range(args.warmup + args.steps):
-        dt = oracle_plane_seconds_only(wl, planes_per_step)
+        dt = oracle_plane_seconds_only(wl, planes_per_step, args.chunk)
         if s >= args.warmup:
             times.append(dt)
     tot = sum(times)
@@ -119,7 +122,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": config_of(wl, world),
+        "config": config_of(wl, world, args.chunk),
         "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": f"{planes_per_step} of {wl.N * wl.C} planes per step, float64 C oracle, "
                                    "one thread; ms_per_step extrapolated to the full batch"},
@@ -234,14 +237,14 @@ def run_libgspn(args):
     dev = torch.device("cuda", local_rank)
     t = gspn_inputs.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
     x, a, lam, u = t["x"], t["a"], t["lam"], t["u"]
-    desc = g.desc_for(x, wl.wmode, wl.mask)
+    desc = g.desc_for(x, wl.wmode, wl.mask, chunk=args.chunk)
     algo = g.selected_algo(desc)
     ws = g.alloc_workspace(desc, False, dev)
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
 
     def step():
-        g.forward(x, a, lam, u, wl.wmode, wl.mask, y=y, ws=ws)
+        g.forward(x, a, lam, u, wl.wmode, wl.mask, y=y, ws=ws, chunk=args.chunk)
 
     for _ in range(args.warmup):
         step()
@@ -314,12 +317,12 @@ def run_libgspn(args):
     if args.backward or wl.name == "train":
         dy = torch.randn(x.shape, generator=torch.Generator(device=dev).manual_seed(wl.seed + 7), device=dev,
                          dtype=torch.float32).to(x.dtype)
-        bdesc = g.desc_for(x, wl.wmode, wl.mask)
+        bdesc = g.desc_for(x, wl.wmode, wl.mask, chunk=args.chunk)
         bws = g.alloc_workspace(bdesc, True, dev)
         outs = (torch.empty_like(x), torch.empty_like(a), torch.empty_like(x), torch.empty_like(x))
 
         def bstep():
-            g.backward(x, a, lam, u, dy, wl.wmode, wl.mask, out=outs, ws=bws)
+            g.backward(x, a, lam, u, dy, wl.wmode, wl.mask, out=outs, ws=bws, chunk=args.chunk)
 
         for _ in range(max(3, args.warmup // 2)):
             bstep()
@@ -396,7 +399,7 @@ def run_libgspn(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs = oracle_plane_seconds_only(wl, args.cpu_planes)
+        secs = oracle_plane_seconds_only(wl, args.cpu_planes, args.chunk)
         cpu = {"value": round(plane_bytes(wl) * args.cpu_planes / secs / 1e9, 6), "unit": "GB/s", "cores": 1,
                "kind": "oracle",
                "sample": f"{args.cpu_planes} of {wl.N * wl.C} (n,c) planes, float64 C oracle, one thread, "
@@ -410,7 +413,7 @@ def run_libgspn(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": dtype_name(wl), "data": "synthetic (seeded torch.randn/rand on device)",
-            "config": config_of(wl, world),
+            "config": config_of(wl, world, args.chunk),
             "algo": g.ALGO_NAMES.get(algo, str(algo)),
             "roofline": roofline,
             "copy_ceiling_gbs": round(copy_gbs, 1),

@@ -66,7 +66,7 @@ __device__ __forceinline__ int plane_pix(int H, int W, int Wp, int i, int j) {
 // pipelined: the shared-memory operands of step i + 1 (z, w0, w2 and the running sum) are
 // loaded while step i's new line is formed, so a step waits only for the shuffles and FMAs of
 // the recurrence. Lanes past the line (j >= M) read index 0 and contribute nothing.
-template <unsigned D, int LPT>
+template <unsigned D, int LPT, bool LOCAL>
 __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, const float* w2b, float* acc, int H,
                                            int W, int Wp, int chunk, int lane) {
     constexpr bool V = D == kTB || D == kBT;
@@ -74,6 +74,8 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
     float h[LPT], cz[LPT], cw0[LPT], cw2[LPT], ca[LPT];
     int cq[LPT];
     bool on[LPT];
+    int crem = first_chunk_len(scan_ascending(D), L, chunk);   // steps left in this chunk
+    const int clen = chunk > 0 ? chunk : L;
 #pragma unroll
     for (int e = 0; e < LPT; ++e) {
         h[e] = 0.f;
@@ -113,8 +115,12 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
         }
         // the running sum of step i + 1 is read after this step's writes (different pixels
         // except at the same lane, which this thread owns); a chunk's first step starts from
-        // h = 0 (local propagation)
-        const bool restart = more && chunk_start(scan_ascending(D), L, chunk, i + 1);
+        // h = 0 (local propagation; counted down, no division per step)
+        bool restart = false;
+        if constexpr (LOCAL) {
+            restart = --crem == 0;
+            if (restart) crem = clen;
+        }
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
             na[e] = acc[nq[e]];
@@ -171,16 +177,16 @@ __device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2
     }
 }
 
-template <typename T, unsigned D, int LPT>
+template <typename T, unsigned D, int LPT, bool LOCAL>
 __device__ __forceinline__ void plane_direction(const T* a3, const float* z, float* w0b, float* w2b, float* acc, int H,
                                                 int W, int Wp, int chunk, int tid) {
     plane_weights<T, D>(a3, w0b, w2b, H, W, Wp, tid);
     __syncthreads();
-    if (tid < 32) plane_scan<D, LPT>(z, w0b, w2b, acc, H, W, Wp, chunk, tid);
+    if (tid < 32) plane_scan<D, LPT, LOCAL>(z, w0b, w2b, acc, H, W, Wp, chunk, tid);
     __syncthreads();
 }
 
-template <typename T, int LPT>
+template <typename T, int LPT, bool LOCAL>
 __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
     extern __shared__ float sm[];
     const int H = p.H, W = p.W, Wp = p.Wp;
@@ -224,10 +230,10 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
         auto a_of = [&](int s) {
             return (const T*)p.a + (((long long)s * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
         };
-        if (p.mask & kTB) plane_direction<T, kTB, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
-        if (p.mask & kBT) plane_direction<T, kBT, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
-        if (p.mask & kLR) plane_direction<T, kLR, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
-        if (p.mask & kRL) plane_direction<T, kRL, LPT>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
+        if (p.mask & kTB) plane_direction<T, kTB, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
+        if (p.mask & kBT) plane_direction<T, kBT, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
+        if (p.mask & kLR) plane_direction<T, kLR, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
+        if (p.mask & kRL) plane_direction<T, kRL, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
         // y = u * sum
         if (vec) {
             for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
@@ -266,7 +272,7 @@ struct PlaneBwdArgs {
 
 // Forward recompute of direction D by one warp: hb = h^D (plane layout), acc += h^D. Software
 // pipelined like plane_scan.
-template <unsigned D, int LPT>
+template <unsigned D, int LPT, bool LOCAL>
 __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b, const float* w2b, float* hb,
                                                 float* acc, int H, int W, int Wp, int chunk, int lane) {
     constexpr bool V = D == kTB || D == kBT;
@@ -274,6 +280,8 @@ __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b
     float h[LPT], cz[LPT], cw0[LPT], cw2[LPT];
     int cq[LPT];
     bool on[LPT];
+    int crem = first_chunk_len(scan_ascending(D), L, chunk);   // steps left in this chunk
+    const int clen = chunk > 0 ? chunk : L;
 #pragma unroll
     for (int e = 0; e < LPT; ++e) {
         h[e] = 0.f;
@@ -310,7 +318,11 @@ __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b
                 acc[cq[e]] += v;
             }
         }
-        const bool restart = more && chunk_start(scan_ascending(D), L, chunk, i + 1);
+        bool restart = false;
+        if constexpr (LOCAL) {
+            restart = --crem == 0;
+            if (restart) crem = clen;
+        }
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
             h[e] = restart ? 0.f : hn[e];
@@ -322,21 +334,22 @@ __device__ __forceinline__ void plane_recompute(const float* z, const float* w0b
     }
 }
 
-// Whether step i's weights act on h_{i-1} (false at step 0 and at every chunk start).
-__device__ __forceinline__ bool on_any_weights(bool asc, int L, int chunk, int i) { return !chunk_start(asc, L, chunk, i); }
-
 // Reverse scan of direction D by one warp, delta only (no global memory):
 //   delta_i[j] = g_i[j] + w_{i+1}[j-1][2] delta_{i+1}[j-1] + w_{i+1}[j][1] delta_{i+1}[j]
 //                + w_{i+1}[j+1][0] delta_{i+1}[j+1]
 // into db (plane layout), and dz += delta. The operands of step i - 1 are loaded while step i
 // is formed.
-template <unsigned D, int LPT>
+template <unsigned D, int LPT, bool LOCAL>
 __device__ __forceinline__ void plane_reverse(const float* g, const float* w0b, const float* w2b, float* db, float* dz,
                                              int H, int W, int Wp, int chunk, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
     float del[LPT], pw0[LPT], pw1[LPT], pw2[LPT];   // delta and weights of step i + 1
     float cg[LPT], cw0[LPT], cw2[LPT];              // g and weights of step i
+    // steps from the start of the chunk holding step i (0: step i starts a chunk), counted down
+    const int cfirst = first_chunk_len(scan_ascending(D), L, chunk);
+    const int clen = chunk > 0 ? chunk : L;
+    int kin = L - 1 < cfirst ? L - 1 : (L - 1 - cfirst) % clen;
     int cq[LPT];
     bool on[LPT];
 #pragma unroll
@@ -378,7 +391,11 @@ __device__ __forceinline__ void plane_reverse(const float* g, const float* w0b, 
         }
         // step i's weights become the "next step" weights of step i - 1; a step that starts a
         // chunk (step 0 included) does not see h_{i-1}, so nothing flows back through it
-        const bool live = on_any_weights(scan_ascending(D), L, chunk, i);
+        bool live = i != 0;
+        if constexpr (LOCAL) {
+            live = kin != 0;
+            kin = kin != 0 ? kin - 1 : (i - 1 < cfirst ? i - 1 : clen - 1);
+        }
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
             del[e] = dn[e];
@@ -452,23 +469,23 @@ __device__ __forceinline__ void plane_logit_grads(const T* a3, T* da3, const flo
     }
 }
 
-template <typename T, unsigned D, int LPT>
+template <typename T, unsigned D, int LPT, bool LOCAL>
 __device__ __forceinline__ void plane_bwd_direction(const T* a3, T* da3, const float* z, const float* g, float* w0b,
                                                     float* w2b, float* hb, float* db, float* acc, float* dz, int H,
                                                     int W, int Wp, int chunk, int tid) {
     plane_weights<T, D, kPlaneBwdThreads>(a3, w0b, w2b, H, W, Wp, tid);
     __syncthreads();
     if (tid < 32) {
-        plane_recompute<D, LPT>(z, w0b, w2b, hb, acc, H, W, Wp, chunk, tid);
+        plane_recompute<D, LPT, LOCAL>(z, w0b, w2b, hb, acc, H, W, Wp, chunk, tid);
         __syncwarp();
-        plane_reverse<D, LPT>(g, w0b, w2b, db, dz, H, W, Wp, chunk, tid);
+        plane_reverse<D, LPT, LOCAL>(g, w0b, w2b, db, dz, H, W, Wp, chunk, tid);
     }
     __syncthreads();
     plane_logit_grads<T, D, kPlaneBwdThreads>(a3, da3, w0b, w2b, hb, db, H, W, Wp, chunk, tid);
     __syncthreads();
 }
 
-template <typename T, int LPT>
+template <typename T, int LPT, bool LOCAL>
 __global__ void __launch_bounds__(kPlaneBwdThreads) k_plane_bwd(PlaneBwdArgs p) {
     extern __shared__ float sm[];
     const int H = p.H, W = p.W, Wp = p.Wp;
@@ -498,10 +515,10 @@ __global__ void __launch_bounds__(kPlaneBwdThreads) k_plane_bwd(PlaneBwdArgs p) 
         __syncthreads();
         int slot = 0;
         auto aoff = [&](int s) { return (((long long)s * p.N + n) * p.C + c) * 3 * HW; };
-        if (p.mask & kTB) { const long long o = aoff(slot++); plane_bwd_direction<T, kTB, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
-        if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
-        if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
-        if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
+        if (p.mask & kTB) { const long long o = aoff(slot++); plane_bwd_direction<T, kTB, LPT, LOCAL>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
+        if (p.mask & kBT) { const long long o = aoff(slot++); plane_bwd_direction<T, kBT, LPT, LOCAL>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
+        if (p.mask & kLR) { const long long o = aoff(slot++); plane_bwd_direction<T, kLR, LPT, LOCAL>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
+        if (p.mask & kRL) { const long long o = aoff(slot++); plane_bwd_direction<T, kRL, LPT, LOCAL>((const T*)p.a + o, (T*)p.da + o, z, g, w0b, w2b, hb, db, acc, dz, H, W, Wp, p.chunk, tid); }
         for (int e = tid; e < HW; e += kPlaneBwdThreads) {
             const int q = (e / W) * Wp + e % W;
             Io<T>::st((T*)p.dx + po + e, Io<T>::ld(lam + e) * dz[q]);
@@ -521,38 +538,48 @@ int plane_lanes(const Problem& P) {
 
 size_t plane_bwd_smem(const Problem& P) { return 8 * (size_t)P.H * plane_wp(P) * sizeof(float); }
 
-template <typename T, int LPT>
-cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
+template <typename T, int LPT, bool LOCAL>
+cudaError_t plane_bwd_launch3(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
     const size_t smem = plane_bwd_smem(P);
-    cudaError_t e = cudaFuncSetAttribute(k_plane_bwd<T, LPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_plane_bwd<T, LPT, LOCAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaFuncSetAttribute(k_plane_bwd<T, LPT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(k_plane_bwd<T, LPT, LOCAL>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int per_sm = 1;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_bwd<T, LPT>, kPlaneBwdThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_bwd<T, LPT, LOCAL>, kPlaneBwdThreads, smem);
     if (e != cudaSuccess) return e;
     const long long want = (long long)std::max(1, per_sm) * device_sm_count();
     const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
     launch_begin(st);
-    k_plane_bwd<T, LPT><<<grid, kPlaneBwdThreads, smem, st>>>(a);
+    k_plane_bwd<T, LPT, LOCAL><<<grid, kPlaneBwdThreads, smem, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
 }
 
-template <typename T, int LPT>
-cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
+template <typename T, int LPT, bool LOCAL>
+cudaError_t plane_fwd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
     const size_t smem = plane_smem(P);
-    cudaError_t e = cudaFuncSetAttribute(k_plane_fwd<T, LPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_plane_fwd<T, LPT, LOCAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaFuncSetAttribute(k_plane_fwd<T, LPT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(k_plane_fwd<T, LPT, LOCAL>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int per_sm = 1;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_fwd<T, LPT>, kPlaneThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_fwd<T, LPT, LOCAL>, kPlaneThreads, smem);
     if (e != cudaSuccess) return e;
     const long long want = (long long)std::max(1, per_sm) * device_sm_count();
     const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
     launch_begin(st);
-    k_plane_fwd<T, LPT><<<grid, kPlaneThreads, smem, st>>>(a);
+    k_plane_fwd<T, LPT, LOCAL><<<grid, kPlaneThreads, smem, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
+}
+
+// Local propagation has its own instantiations, so the global scans carry no chunk counters.
+template <typename T, int LPT>
+cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
+    return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true>(P, a, st) : plane_fwd_launch3<T, LPT, false>(P, a, st);
+}
+template <typename T, int LPT>
+cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
+    return P.chunk > 0 ? plane_bwd_launch3<T, LPT, true>(P, a, st) : plane_bwd_launch3<T, LPT, false>(P, a, st);
 }
 
 template <typename T>
