@@ -117,6 +117,18 @@ def backward(x, a, lam, u, dy, wmode: int = 0, mask: int = 15, chunk: int = 0):
     return dx, da, dlam, du
 
 
+def proxy_forward(x, p_in, a, lam, u, p_out, wmode: int = 1, mask: int = 15, chunk: int = 0) -> np.ndarray:
+    """Compressive channel proxy ("GSPN-2: Efficient Parallel Sequence Modeling" paper notes,
+    section "Optimisation 2: compact channel propagation"): per pixel xp = P_in x (C_proxy x C
+    matrix over channels), the propagation in proxy space, then y = P_out yp (C x C_proxy), all in
+    float64. The channel products are numpy's (a library primitive as a step); lam, u and the
+    logits are in proxy space."""
+    x, p_in, p_out = _f64(x), _f64(p_in), _f64(p_out)
+    xp = np.einsum("pc,nchw->nphw", p_in, x)
+    yp = forward(xp, a, lam, u, wmode, mask, chunk)
+    return np.einsum("cp,nphw->nchw", p_out, yp)
+
+
 def plane_inputs(x, a, lam, u, n: int, c: int, wmode: int):
     """Slices the inputs of one (n, c) plane as an N=1, C=1 problem (both weight modes).
 

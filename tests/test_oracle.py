@@ -422,3 +422,53 @@ def test_chunk_start_logits_have_zero_gradient():
     for r in (0, 3, 6):
         assert np.all(da[0, 0, 0, :, r, :] == 0.0)
     assert np.abs(da[0, 0, 0, :, 1, :]).max() > 0.0
+
+
+# ----------------------------------------------------------------------------- channel proxy
+def _proxy_case(rng, N, C, Cp, H, W, mask=15, wmode=1):
+    x = rng.standard_normal((N, C, H, W))
+    _, a, lam, u = rand_case(rng, N, Cp, H, W, mask, wmode)
+    p_in = rng.standard_normal((Cp, C)) / np.sqrt(C)
+    p_out = rng.standard_normal((C, Cp)) / np.sqrt(Cp)
+    return x, p_in, a, lam, u, p_out
+
+
+def test_proxy_with_identity_projections_is_the_plain_propagation():
+    rng = np.random.default_rng(200)
+    x, _, a, lam, u, _ = _proxy_case(rng, 2, 3, 3, 5, 6)
+    eye = np.eye(3)
+    y = oracle.proxy_forward(x, eye, a, lam, u, eye, 1, 15)
+    assert np.abs(y - oracle.forward(x, a, lam, u, 1, 15)).max() <= 1e-12
+
+
+def test_proxy_matches_pixel_loops():
+    """The channel products written as explicit loops over pixels and channels (pins the
+    operand orientation of both projections)."""
+    rng = np.random.default_rng(201)
+    N, C, Cp, H, W = 2, 5, 3, 4, 3
+    x, p_in, a, lam, u, p_out = _proxy_case(rng, N, C, Cp, H, W)
+    xp = np.zeros((N, Cp, H, W))
+    for n in range(N):
+        for q in range(Cp):
+            for c in range(C):
+                xp[n, q] += p_in[q, c] * x[n, c]
+    yp = oracle.forward(xp, a, lam, u, 1, 15)
+    y = np.zeros((N, C, H, W))
+    for n in range(N):
+        for c in range(C):
+            for q in range(Cp):
+                y[n, c] += p_out[c, q] * yp[n, q]
+    assert np.abs(oracle.proxy_forward(x, p_in, a, lam, u, p_out, 1, 15) - y).max() <= 1e-12
+
+
+def test_proxy_selecting_one_channel():
+    """C_proxy = 1 with P_in = e_k^T and P_out = e_k: channel k is propagated alone, the others
+    come out zero."""
+    rng = np.random.default_rng(202)
+    N, C, H, W, k = 1, 4, 5, 5, 2
+    x, _, a, lam, u, _ = _proxy_case(rng, N, C, 1, H, W)
+    p_in = np.zeros((1, C)); p_in[0, k] = 1.0
+    p_out = np.zeros((C, 1)); p_out[k, 0] = 1.0
+    y = oracle.proxy_forward(x, p_in, a, lam, u, p_out, 1, 15)
+    assert np.abs(y[:, k:k + 1] - oracle.forward(x[:, k:k + 1], a, lam, u, 1, 15)).max() <= 1e-12
+    assert np.all(np.delete(y, k, axis=1) == 0.0)
