@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="also time the backward (gradients of x, logits, lambda, u); on by default for 'train'")
+    ap.add_argument("--proxy", type=int, default=0,
+                    help="compressive channel proxy: project C channels to this many, propagate, project back")
     ap.add_argument("--chunk", type=int, default=0,
                     help="local propagation: lines per chunk along each scan axis (0 = global, the metric's)")
     ap.add_argument("--batch", type=int, default=0,
@@ -428,10 +430,86 @@ def run_libgspn(args):
         dist.destroy_process_group()
 
 
+def run_proxy(args):
+    """Compressive channel proxy on the named workload: x has the workload's C channels, the
+    propagation runs on args.proxy channels (logits, lambda and u in proxy space), the two
+    projections are GEMMs on the tensor cores. Reports the whole proxied forward and, timed
+    separately, its propagation alone."""
+    import torch
+    import linear_spatial_propagation_gspn_b200 as g
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    wl = gspn_inputs.WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.with_(N=args.batch)
+    Cp = args.proxy
+    pw = wl.with_(C=Cp)
+    t = gspn_inputs.make_inputs(wl, device=dev)
+    tp = gspn_inputs.make_inputs(pw, device=dev, seed=wl.seed + 17)
+    x = t["x"]
+    a, lam, u = tp["a"], tp["lam"], tp["u"]
+    gen = torch.Generator(device=dev).manual_seed(wl.seed + 29)
+    p_in = (torch.randn(Cp, wl.C, generator=gen, device=dev) / wl.C ** 0.5).to(x.dtype)
+    p_out = (torch.randn(wl.C, Cp, generator=gen, device=dev) / Cp ** 0.5).to(x.dtype)
+    y = torch.empty_like(x)
+    desc = g.make_desc(wl.N, Cp, wl.H, wl.W, wl.wmode, wl.mask, g._dtype_code(x.dtype), chunk=args.chunk)
+    ws = torch.empty(int(g.lib().gspn_proxy_workspace_size(desc, wl.C)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        g.proxy_forward(x, p_in, a, lam, u, p_out, wl.wmode, wl.mask, y=y, ws=ws, chunk=args.chunk)
+
+    def timed(fn, k):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / k
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    ms = timed(step, args.steps)
+    clocks = sampler.stop()
+    xp = tp["x"]
+    yp = torch.empty_like(xp)
+    sws = g.alloc_workspace(g.desc_for(xp, wl.wmode, wl.mask, chunk=args.chunk), False, dev)
+    scan_ms = timed(lambda: g.forward(xp, a, lam, u, wl.wmode, wl.mask, y=yp, ws=sws, chunk=args.chunk),
+                    max(5, args.steps // 2))
+    es = wl.elem_bytes
+    hw = wl.H * wl.W
+    comp = (2 * wl.N * wl.C * hw + 2 * wl.N * Cp * hw + 2 * Cp * wl.C + a.numel()) * es
+    flops = 2 * 2 * wl.N * hw * wl.C * Cp
+    peak, peak_kind = measured_peak()
+    line = {
+        "metric": METRIC, "variant": f"compressive channel proxy {wl.C} -> {Cp} channels",
+        "value": round(comp / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": dtype_name(wl), "data": "synthetic (seeded torch.randn/rand on device)",
+        "config": dict(config_of(wl, 1, args.chunk), proxy=Cp),
+        "proxy": {"C": wl.C, "C_proxy": Cp, "scan_ms": round(scan_ms, 4),
+                  "projections_ms": round(ms - scan_ms, 4), "projection_tflop_per_step": round(flops / 1e12, 4),
+                  "projection_tflops": round(flops / ((ms - scan_ms) * 1e-3) / 1e12, 1) if ms > scan_ms else None,
+                  "compulsory_bytes": comp,
+                  "what": "x read and y written at C channels; lambda, u, logits at C_proxy; P_in, P_out"},
+        "roofline": {"bound": "hbm", "achieved": round(comp / (ms * 1e-3) / 1e9, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(comp / (ms * 1e-3) / 1e9 / peak, 4), "traffic": None, "peak_kind": peak_kind},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.proxy:
+        run_proxy(args)
     else:
         run_libgspn(args)
 

@@ -150,8 +150,8 @@ GSPN_API gspn_status gspn_forward_host(const gspn_desc *desc, const void *hx, co
  * Returns GSPN_OK, GSPN_ERR_DEVICE_TIMEOUT (a bounded device wait ran out) or GSPN_ERR_CUDA. */
 GSPN_API gspn_status gspn_device_status(void *ws, void *stream);
 
-/* Test hook for the failure path: launches one CTA that waits, through the same bounded
- * wait the TMA pipelines use, on a flag in `ws` that nothing sets, giving up after
+/* Test hook for the failure path: launches one CTA that waits, through the same kind of bounded
+ * wait the kernels' hand-offs use, on a flag in `ws` that nothing sets, giving up after
  * `limit_ns` nanoseconds and recording GSPN_ERR_DEVICE_TIMEOUT in the status word. */
 GSPN_API gspn_status gspn_debug_wait_timeout(void *ws, size_t ws_bytes, unsigned long long limit_ns,
                                     void *stream);
@@ -159,6 +159,21 @@ GSPN_API gspn_status gspn_debug_wait_timeout(void *ws, size_t ws_bytes, unsigned
 /* Plain device-to-device copy of `bytes` (multiple of 16, 16-byte aligned pointers) with a
  * vectorised grid-stride kernel: the bandwidth ceiling the sweeps are compared with. */
 GSPN_API gspn_status gspn_copy_ceiling(const void *src, void *dst, size_t bytes, void *stream);
+
+/* Compressive channel proxy around the propagation ("GSPN-2: Efficient Parallel Sequence
+ * Modeling" paper notes, "Optimisation 2: compact channel propagation": project the C channels
+ * to a low-dimensional proxy, propagate there, restore with a 1x1 convolution):
+ *     xp = P_in x,   yp = propagation of xp (gspn_forward),   y = P_out yp,
+ * per pixel, with P_in a C_proxy x C and P_out a C x C_proxy matrix (row-major, storage dtype).
+ * `desc` describes the proxy-space propagation: desc->C = C_proxy, and the logits a, lam and u
+ * are in proxy space (shapes as for gspn_forward with C = C_proxy). x and y: N x c_full x H x W.
+ * The projections are strided batched GEMMs on the tensor cores (cuBLAS; bf16 storage: bf16
+ * operands with fp32 accumulation; fp32 storage: exact fp32), xp and yp live in the workspace in
+ * the storage dtype. All pointers are device pointers. */
+GSPN_API size_t gspn_proxy_workspace_size(const gspn_desc *desc, int c_full);
+GSPN_API gspn_status gspn_proxy_forward(const gspn_desc *desc, int c_full, const void *x, const void *p_in,
+                               const void *a, const void *lam, const void *u, const void *p_out,
+                               void *y, void *ws, size_t ws_bytes, void *stream);
 
 /* Size of the fixed device scratch array used by gspn_forward_noalloc (64 MiB). */
 #define GSPN_NOALLOC_SCRATCH_BYTES (64u << 20)

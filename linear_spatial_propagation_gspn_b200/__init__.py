@@ -63,6 +63,8 @@ SIGNATURES = {
     "gspn_debug_wait_timeout": (_I, [_VP, _SZ, _U64, _VP]),
     "gspn_copy_ceiling": (_I, [_VP, _VP, _SZ, _VP]),
     "gspn_forward_noalloc": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "gspn_proxy_workspace_size": (_SZ, [_DP, _I]),
+    "gspn_proxy_forward": (_I, [_DP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "gspn_status_string": (ctypes.c_char_p, [_I]),
     "gspn_version": (_I, []),
 }
@@ -187,6 +189,36 @@ def backward(x, a, lam, u, dy, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL
     if s != GSPN_OK:
         raise GspnError(s, "gspn_backward")
     return dx, da, dlam, du
+
+
+def proxy_forward(x, p_in, a, lam, u, p_out, wmode: int = SHARED, dir_mask: int = DIR_ALL, algo: int = ALGO_AUTO,
+                  y=None, ws=None, stream=None, chunk: int = 0) -> torch.Tensor:
+    """Compressive channel proxy: y = P_out . propagate(P_in . x) per pixel. x: (N, C, H, W);
+    p_in: (Cp, C); p_out: (C, Cp); a, lam, u in proxy space (C = Cp); all one dtype."""
+    _check({"x": x, "p_in": p_in, "a": a, "lam": lam, "u": u, "p_out": p_out}, x)
+    N, C, H, W = x.shape
+    Cp = p_in.shape[0]
+    if tuple(p_in.shape) != (Cp, C) or tuple(p_out.shape) != (C, Cp):
+        raise ValueError(f"projection shapes {tuple(p_in.shape)}, {tuple(p_out.shape)}; expected ({Cp}, {C}), ({C}, {Cp})")
+    if tuple(lam.shape) != (N, Cp, H, W) or tuple(u.shape) != (N, Cp, H, W):
+        raise ValueError("lam and u must be (N, C_proxy, H, W)")
+    if tuple(a.shape) != logits_shape(N, Cp, H, W, wmode, dir_mask):
+        raise ValueError(f"logits shape {tuple(a.shape)}, expected {logits_shape(N, Cp, H, W, wmode, dir_mask)}")
+    desc = make_desc(N, Cp, H, W, wmode, dir_mask, _dtype_code(x.dtype), algo, chunk)
+    if y is None:
+        y = torch.empty_like(x)
+    _check({"y": y}, x)
+    if ws is None:
+        nb = int(lib().gspn_proxy_workspace_size(ctypes.byref(desc), C))
+        if nb == 0:
+            raise GspnError(GSPN_ERR_UNSUPPORTED, "gspn_proxy_workspace_size")
+        ws = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    s = lib().gspn_proxy_forward(ctypes.byref(desc), C, x.data_ptr(), p_in.data_ptr(), a.data_ptr(), lam.data_ptr(),
+                                 u.data_ptr(), p_out.data_ptr(), y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                 _stream_ptr(stream))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_proxy_forward")
+    return y
 
 
 def forward_timed(x, a, lam, u, y, ws, desc: GspnDesc, events, stream=None) -> int:
