@@ -192,9 +192,9 @@ def measured_peak():
     return 6650.0, "fallback"
 
 
-# Sources that build the large-map forward the traffic summary describes (the sweep family,
-# its shared helpers and the entry points); other families do not affect it.
-SWEEP_SOURCES = ("gspn_api.cu", "gspn_common.cuh", "gspn_internal.h", "k_sweep.cu")
+# Sources of the kernels the traffic summary describes (the sweep family and its device
+# helpers); host-side entry points and the other families do not change their traffic.
+SWEEP_SOURCES = ("gspn_common.cuh", "k_sweep.cu")
 
 
 def kernel_source_sha():
