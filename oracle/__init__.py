@@ -56,11 +56,11 @@ def _load():
         lib.gspn_ref_forward.restype = ctypes.c_int
         lib.gspn_ref_backward.argtypes = args + [dp] * 9
         lib.gspn_ref_backward.restype = ctypes.c_int
-        lib.gspn_ref_forward_chunked.argtypes = args + [ctypes.c_int] + [dp] * 5
-        lib.gspn_ref_forward_chunked.restype = ctypes.c_int
-        lib.gspn_ref_backward_chunked.argtypes = args + [ctypes.c_int] + [dp] * 9
-        lib.gspn_ref_backward_chunked.restype = ctypes.c_int
-        if lib.gspn_ref_abi_version() != 2:
+        lib.gspn_ref_forward_ex.argtypes = args + [ctypes.c_int, ctypes.c_int] + [dp] * 5
+        lib.gspn_ref_forward_ex.restype = ctypes.c_int
+        lib.gspn_ref_backward_ex.argtypes = args + [ctypes.c_int, ctypes.c_int] + [dp] * 9
+        lib.gspn_ref_backward_ex.restype = ctypes.c_int
+        if lib.gspn_ref_abi_version() != 3:
             raise RuntimeError("stale oracle build; rebuild with oracle.build(force=True)")
         _lib = lib
     return _lib
@@ -78,40 +78,42 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def _check_shapes(x, a, lam, u, wmode, mask):
+def _check_shapes(x, a, lam, u, wmode, mask, per_dir=0):
     N, C, H, W = x.shape
     Cw = 1 if wmode else C
     want_a = (popcount(mask), N, Cw, 3, H, W)
     if a.shape != want_a:
         raise ValueError(f"logits shape {a.shape}, expected {want_a}")
-    if lam.shape != x.shape or u.shape != x.shape:
-        raise ValueError("lam and u must have the shape of x")
+    want_lu = ((popcount(mask),) if per_dir else ()) + x.shape
+    if lam.shape != want_lu or u.shape != want_lu:
+        raise ValueError(f"lam and u must be {want_lu}")
     return N, C, H, W
 
 
-def forward(x, a, lam, u, wmode: int = 0, mask: int = 15, chunk: int = 0) -> np.ndarray:
+def forward(x, a, lam, u, wmode: int = 0, mask: int = 15, chunk: int = 0, per_dir: int = 0) -> np.ndarray:
     """y = u * sum_{d in mask} h^d, float64. ``wmode`` 0 = per-channel, 1 = shared; ``chunk``
-    > 0: local propagation within image-aligned chunks of that many lines (0 = global)."""
+    > 0: local propagation within image-aligned chunks of that many lines (0 = global);
+    ``per_dir`` = 1: lam and u have a direction axis and y = sum_d u_d * h^d(lam_d x)."""
     x, a, lam, u = _f64(x), _f64(a), _f64(lam), _f64(u)
-    N, C, H, W = _check_shapes(x, a, lam, u, wmode, mask)
+    N, C, H, W = _check_shapes(x, a, lam, u, wmode, mask, per_dir)
     y = np.empty_like(x)
-    rc = _load().gspn_ref_forward_chunked(N, C, H, W, int(wmode), int(mask), int(chunk), _ptr(x), _ptr(a),
-                                          _ptr(lam), _ptr(u), _ptr(y))
+    rc = _load().gspn_ref_forward_ex(N, C, H, W, int(wmode), int(mask), int(chunk), int(per_dir), _ptr(x), _ptr(a),
+                                     _ptr(lam), _ptr(u), _ptr(y))
     if rc:
         raise RuntimeError(f"gspn_ref_forward failed ({rc})")
     return y
 
 
-def backward(x, a, lam, u, dy, wmode: int = 0, mask: int = 15, chunk: int = 0):
+def backward(x, a, lam, u, dy, wmode: int = 0, mask: int = 15, chunk: int = 0, per_dir: int = 0):
     """Returns (dx, da, dlam, du), float64, for the loss sum(dy * y)."""
     x, a, lam, u, dy = _f64(x), _f64(a), _f64(lam), _f64(u), _f64(dy)
-    N, C, H, W = _check_shapes(x, a, lam, u, wmode, mask)
+    N, C, H, W = _check_shapes(x, a, lam, u, wmode, mask, per_dir)
     if dy.shape != x.shape:
         raise ValueError("dy must have the shape of x")
-    dx, dlam, du = np.empty_like(x), np.empty_like(x), np.empty_like(x)
+    dx, dlam, du = np.empty_like(x), np.empty_like(lam), np.empty_like(u)
     da = np.empty_like(a)
-    rc = _load().gspn_ref_backward_chunked(N, C, H, W, int(wmode), int(mask), int(chunk), _ptr(x), _ptr(a),
-                                           _ptr(lam), _ptr(u), _ptr(dy), _ptr(dx), _ptr(da), _ptr(dlam), _ptr(du))
+    rc = _load().gspn_ref_backward_ex(N, C, H, W, int(wmode), int(mask), int(chunk), int(per_dir), _ptr(x), _ptr(a),
+                                      _ptr(lam), _ptr(u), _ptr(dy), _ptr(dx), _ptr(da), _ptr(dlam), _ptr(du))
     if rc:
         raise RuntimeError(f"gspn_ref_backward failed ({rc})")
     return dx, da, dlam, du

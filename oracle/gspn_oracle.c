@@ -49,6 +49,13 @@
  * TB/BT, columns for LR/RL) and propagation does not cross a chunk boundary: the scan
  * restarts from h = 0 at the first line of every chunk in scan order. K = 0 is the global
  * scan. The *_chunked entry points take K; the plain ones are K = 0.
+ *
+ * Per-direction lambda and u (the *_ex entry points with per_dir = 1): the pages' models merge
+ * the four directions with a learnable merge ("Parallel Sequence Modeling via Generalized
+ * Spatial Propagation Network" summary, section "Measured effects"). Reading: lambda and u carry
+ * a direction axis (D x N x C x H x W, slots ordered as the logits), h^d is driven by
+ * lambda_d (.) x, and y = sum_d u_d (.) h^d, i.e. a per-pixel, per-channel learnable weighting
+ * of the directions. per_dir = 0 is the shared lambda / u above.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -145,11 +152,11 @@ static long logit_base(int slot, int n, int cw, int N, int Cw, long HW) {
     return (((long)slot * N + n) * Cw + cw) * 3 * HW;
 }
 
-int gspn_ref_forward_chunked(int N, int C, int H, int W, int wmode, unsigned mask, int chunk,
-                             const double *x, const double *a, const double *lam, const double *u,
-                             double *y) {
-    if (check_args(N, C, H, W, wmode, mask, chunk)) return 1;
+int gspn_ref_forward_ex(int N, int C, int H, int W, int wmode, unsigned mask, int chunk, int per_dir,
+                        const double *x, const double *a, const double *lam, const double *u, double *y) {
+    if (check_args(N, C, H, W, wmode, mask, chunk) || (per_dir != 0 && per_dir != 1)) return 1;
     const long HW = (long)H * W;
+    const long U = (long)N * C * HW; /* elements of one N x C x H x W tensor */
     const int Cw = wmode ? 1 : C;
     const int Lmax = H > W ? H : W;
     double *hbuf = (double *)malloc(sizeof(double) * (size_t)Lmax * (size_t)Lmax);
@@ -163,14 +170,20 @@ int gspn_ref_forward_chunked(int N, int C, int H, int W, int wmode, unsigned mas
             for (unsigned d = DIR_TB; d <= DIR_RL; d <<= 1) {
                 if (!(mask & d)) continue;
                 const double *a3 = a + logit_base(slot, n, wmode ? 0 : c, N, Cw, HW);
-                scan_forward(d, H, W, chunk, x + off, lam + off, a3, hbuf);
+                const double *lam_d = lam + (per_dir ? slot * U : 0) + off;
+                const double *u_d = u + (per_dir ? slot * U : 0) + off;
+                scan_forward(d, H, W, chunk, x + off, lam_d, a3, hbuf);
                 int L, M;
                 geom(d, H, W, &L, &M);
                 for (int i = 0; i < L; ++i)
-                    for (int j = 0; j < M; ++j) acc[pix(d, H, W, i, j)] += hbuf[(long)i * M + j];
+                    for (int j = 0; j < M; ++j) {
+                        const long p = pix(d, H, W, i, j);
+                        /* per-direction u weights h^d here; the shared u is applied once below */
+                        acc[p] += (per_dir ? u_d[p] : 1.0) * hbuf[(long)i * M + j];
+                    }
                 ++slot;
             }
-            for (long p = 0; p < HW; ++p) y[off + p] = u[off + p] * acc[p];
+            for (long p = 0; p < HW; ++p) y[off + p] = per_dir ? acc[p] : u[off + p] * acc[p];
         }
     }
     free(hbuf);
@@ -178,10 +191,16 @@ int gspn_ref_forward_chunked(int N, int C, int H, int W, int wmode, unsigned mas
     return 0;
 }
 
+int gspn_ref_forward_chunked(int N, int C, int H, int W, int wmode, unsigned mask, int chunk,
+                             const double *x, const double *a, const double *lam, const double *u,
+                             double *y) {
+    return gspn_ref_forward_ex(N, C, H, W, wmode, mask, chunk, 0, x, a, lam, u, y);
+}
+
 int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
                      const double *x, const double *a, const double *lam, const double *u,
                      double *y) {
-    return gspn_ref_forward_chunked(N, C, H, W, wmode, mask, 0, x, a, lam, u, y);
+    return gspn_ref_forward_ex(N, C, H, W, wmode, mask, 0, 0, x, a, lam, u, y);
 }
 
 /*
@@ -198,12 +217,15 @@ int gspn_ref_forward(int N, int C, int H, int W, int wmode, unsigned mask,
  *     da_k = 0 for out-of-range k. In the shared mode da is summed over channels.
  *   With chunks, a step that starts a chunk behaves like step 0: its weights multiply
  *   h = 0 (zero logit gradient) and no delta flows back through them.
+ *   Per-direction lambda / u: g^d = dy (.) u_d, du_d = dy (.) h^d, dlam_d = x (.) delta^d,
+ *   dx = sum_d lam_d (.) delta^d.
  */
-int gspn_ref_backward_chunked(int N, int C, int H, int W, int wmode, unsigned mask, int chunk,
-                              const double *x, const double *a, const double *lam, const double *u,
-                              const double *dy, double *dx, double *da, double *dlam, double *du) {
-    if (check_args(N, C, H, W, wmode, mask, chunk)) return 1;
+int gspn_ref_backward_ex(int N, int C, int H, int W, int wmode, unsigned mask, int chunk, int per_dir,
+                         const double *x, const double *a, const double *lam, const double *u,
+                         const double *dy, double *dx, double *da, double *dlam, double *du) {
+    if (check_args(N, C, H, W, wmode, mask, chunk) || (per_dir != 0 && per_dir != 1)) return 1;
     const long HW = (long)H * W;
+    const long U = (long)N * C * HW;
     const int Cw = wmode ? 1 : C;
     const int D = popcount4(mask);
     const int Lmax = H > W ? H : W;
@@ -213,8 +235,9 @@ int gspn_ref_backward_chunked(int N, int C, int H, int W, int wmode, unsigned ma
     double *dcur = (double *)malloc(sizeof(double) * (size_t)Lmax);
     double *dnext = (double *)malloc(sizeof(double) * (size_t)Lmax);
     double *wnext = (double *)malloc(sizeof(double) * 3 * (size_t)Lmax);
-    if (!hbuf || !acc || !dz || !dcur || !dnext || !wnext) {
-        free(hbuf); free(acc); free(dz); free(dcur); free(dnext); free(wnext);
+    double *dd = (double *)malloc(sizeof(double) * (size_t)HW); /* delta^d, image coordinates */
+    if (!hbuf || !acc || !dz || !dcur || !dnext || !wnext || !dd) {
+        free(hbuf); free(acc); free(dz); free(dcur); free(dnext); free(wnext); free(dd);
         return 2;
     }
     memset(da, 0, sizeof(double) * (size_t)D * N * Cw * 3 * HW);
@@ -231,16 +254,23 @@ int gspn_ref_backward_chunked(int N, int C, int H, int W, int wmode, unsigned ma
                 const long ab = logit_base(slot, n, wmode ? 0 : c, N, Cw, HW);
                 const double *a3 = a + ab;
                 double *da3 = da + ab;
+                const long so = per_dir ? slot * U : 0;   /* this direction's lambda / u */
+                const double *lp_d = lam + so + off, *up_d = u + so + off;
                 int L, M;
                 geom(d, H, W, &L, &M);
-                scan_forward(d, H, W, chunk, xp, lp, a3, hbuf);
+                scan_forward(d, H, W, chunk, xp, lp_d, a3, hbuf);
                 for (int i = 0; i < L; ++i)
-                    for (int j = 0; j < M; ++j) acc[pix(d, H, W, i, j)] += hbuf[(long)i * M + j];
+                    for (int j = 0; j < M; ++j) {
+                        const long p = pix(d, H, W, i, j);
+                        if (per_dir) du[so + off + p] = dyp[p] * hbuf[(long)i * M + j];
+                        else acc[p] += hbuf[(long)i * M + j];
+                    }
+                memset(dd, 0, sizeof(double) * (size_t)HW);
                 /* reverse scan */
                 for (int i = L - 1; i >= 0; --i) {
                     for (int j = 0; j < M; ++j) {
                         long p = pix(d, H, W, i, j);
-                        double del = dyp[p] * up[p];
+                        double del = dyp[p] * up_d[p];
                         if (i < L - 1) {
                             /* w_{i+1}^T delta_{i+1}: row j' of w_{i+1} touches lane j through k = j - j' + 1 */
                             for (int jp = j - 1; jp <= j + 1; ++jp) {
@@ -250,7 +280,7 @@ int gspn_ref_backward_chunked(int N, int C, int H, int W, int wmode, unsigned ma
                             }
                         }
                         dcur[j] = del;
-                        dz[p] += del;
+                        dd[p] = del;
                     }
                     /* weights of step i (used by step i-1's transpose product) and da_i */
                     for (int j = 0; j < M; ++j) {
@@ -279,24 +309,42 @@ int gspn_ref_backward_chunked(int N, int C, int H, int W, int wmode, unsigned ma
                     }
                     for (int j = 0; j < M; ++j) dnext[j] = dcur[j];
                 }
+                for (long p = 0; p < HW; ++p) {
+                    if (per_dir) {
+                        dlam[so + off + p] = xp[p] * dd[p];
+                        dz[p] += lp_d[p] * dd[p];   /* dz accumulates dx directly */
+                    } else {
+                        dz[p] += dd[p];
+                    }
+                }
                 ++slot;
             }
             for (long p = 0; p < HW; ++p) {
-                du[off + p] = dyp[p] * acc[p];
-                dx[off + p] = lp[p] * dz[p];
-                dlam[off + p] = xp[p] * dz[p];
+                if (per_dir) {
+                    dx[off + p] = dz[p];
+                } else {
+                    du[off + p] = dyp[p] * acc[p];
+                    dx[off + p] = lp[p] * dz[p];
+                    dlam[off + p] = xp[p] * dz[p];
+                }
             }
         }
     }
-    free(hbuf); free(acc); free(dz); free(dcur); free(dnext); free(wnext);
+    free(hbuf); free(acc); free(dz); free(dcur); free(dnext); free(wnext); free(dd);
     return 0;
+}
+
+int gspn_ref_backward_chunked(int N, int C, int H, int W, int wmode, unsigned mask, int chunk,
+                              const double *x, const double *a, const double *lam, const double *u,
+                              const double *dy, double *dx, double *da, double *dlam, double *du) {
+    return gspn_ref_backward_ex(N, C, H, W, wmode, mask, chunk, 0, x, a, lam, u, dy, dx, da, dlam, du);
 }
 
 int gspn_ref_backward(int N, int C, int H, int W, int wmode, unsigned mask,
                       const double *x, const double *a, const double *lam, const double *u,
                       const double *dy, double *dx, double *da, double *dlam, double *du) {
-    return gspn_ref_backward_chunked(N, C, H, W, wmode, mask, 0, x, a, lam, u, dy, dx, da, dlam, du);
+    return gspn_ref_backward_ex(N, C, H, W, wmode, mask, 0, 0, x, a, lam, u, dy, dx, da, dlam, du);
 }
 
 /* Version tag so that a loader can check it got this file's build. */
-int gspn_ref_abi_version(void) { return 2; }
+int gspn_ref_abi_version(void) { return 3; }

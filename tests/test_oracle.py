@@ -472,3 +472,70 @@ def test_proxy_selecting_one_channel():
     y = oracle.proxy_forward(x, p_in, a, lam, u, p_out, 1, 15)
     assert np.abs(y[:, k:k + 1] - oracle.forward(x[:, k:k + 1], a, lam, u, 1, 15)).max() <= 1e-12
     assert np.all(np.delete(y, k, axis=1) == 0.0)
+
+
+# ----------------------------------------------------------------------------- per-direction lambda / u
+def _per_dir_case(rng, N, C, H, W, mask, wmode):
+    x, a, lam, u = rand_case(rng, N, C, H, W, mask, wmode)
+    D = bin(mask).count("1")
+    lam_d = rng.uniform(0.0, 1.0, (D,) + x.shape)
+    u_d = rng.standard_normal((D,) + x.shape)
+    return x, a, lam_d, u_d
+
+
+def test_per_direction_with_equal_slots_is_the_shared_form():
+    rng = np.random.default_rng(300)
+    x, a, lam, u = rand_case(rng, 1, 2, 5, 6, 15, 1)
+    lam_d, u_d = np.stack([lam] * 4), np.stack([u] * 4)
+    y = oracle.forward(x, a, lam_d, u_d, 1, 15, per_dir=1)
+    assert np.abs(y - oracle.forward(x, a, lam, u, 1, 15)).max() <= 1e-12
+    dy = rng.standard_normal(x.shape)
+    gs = oracle.backward(x, a, lam, u, dy, 1, 15)
+    gd = oracle.backward(x, a, lam_d, u_d, dy, 1, 15, per_dir=1)
+    assert np.abs(gd[0] - gs[0]).max() <= 1e-12          # dx
+    assert np.abs(gd[1] - gs[1]).max() <= 1e-12          # da
+    assert np.abs(gd[2].sum(0) - gs[2]).max() <= 1e-12   # sum_d dlam_d = dlam
+    assert np.abs(gd[3].sum(0) - gs[3]).max() <= 1e-12   # sum_d du_d = du
+
+
+@pytest.mark.parametrize("mask", [15, 6, 9])
+def test_per_direction_is_the_sum_of_single_direction_scans(mask):
+    """y = sum_d u_d * h^d(lam_d x): each term is the single-direction scan with that slot's
+    lambda and u (pins the slot order of the direction axis)."""
+    rng = np.random.default_rng(310 + mask)
+    x, a, lam_d, u_d = _per_dir_case(rng, 2, 2, 5, 7, mask, 0)
+    y = oracle.forward(x, a, lam_d, u_d, 0, mask, per_dir=1)
+    ref = np.zeros_like(x)
+    for s, d in enumerate([d for d in (1, 2, 4, 8) if mask & d]):
+        ref += oracle.forward(x, a[s:s + 1], lam_d[s], u_d[s], 0, d)
+    assert np.abs(y - ref).max() <= 1e-12
+
+
+@pytest.mark.parametrize("wmode", [0, 1])
+@pytest.mark.parametrize("mask", [15, 5])
+def test_per_direction_backward_finite_differences(wmode, mask):
+    rng = np.random.default_rng(320 + mask + 10 * wmode)
+    x, a, lam_d, u_d = _per_dir_case(rng, 1, 2, 4, 5, mask, wmode)
+    dy = rng.standard_normal(x.shape)
+    grads = oracle.backward(x, a, lam_d, u_d, dy, wmode, mask, per_dir=1)
+    args = [x, a, lam_d, u_d]
+    eps = 1e-6
+
+    def loss():
+        return float((dy * oracle.forward(*args, wmode, mask, per_dir=1)).sum())
+
+    for gi in range(4):
+        base = args[gi]
+        fd = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = base[idx]
+            base[idx] = old + eps
+            lp = loss()
+            base[idx] = old - eps
+            lm = loss()
+            base[idx] = old
+            fd[idx] = (lp - lm) / (2 * eps)
+        scale = max(1.0, np.abs(fd).max())
+        assert np.abs(grads[gi] - fd).max() <= 1e-6 * scale, (gi, np.abs(grads[gi] - fd).max())
