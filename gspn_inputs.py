@@ -94,8 +94,10 @@ WORKLOADS = {
 }
 
 
-def make_inputs(wl: Workload, device="cpu", with_dy: bool = False, seed: int | None = None):
-    """Returns a dict with x, a, lam, u (and dy) in the workload's storage dtype on ``device``."""
+def make_inputs(wl: Workload, device="cpu", with_dy: bool = False, seed: int | None = None,
+                per_dir: bool = False):
+    """Returns a dict with x, a, lam, u (and dy) in the workload's storage dtype on ``device``.
+    ``per_dir``: lam and u get a leading direction axis of length D (one map per direction)."""
     g = torch.Generator(device=device)
     g.manual_seed(wl.seed if seed is None else seed)
     shp = (wl.N, wl.C, wl.H, wl.W)
@@ -108,8 +110,9 @@ def make_inputs(wl: Workload, device="cpu", with_dy: bool = False, seed: int | N
         a.mul_(wl.a_std)
     out["a"] = a.to(dt)
     del a
-    out["lam"] = torch.rand(shp, generator=g, device=device, dtype=torch.float32).to(dt)
-    out["u"] = torch.randn(shp, generator=g, device=device, dtype=torch.float32).to(dt)
+    lu = ((wl.D,) if per_dir else ()) + shp
+    out["lam"] = torch.rand(lu, generator=g, device=device, dtype=torch.float32).to(dt)
+    out["u"] = torch.randn(lu, generator=g, device=device, dtype=torch.float32).to(dt)
     if with_dy:
         out["dy"] = torch.randn(shp, generator=g, device=device, dtype=torch.float32).to(dt)
     return out

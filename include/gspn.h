@@ -103,7 +103,17 @@ typedef struct {
     int dtype;          /* gspn_dtype */
     int algo;           /* GSPN_ALGO_*, 0 = AUTO */
     int chunk;          /* lines per local chunk; 0 = global */
+    int per_dir;        /* 1: lam and u have a direction axis (see below); 0: shared */
 } gspn_desc;
+
+/* per_dir = 1: lam and u are D x N x C x H x W (slots ordered as the logits' direction slots);
+ * direction d's scan is driven by lam_d * x and the output is y = sum_d u_d * h^d, a learnable
+ * per-pixel weighting of the directions (the pages' models merge the four directions with a
+ * learnable merge: "Parallel Sequence Modeling via Generalized Spatial Propagation Network"
+ * summary, section "Measured effects"). Gradients: dlam_d = x * delta^d, du_d = dy * h^d,
+ * dx = sum_d lam_d * delta^d, with g^d = u_d * dy starting each reverse scan. The generic family
+ * runs it forward and backward, the plane family forward; values other than 0 / 1:
+ * GSPN_ERR_INVALID_ARG. */
 
 /* Bytes of device workspace that gspn_forward (for_backward = 0) or gspn_backward
  * (for_backward = 1) needs for this descriptor; 0 if the descriptor is invalid or its

@@ -37,7 +37,7 @@ ALGO_NAMES = {ALGO_GENERIC: "generic", ALGO_PLANE: "plane", ALGO_SWEEP: "sweep"}
 class GspnDesc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int), ("C", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
                 ("wmode", ctypes.c_int), ("dir_mask", ctypes.c_uint), ("dtype", ctypes.c_int),
-                ("algo", ctypes.c_int), ("chunk", ctypes.c_int)]
+                ("algo", ctypes.c_int), ("chunk", ctypes.c_int), ("per_dir", ctypes.c_int)]
 
 
 class GspnError(RuntimeError):
@@ -103,13 +103,20 @@ def _dtype_code(t: torch.dtype) -> int:
     raise TypeError(f"unsupported dtype {t} (float32 or bfloat16)")
 
 
-def make_desc(N, C, H, W, wmode=PER_CHANNEL, dir_mask=DIR_ALL, dtype=F32, algo=ALGO_AUTO, chunk=0) -> GspnDesc:
-    return GspnDesc(int(N), int(C), int(H), int(W), int(wmode), int(dir_mask), int(dtype), int(algo), int(chunk))
+def make_desc(N, C, H, W, wmode=PER_CHANNEL, dir_mask=DIR_ALL, dtype=F32, algo=ALGO_AUTO, chunk=0,
+              per_dir=0) -> GspnDesc:
+    return GspnDesc(int(N), int(C), int(H), int(W), int(wmode), int(dir_mask), int(dtype), int(algo), int(chunk),
+                    int(per_dir))
 
 
-def desc_for(x: torch.Tensor, wmode: int, dir_mask: int, algo: int = ALGO_AUTO, chunk: int = 0) -> GspnDesc:
+def desc_for(x: torch.Tensor, wmode: int, dir_mask: int, algo: int = ALGO_AUTO, chunk: int = 0,
+             per_dir: int = 0) -> GspnDesc:
     N, C, H, W = x.shape
-    return make_desc(N, C, H, W, wmode, dir_mask, _dtype_code(x.dtype), algo, chunk)
+    return make_desc(N, C, H, W, wmode, dir_mask, _dtype_code(x.dtype), algo, chunk, per_dir)
+
+
+def _lu_shape(x: torch.Tensor, dir_mask: int, per_dir: int):
+    return ((bin(dir_mask & 15).count("1"),) if per_dir else ()) + tuple(x.shape)
 
 
 def workspace_size(desc: GspnDesc, backward: bool = False) -> int:
@@ -149,15 +156,16 @@ def alloc_workspace(desc: GspnDesc, backward: bool, device) -> torch.Tensor:
 
 
 def forward(x, a, lam, u, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, algo: int = ALGO_AUTO,
-            y=None, ws=None, stream=None, chunk: int = 0) -> torch.Tensor:
+            y=None, ws=None, stream=None, chunk: int = 0, per_dir: int = 0) -> torch.Tensor:
     """y = u * sum_d h^d. x, lam, u: (N, C, H, W); a: (D, N, Cw, 3, H, W); all one dtype.
-    chunk > 0: local propagation within image-aligned chunks of that many lines."""
+    chunk > 0: local propagation within image-aligned chunks of that many lines. per_dir = 1:
+    lam and u are (D, N, C, H, W) and y = sum_d u_d * h^d(lam_d * x)."""
     _check({"x": x, "a": a, "lam": lam, "u": u}, x)
     if tuple(a.shape) != logits_shape(*x.shape, wmode, dir_mask):
         raise ValueError(f"logits shape {tuple(a.shape)}, expected {logits_shape(*x.shape, wmode, dir_mask)}")
-    if lam.shape != x.shape or u.shape != x.shape:
-        raise ValueError("lam and u must have the shape of x")
-    desc = desc_for(x, wmode, dir_mask, algo, chunk)
+    if tuple(lam.shape) != _lu_shape(x, dir_mask, per_dir) or tuple(u.shape) != _lu_shape(x, dir_mask, per_dir):
+        raise ValueError(f"lam and u must be {_lu_shape(x, dir_mask, per_dir)}")
+    desc = desc_for(x, wmode, dir_mask, algo, chunk, per_dir)
     if y is None:
         y = torch.empty_like(x)
     _check({"y": y}, x)
@@ -171,14 +179,16 @@ def forward(x, a, lam, u, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, alg
 
 
 def backward(x, a, lam, u, dy, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, algo: int = ALGO_AUTO,
-             out=None, ws=None, stream=None, chunk: int = 0):
+             out=None, ws=None, stream=None, chunk: int = 0, per_dir: int = 0):
     """Gradients (dx, da, dlam, du) of sum(dy * y)."""
     _check({"x": x, "a": a, "lam": lam, "u": u, "dy": dy}, x)
     if tuple(a.shape) != logits_shape(*x.shape, wmode, dir_mask):
         raise ValueError("logits shape mismatch")
-    desc = desc_for(x, wmode, dir_mask, algo, chunk)
+    if tuple(lam.shape) != _lu_shape(x, dir_mask, per_dir) or tuple(u.shape) != _lu_shape(x, dir_mask, per_dir):
+        raise ValueError(f"lam and u must be {_lu_shape(x, dir_mask, per_dir)}")
+    desc = desc_for(x, wmode, dir_mask, algo, chunk, per_dir)
     if out is None:
-        out = (torch.empty_like(x), torch.empty_like(a), torch.empty_like(x), torch.empty_like(x))
+        out = (torch.empty_like(x), torch.empty_like(a), torch.empty_like(lam), torch.empty_like(u))
     dx, da, dlam, du = out
     _check({"dx": dx, "da": da, "dlam": dlam, "du": du}, x)
     if ws is None:
@@ -270,18 +280,20 @@ class GSPNFunction(torch.autograd.Function):
     """Autograd wrapper: forward and backward both run in libgspn."""
 
     @staticmethod
-    def forward(ctx, x, a, lam, u, wmode, dir_mask, chunk=0):
+    def forward(ctx, x, a, lam, u, wmode, dir_mask, chunk=0, per_dir=0):
         ctx.save_for_backward(x, a, lam, u)
-        ctx.wmode, ctx.dir_mask, ctx.chunk = wmode, dir_mask, chunk
-        return forward(x, a, lam, u, wmode, dir_mask, chunk=chunk)
+        ctx.wmode, ctx.dir_mask, ctx.chunk, ctx.per_dir = wmode, dir_mask, chunk, per_dir
+        return forward(x, a, lam, u, wmode, dir_mask, chunk=chunk, per_dir=per_dir)
 
     @staticmethod
     def backward(ctx, dy):
         x, a, lam, u = ctx.saved_tensors
-        dx, da, dlam, du = backward(x, a, lam, u, dy.contiguous(), ctx.wmode, ctx.dir_mask, chunk=ctx.chunk)
-        return dx, da, dlam, du, None, None, None
+        dx, da, dlam, du = backward(x, a, lam, u, dy.contiguous(), ctx.wmode, ctx.dir_mask, chunk=ctx.chunk,
+                                    per_dir=ctx.per_dir)
+        return dx, da, dlam, du, None, None, None, None
 
 
-def gspn(x, a, lam, u, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, chunk: int = 0):
-    """Differentiable GSPN propagation (libgspn forward and backward); chunk > 0 = local."""
-    return GSPNFunction.apply(x, a, lam, u, wmode, dir_mask, chunk)
+def gspn(x, a, lam, u, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, chunk: int = 0, per_dir: int = 0):
+    """Differentiable GSPN propagation (libgspn forward and backward); chunk > 0 = local;
+    per_dir = 1: per-direction lam and u (D, N, C, H, W)."""
+    return GSPNFunction.apply(x, a, lam, u, wmode, dir_mask, chunk, per_dir)

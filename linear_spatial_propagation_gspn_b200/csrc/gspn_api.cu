@@ -20,6 +20,7 @@ bool make_problem(const gspn_desc* d, Problem* p) {
     if (d->dtype != GSPN_F32 && d->dtype != GSPN_BF16) return false;
     if (d->algo < GSPN_ALGO_AUTO || d->algo > GSPN_ALGO_SWEEP) return false;
     if (d->chunk < 0) return false;
+    if (d->per_dir != 0 && d->per_dir != 1) return false;
     if ((long long)d->N * d->C > 0x7fffffffLL) return false;
     p->N = d->N; p->C = d->C; p->H = d->H; p->W = d->W;
     p->wmode = d->wmode;
@@ -32,17 +33,21 @@ bool make_problem(const gspn_desc* d, Problem* p) {
     p->HW = (long long)d->H * d->W;
     p->U = (long long)d->N * d->C * p->HW;
     p->A = (long long)p->D * d->N * p->Cw * 3 * p->HW;
+    p->per_dir = d->per_dir;
+    p->LU = d->per_dir ? p->D * p->U : p->U;
     return true;
 }
 
 int select_algo(const gspn_desc* d, const Problem& p, bool bwd) {
+    // per-direction lambda / u: the sweep family does not run it
+    if (p.per_dir && d->algo == GSPN_ALGO_SWEEP) return -1;
     switch (d->algo) {
     case GSPN_ALGO_GENERIC: return generic_supports(p, bwd) ? GSPN_ALGO_GENERIC : -1;
     case GSPN_ALGO_PLANE: return plane_supports(p, bwd) ? GSPN_ALGO_PLANE : -1;
     case GSPN_ALGO_SWEEP: return sweep_supports(p, bwd) ? GSPN_ALGO_SWEEP : -1;
     default:
         if (plane_supports(p, bwd)) return GSPN_ALGO_PLANE;
-        if (sweep_supports(p, bwd)) return GSPN_ALGO_SWEEP;
+        if (!p.per_dir && sweep_supports(p, bwd)) return GSPN_ALGO_SWEEP;
         if (generic_supports(p, bwd)) return GSPN_ALGO_GENERIC;
         return -1;
     }
@@ -226,7 +231,7 @@ size_t gspn_forward_host_buffer_size(const gspn_desc* desc) {
     const size_t ws = gspn_workspace_size(desc, 0);
     if (ws == 0) return 0;
     const size_t es = p.esize();
-    return 4 * align256(p.U * es) + align256(p.A * es) + align256(ws);
+    return 2 * align256(p.U * es) + 2 * align256(p.LU * es) + align256(p.A * es) + align256(ws);
 }
 
 gspn_status gspn_forward_host(const gspn_desc* desc, const void* hx, const void* ha, const void* hlam, const void* hu,
@@ -239,20 +244,20 @@ gspn_status gspn_forward_host(const gspn_desc* desc, const void* hx, const void*
     if (need == 0) return GSPN_ERR_UNSUPPORTED;
     if (dev_bytes < need) return GSPN_ERR_WORKSPACE;
     const size_t es = p.esize();
-    const size_t ub = p.U * es, ab = p.A * es;
+    const size_t ub = p.U * es, lb = p.LU * es, ab = p.A * es;
     char* base = (char*)dev;
     char* dx = base;
     char* dlam = dx + align256(ub);
-    char* du = dlam + align256(ub);
-    char* dyo = du + align256(ub);
+    char* du = dlam + align256(lb);
+    char* dyo = du + align256(lb);
     char* da = dyo + align256(ub);
     char* dws = da + align256(ab);
     const size_t wsb = dev_bytes - (size_t)(dws - base);
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaMemcpyAsync(dx, hx, ub, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
     if (cudaMemcpyAsync(da, ha, ab, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(dlam, hlam, ub, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(du, hu, ub, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaMemcpyAsync(dlam, hlam, lb, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaMemcpyAsync(du, hu, lb, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
     gspn_status s = gspn_forward(desc, dx, da, dlam, du, dyo, dws, wsb, stream);
     if (s != GSPN_OK) return s;
     if (cudaMemcpyAsync(hy, dyo, ub, cudaMemcpyDeviceToHost, st) != cudaSuccess) return GSPN_ERR_CUDA;

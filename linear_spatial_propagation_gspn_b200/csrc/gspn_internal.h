@@ -17,6 +17,8 @@ struct Problem {
     unsigned mask;
     int dtype;       // GSPN_F32 / GSPN_BF16
     int chunk;       // lines per local chunk (0: global)
+    int per_dir;     // lam and u carry a direction axis
+    long long LU;    // elements of lam (and of u): U, or D * U with per_dir
     long long HW;    // H * W
     long long U;     // N * C * H * W
     long long A;     // D * N * Cw * 3 * H * W

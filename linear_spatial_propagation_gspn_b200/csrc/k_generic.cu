@@ -32,6 +32,7 @@ struct GenArgs {
     int slot;
     int first, last;    // first / last direction of the mask
     int chunk;          // lines per local chunk (0: global)
+    int per_dir;        // lam and u carry a direction axis: this direction's are at slot * U
 };
 
 // Forward scan of one direction for plane blockIdx.x. Writes y (last direction), the fp32
@@ -44,9 +45,10 @@ __global__ void k_gen_fwd(GenArgs p) {
     const long long HW = (long long)p.H * p.W;
     const int L = is_vertical(p.dir) ? p.H : p.W;
     const int M = is_vertical(p.dir) ? p.W : p.H;
+    const long long lu = p.per_dir ? (long long)p.slot * p.N * p.C * HW : 0;   // this direction's lam / u
     const T* x = (const T*)p.x + plane * HW;
-    const T* lam = (const T*)p.lam + plane * HW;
-    const T* u = (const T*)p.u + plane * HW;
+    const T* lam = (const T*)p.lam + lu + plane * HW;
+    const T* u = (const T*)p.u + lu + plane * HW;
     T* y = (T*)p.y + plane * HW;
     const T* a3 = (const T*)p.a + (((long long)p.slot * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
     float* acc = p.acc ? p.acc + plane * HW : nullptr;
@@ -67,15 +69,17 @@ __global__ void k_gen_fwd(GenArgs p) {
             }
             hc[j] = h;
             if (hst) hst[q] = h;
+            // shared u gates the sum once at the end; a per-direction u weights each term
+            const float hv = p.per_dir ? Io<T>::ld(u + q) * h : h;
             if (p.first && p.last) {
-                if (y != nullptr && !hst) Io<T>::st(y + q, Io<T>::ld(u + q) * h);
-                if (acc) acc[q] = h;
+                if (y != nullptr && !hst) Io<T>::st(y + q, p.per_dir ? hv : Io<T>::ld(u + q) * h);
+                if (acc) acc[q] = hv;
             } else if (p.first) {
-                acc[q] = h;
+                acc[q] = hv;
             } else if (p.last && !hst) {
-                Io<T>::st(y + q, Io<T>::ld(u + q) * (acc[q] + h));
+                Io<T>::st(y + q, p.per_dir ? acc[q] + hv : Io<T>::ld(u + q) * (acc[q] + h));
             } else {
-                acc[q] += h;
+                acc[q] += hv;
             }
         }
         __syncthreads();
@@ -98,6 +102,11 @@ struct GenBwdArgs {
     int slot;
     int first;
     int chunk;           // lines per local chunk (0: global)
+    int per_dir;         // lam and u carry a direction axis (then dlam, du are written here)
+    const void* x;       // per_dir: x, this direction's lam, dlam_d and du_d outputs
+    const void* lam;
+    void* dlam;
+    void* du;
 };
 
 // Reverse scan of one direction for plane blockIdx.x:
@@ -110,7 +119,8 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
     const long long HW = (long long)p.H * p.W;
     const int L = is_vertical(p.dir) ? p.H : p.W;
     const int M = is_vertical(p.dir) ? p.W : p.H;
-    const T* u = (const T*)p.u + plane * HW;
+    const long long lu = p.per_dir ? (long long)p.slot * p.N * p.C * HW : 0;   // this direction's lam / u
+    const T* u = (const T*)p.u + lu + plane * HW;
     const T* dy = (const T*)p.dy + plane * HW;
     const long long abase = (((long long)p.slot * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
     const T* a3 = (const T*)p.a + abase;
@@ -135,8 +145,18 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
                 if (j < M - 1) del = fmaf(wprev[j + 1], dprev[j + 1], del);
             }
             dcur[j] = del;
-            if (p.first) dz[q] = del;
-            else dz[q] += del;
+            if (p.per_dir) {
+                // dlam_d = x delta^d, du_d = dy h^d; dz accumulates dx = sum_d lam_d delta^d
+                const long long pq = lu + plane * HW + q;
+                const float lamv = Io<T>::ld((const T*)p.lam + pq);
+                Io<T>::st((T*)p.dlam + pq, Io<T>::ld((const T*)p.x + plane * HW + q) * del);
+                Io<T>::st((T*)p.du + pq, Io<T>::ld(dy + q) * hs[q]);
+                if (p.first) dz[q] = lamv * del;
+                else dz[q] += lamv * del;
+            } else {
+                if (p.first) dz[q] = del;
+                else dz[q] += del;
+            }
             if (!chunk_start(scan_ascending(p.dir), L, p.chunk, i)) {
                 const bool hl = j > 0, hr = j < M - 1;
                 LaneJac J = lane_jacobian(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q), Io<T>::ld(a3 + 2 * HW + q),
@@ -200,7 +220,7 @@ cudaError_t gen_forward_t(const Problem& P, const void* x, const void* a, const 
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
         GenArgs g{x, a, lam, u, y, acc, nullptr, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, seen == P.D - 1,
-                  P.chunk};
+                  P.chunk, P.per_dir};
         const int M = is_vertical(d) ? P.W : P.H;
         const size_t smem = 2 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -234,7 +254,7 @@ cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const
         const int M = is_vertical(d) ? P.W : P.H;
         // 1) recompute this direction's h (image coordinates) and accumulate sum_d h for du
         GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, false,
-                  P.chunk};
+                  P.chunk, P.per_dir};
         if (P.D == 1) g.first = 1;
         size_t smem = 2 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -242,7 +262,7 @@ cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         // 2) reverse scan
         GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, P.H, P.W, P.Cw, d, slot, seen == 0,
-                     P.chunk};
+                     P.chunk, P.per_dir, x, lam, dlam, du};
         smem = 8 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_gen_bwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(b);
@@ -251,8 +271,12 @@ cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const
         ++seen;
     }
     const int blocks = (int)std::max<long long>(1, std::min<long long>(4096, (P.U + 255) / 256));
-    k_gen_bwd_final<T><<<blocks, 256, 0, st>>>((const T*)x, (const T*)lam, (const T*)dy, dz, acc, (T*)dx,
-                                               (T*)dlam, (T*)du, P.U);
+    if (P.per_dir) {
+        k_f32_to<T><<<blocks, 256, 0, st>>>(dz, (T*)dx, P.U);   // dlam_d, du_d written per direction
+    } else {
+        k_gen_bwd_final<T><<<blocks, 256, 0, st>>>((const T*)x, (const T*)lam, (const T*)dy, dz, acc, (T*)dx,
+                                                   (T*)dlam, (T*)du, P.U);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (dacc) {
         const int ab = (int)std::max<long long>(1, std::min<long long>(4096, (P.A + 255) / 256));

@@ -66,8 +66,10 @@ __device__ __forceinline__ int plane_pix(int H, int W, int Wp, int i, int j) {
 // pipelined: the shared-memory operands of step i + 1 (z, w0, w2 and the running sum) are
 // loaded while step i's new line is formed, so a step waits only for the shuffles and FMAs of
 // the recurrence. Lanes past the line (j >= M) read index 0 and contribute nothing.
-template <unsigned D, int LPT, bool LOCAL>
-__device__ __forceinline__ void plane_scan(const float* z, const float* w0b, const float* w2b, float* acc, int H,
+// PD (per-direction lambda / u): the scan writes h^D over z (each z value is read before its
+// pixel's h is written) and leaves the running sum to the caller, which weights h^D by u_D.
+template <unsigned D, int LPT, bool LOCAL, bool PD = false>
+__device__ __forceinline__ void plane_scan(float* z, const float* w0b, const float* w2b, float* acc, int H,
                                            int W, int Wp, int chunk, int lane) {
     constexpr bool V = D == kTB || D == kBT;
     const int L = V ? H : W, M = V ? W : H;
@@ -85,7 +87,7 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
         cz[e] = z[cq[e]];
         cw0[e] = 0.f;   // step 0 has no predecessor: h_0 = z
         cw2[e] = 0.f;
-        ca[e] = acc[cq[e]];
+        ca[e] = PD ? 0.f : acc[cq[e]];
     }
     for (int i = 0; i < L; ++i) {
         // operands of step i + 1
@@ -111,7 +113,10 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
             const float right = e == LPT - 1 ? hr : h[e + 1];
             const float v = fmaf(cw0[e], left, fmaf(1.f - cw0[e] - cw2[e], h[e], fmaf(cw2[e], right, cz[e])));
             hn[e] = on[e] ? v : 0.f;
-            if (on[e]) acc[cq[e]] = ca[e] + v;
+            if (on[e]) {
+                if (PD) z[cq[e]] = v;
+                else acc[cq[e]] = ca[e] + v;
+            }
         }
         // the running sum of step i + 1 is read after this step's writes (different pixels
         // except at the same lane, which this thread owns); a chunk's first step starts from
@@ -123,7 +128,7 @@ __device__ __forceinline__ void plane_scan(const float* z, const float* w0b, con
         }
 #pragma unroll
         for (int e = 0; e < LPT; ++e) {
-            na[e] = acc[nq[e]];
+            na[e] = PD ? 0.f : acc[nq[e]];
             h[e] = restart ? 0.f : hn[e];
             cz[e] = nz[e];
             cw0[e] = nw0[e];
@@ -177,16 +182,48 @@ __device__ __forceinline__ void plane_weights(const T* a3, float* w0b, float* w2
     }
 }
 
-template <typename T, unsigned D, int LPT, bool LOCAL>
-__device__ __forceinline__ void plane_direction(const T* a3, const float* z, float* w0b, float* w2b, float* acc, int H,
+template <typename T, unsigned D, int LPT, bool LOCAL, bool PD = false>
+__device__ __forceinline__ void plane_direction(const T* a3, float* z, float* w0b, float* w2b, float* acc, int H,
                                                 int W, int Wp, int chunk, int tid) {
     plane_weights<T, D>(a3, w0b, w2b, H, W, Wp, tid);
     __syncthreads();
-    if (tid < 32) plane_scan<D, LPT, LOCAL>(z, w0b, w2b, acc, H, W, Wp, chunk, tid);
+    if (tid < 32) plane_scan<D, LPT, LOCAL, PD>(z, w0b, w2b, acc, H, W, Wp, chunk, tid);
     __syncthreads();
 }
 
-template <typename T, int LPT, bool LOCAL>
+// z = lam * x over the plane (all threads; plane layout with row stride Wp).
+template <typename T>
+__device__ __forceinline__ void plane_load_z(const T* x, const T* lam, float* z, int H, int W, int Wp, int tid) {
+    const int HW = H * W;
+    if (W % 4 == 0) {
+        for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
+            const int r = e / W, col = e - r * W;
+            float xv[4], lv[4];
+            ld_lanes<T, 4>(x + e, xv);
+            ld_lanes<T, 4>(lam + e, lv);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) z[r * Wp + col + k] = lv[k] * xv[k];
+        }
+    } else {
+        for (int e = tid; e < HW; e += kPlaneThreads) {
+            const int r = e / W, col = e - r * W;
+            z[r * Wp + col] = Io<T>::ld(lam + e) * Io<T>::ld(x + e);
+        }
+    }
+}
+
+// acc (+)= g * src over the plane, g a storage-dtype tensor in image layout (all threads).
+template <typename T, bool FIRST>
+__device__ __forceinline__ void plane_axpy(const T* g, const float* src, float* acc, int H, int W, int Wp, int tid) {
+    const int HW = H * W;
+    for (int e = tid; e < HW; e += kPlaneThreads) {
+        const int q = (e / W) * Wp + e % W;
+        const float v = Io<T>::ld(g + e) * src[q];
+        acc[q] = FIRST ? v : acc[q] + v;
+    }
+}
+
+template <typename T, int LPT, bool LOCAL, bool PD>
 __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
     extern __shared__ float sm[];
     const int H = p.H, W = p.W, Wp = p.Wp;
@@ -198,48 +235,41 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
     const int tid = threadIdx.x;
     const int HW = H * W;
     const int nplanes = p.N * p.C;
-    const bool vec = W % 4 == 0;
+    const long long U = (long long)nplanes * HW;   // one N x C x H x W tensor (per-direction stride)
     for (int plane = blockIdx.x; plane < nplanes; plane += gridDim.x) {
         const int n = plane / p.C, c = plane % p.C;
         const long long po = (long long)plane * HW;
         const T* x = (const T*)p.x + po;
-        const T* lam = (const T*)p.lam + po;
-        const T* u = (const T*)p.u + po;
         T* y = (T*)p.y + po;
-        // z = lambda * x, sum = 0
-        if (vec) {
-            for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
-                const int r = e / W, col = e - r * W;
-                float xv[4], lv[4];
-                ld_lanes<T, 4>(x + e, xv);
-                ld_lanes<T, 4>(lam + e, lv);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    z[r * Wp + col + k] = lv[k] * xv[k];
-                    acc[r * Wp + col + k] = 0.f;
-                }
-            }
-        } else {
-            for (int e = tid; e < HW; e += kPlaneThreads) {
-                const int r = e / W, col = e - r * W;
-                z[r * Wp + col] = Io<T>::ld(lam + e) * Io<T>::ld(x + e);
-                acc[r * Wp + col] = 0.f;
-            }
-        }
+        // shared lam / u: z = lambda * x once and sum = 0; per-direction: sum = 0 (z per direction)
+        if (!PD) plane_load_z<T>(x, (const T*)p.lam + po, z, H, W, Wp, tid);
+        for (int e = tid; e < HW; e += kPlaneThreads) acc[(e / W) * Wp + e % W] = 0.f;
         int slot = 0;
         auto a_of = [&](int s) {
             return (const T*)p.a + (((long long)s * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
         };
-        if (p.mask & kTB) plane_direction<T, kTB, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
-        if (p.mask & kBT) plane_direction<T, kBT, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
-        if (p.mask & kLR) plane_direction<T, kLR, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
-        if (p.mask & kRL) plane_direction<T, kRL, LPT, LOCAL>(a_of(slot++), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid);
-        // y = u * sum
-        if (vec) {
+        // per-direction lam / u: z = lam_s x before the direction (its first barrier orders it),
+        // the scan leaves h^D in z, and sum += u_s h^D after it
+        auto pre = [&](int s) {
+            if (PD) plane_load_z<T>(x, (const T*)p.lam + s * U + po, z, H, W, Wp, tid);
+        };
+        auto post = [&](int s) {
+            if (PD) {
+                plane_axpy<T, false>((const T*)p.u + s * U + po, z, acc, H, W, Wp, tid);
+                __syncthreads();
+            }
+        };
+        if (p.mask & kTB) { pre(slot); plane_direction<T, kTB, LPT, LOCAL, PD>(a_of(slot), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid); post(slot++); }
+        if (p.mask & kBT) { pre(slot); plane_direction<T, kBT, LPT, LOCAL, PD>(a_of(slot), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid); post(slot++); }
+        if (p.mask & kLR) { pre(slot); plane_direction<T, kLR, LPT, LOCAL, PD>(a_of(slot), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid); post(slot++); }
+        if (p.mask & kRL) { pre(slot); plane_direction<T, kRL, LPT, LOCAL, PD>(a_of(slot), z, w0b, w2b, acc, H, W, Wp, p.chunk, tid); post(slot++); }
+        // y = u * sum (shared u) or y = sum (per-direction u already applied)
+        const T* u = (const T*)p.u + po;
+        if (W % 4 == 0) {
             for (int e = tid * 4; e < HW; e += kPlaneThreads * 4) {
                 const int r = e / W, col = e - r * W;
-                float uv[4];
-                ld_lanes<T, 4>(u + e, uv);
+                float uv[4] = {1.f, 1.f, 1.f, 1.f};
+                if (!PD) ld_lanes<T, 4>(u + e, uv);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) uv[k] *= acc[r * Wp + col + k];
                 st_lanes<T, 4>(y + e, uv);
@@ -247,7 +277,7 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
         } else {
             for (int e = tid; e < HW; e += kPlaneThreads) {
                 const int r = e / W, col = e - r * W;
-                Io<T>::st(y + e, Io<T>::ld(u + e) * acc[r * Wp + col]);
+                Io<T>::st(y + e, (PD ? 1.f : Io<T>::ld(u + e)) * acc[r * Wp + col]);
             }
         }
         __syncthreads();
@@ -555,19 +585,19 @@ cudaError_t plane_bwd_launch3(const Problem& P, const PlaneBwdArgs& a, cudaStrea
     return cudaGetLastError();
 }
 
-template <typename T, int LPT, bool LOCAL>
+template <typename T, int LPT, bool LOCAL, bool PD>
 cudaError_t plane_fwd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
     const size_t smem = plane_smem(P);
-    cudaError_t e = cudaFuncSetAttribute(k_plane_fwd<T, LPT, LOCAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_plane_fwd<T, LPT, LOCAL, PD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaFuncSetAttribute(k_plane_fwd<T, LPT, LOCAL>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(k_plane_fwd<T, LPT, LOCAL, PD>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     int per_sm = 1;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_fwd<T, LPT, LOCAL>, kPlaneThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_plane_fwd<T, LPT, LOCAL, PD>, kPlaneThreads, smem);
     if (e != cudaSuccess) return e;
     const long long want = (long long)std::max(1, per_sm) * device_sm_count();
     const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
     launch_begin(st);
-    k_plane_fwd<T, LPT, LOCAL><<<grid, kPlaneThreads, smem, st>>>(a);
+    k_plane_fwd<T, LPT, LOCAL, PD><<<grid, kPlaneThreads, smem, st>>>(a);
     launch_end(st);
     return cudaGetLastError();
 }
@@ -575,7 +605,11 @@ cudaError_t plane_fwd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t
 // Local propagation has its own instantiations, so the global scans carry no chunk counters.
 template <typename T, int LPT>
 cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
-    return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true>(P, a, st) : plane_fwd_launch3<T, LPT, false>(P, a, st);
+    if (P.per_dir)
+        return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true, true>(P, a, st)
+                           : plane_fwd_launch3<T, LPT, false, true>(P, a, st);
+    return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true, false>(P, a, st)
+                       : plane_fwd_launch3<T, LPT, false, false>(P, a, st);
 }
 template <typename T, int LPT>
 cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
@@ -598,7 +632,7 @@ cudaError_t plane_forward_t(const Problem& P, const void* x, const void* a, cons
 bool plane_supports(const Problem& P, bool bwd) {
     if (std::max(P.H, P.W) > kPlaneMaxLanes) return false;
     if ((long long)P.H * P.W > (1LL << 20)) return false;
-    if (bwd) return P.wmode == GSPN_W_PER_CHANNEL && plane_bwd_smem(P) <= kPlaneSmemBudget;
+    if (bwd) return P.wmode == GSPN_W_PER_CHANNEL && !P.per_dir && plane_bwd_smem(P) <= kPlaneSmemBudget;
     return plane_smem(P) <= kPlaneSmemBudget;
 }
 

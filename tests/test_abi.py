@@ -44,7 +44,7 @@ def desc(**kw):
 
 
 @pytest.mark.parametrize("bad", [dict(N=0), dict(C=-1), dict(H=0), dict(W=0), dict(dir_mask=0), dict(dir_mask=16),
-                                 dict(wmode=2), dict(dtype=7), dict(algo=9), dict(chunk=-1)])
+                                 dict(wmode=2), dict(dtype=7), dict(algo=9), dict(chunk=-1), dict(per_dir=2)])
 def test_invalid_descriptor(bad):
     d = desc(**bad)
     assert g.workspace_size(d) == 0
