@@ -284,6 +284,326 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
     }
 }
 
+// ====================================================== forward, directions scanned concurrently
+// One CTA per plane (persistent over planes), one warp per direction: after z = lambda x is in
+// shared memory, the D directions of the mask are scanned at the same time, each warp writing
+// its h^d to a plane buffer of its own; y = u * (h^TB + h^BT + h^LR + h^RL) is then summed in
+// that fixed order, so the result does not depend on warp timing. Each scanning warp streams
+// its three logit planes through a ring of NSL strips of K = 16 / sizeof(T) scan lines filled
+// with 16-byte cp.async copies that bypass L1, so the logits are read from HBM exactly once and
+// the transposed walks of the horizontal directions read one 16-byte run per lane and strip;
+// the weights of a whole strip are formed before its K recurrence steps, off the
+// h chain. Lane j of a scan line is held by thread j % 32 as its element j / 32 (interleaved),
+// which keeps every row and column walk of the odd-stride planes conflict-free.
+
+__device__ __forceinline__ uint32_t cd_saddr(const void* ptr) { return (uint32_t)__cvta_generic_to_shared(ptr); }
+__device__ __forceinline__ void cd_cp16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(cd_saddr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cd_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cd_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Float offset of the rings in shared memory: after z and the nd h planes, rounded up to 16 bytes.
+__host__ __device__ constexpr int cd_ring_offset(int nd, int HWs) { return ((1 + nd) * HWs + 3) & ~3; }
+
+template <typename T> struct CdGeom {
+    static constexpr int K = 16 / (int)sizeof(T);   // scan lines per ring strip = elements per 16 bytes
+};
+// 32-bit words of one ring strip: 3 logit planes x K lines x 32 LPT lanes (both storage types).
+template <int LPT> __host__ __device__ constexpr int cd_slot_words() { return 384 * LPT; }
+
+// Geometry of one direction as seen by its scanning warp. Scan position (i, j) (line i, lane j)
+// is plane-buffer element p0 + i si + j sj (row stride Wp) and image element g0 + i gi + j gj.
+// The direction is a runtime value so that the four warps of a CTA run the same instructions.
+struct CdDir {
+    bool vert, asc;
+    int L, M;
+    int p0, si, sj;
+    int g0, gi, gj;
+};
+
+__device__ __forceinline__ CdDir cd_dir(unsigned d, int H, int W, int Wp) {
+    CdDir g;
+    g.vert = d == kTB || d == kBT;
+    g.asc = d == kTB || d == kLR;
+    g.L = g.vert ? H : W;
+    g.M = g.vert ? W : H;
+    if (d == kTB) { g.p0 = 0; g.si = Wp; g.sj = 1; g.g0 = 0; g.gi = W; g.gj = 1; }
+    else if (d == kBT) { g.p0 = (H - 1) * Wp; g.si = -Wp; g.sj = 1; g.g0 = (H - 1) * W; g.gi = -W; g.gj = 1; }
+    else if (d == kLR) { g.p0 = 0; g.si = 1; g.sj = Wp; g.g0 = 0; g.gi = 1; g.gj = W; }
+    else { g.p0 = W - 1; g.si = -1; g.sj = Wp; g.g0 = W - 1; g.gi = -1; g.gj = W; }
+    return g;
+}
+
+// Issues the copies of strip q (scan lines q K .. q K + K - 1) into one ring slot, all 16-byte
+// cp.async that bypass L1 (image rows are a multiple of 16 bytes). Vertical strips: the K image
+// rows are copied chunk by chunk (the warp's 32 copies cover consecutive chunks) and land
+// line-major, element (k, s, j) at element offset (k K + s) 32 LPT + j. Horizontal strips: every
+// lane (image row) j copies its own 16-byte run of K columns of each logit plane to chunk
+// k 32 LPT + j, read back whole by that thread. Copies past the plane are skipped.
+template <typename T, int LPT>
+__device__ __forceinline__ void cd_fetch(uint32_t* slot, const T* a3, const CdDir& g, int HW, int W, int q, int lane) {
+    constexpr int K = CdGeom<T>::K;
+    const int i0 = q * K;
+    if (g.vert) {
+        const int nc = g.M / K;               // chunks per image row
+        const int rows = min(K, g.L - i0);    // lines of this strip inside the plane
+        const int per_k = rows * nc;
+        T* dst0 = reinterpret_cast<T*>(slot);
+        for (int idx = lane; idx < 3 * per_k; idx += 32) {
+            const int k = idx / per_k, rem = idx - k * per_k;
+            const int s = rem / nc, c = rem - s * nc;
+            cd_cp16(dst0 + (k * K + s) * 32 * LPT + c * K, a3 + k * HW + g.g0 + (i0 + s) * g.gi + c * K);
+        }
+    } else {
+        const int col = g.asc ? i0 : W - K - i0;   // first column of the run
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+#pragma unroll
+            for (int e = 0; e < LPT; ++e) {
+                const int j = e * 32 + lane;
+                if (j < g.M) cd_cp16(slot + (k * 32 * LPT + j) * 4, a3 + k * HW + j * W + col);
+            }
+    }
+}
+
+// All logits of the strip for this thread's lanes: lg[k][s][e] = logit k of line s, lane e 32 + lane.
+template <typename T, int LPT>
+__device__ __forceinline__ void cd_strip_logits(const uint32_t* slot, const CdDir& g, int lane,
+                                                float (&lg)[3][CdGeom<T>::K][LPT]) {
+    constexpr int K = CdGeom<T>::K;
+    if (g.vert) {
+        const T* src = reinterpret_cast<const T*>(slot);
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+#pragma unroll
+            for (int s = 0; s < K; ++s)
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) lg[k][s][e] = Io<T>::ld(src + (k * K + s) * 32 * LPT + e * 32 + lane);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+#pragma unroll
+            for (int e = 0; e < LPT; ++e) {
+                const uint4 v = reinterpret_cast<const uint4*>(slot)[k * 32 * LPT + e * 32 + lane];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                float f[K];   // columns in ascending order
+                if constexpr (sizeof(T) == 4) {
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) f[t] = __uint_as_float(w[t]);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 p2 = unpack2<T>(w[t]);
+                        f[2 * t] = p2.x;
+                        f[2 * t + 1] = p2.y;
+                    }
+                }
+#pragma unroll
+                for (int s = 0; s < K; ++s) lg[k][s][e] = g.asc ? f[s] : f[K - 1 - s];
+            }
+    }
+}
+
+// Issues the first NSL strips (one commit group per strip, empty past the end).
+template <typename T, int LPT, int NSL>
+__device__ __forceinline__ void cd_prime(uint32_t* ring, const T* a3, const CdDir& g, int HW, int W, int lane) {
+    constexpr int K = CdGeom<T>::K;
+    const int nq = (g.L + K - 1) / K;
+#pragma unroll
+    for (int q = 0; q < NSL; ++q) {
+        if (q < nq) cd_fetch<T, LPT>(ring + q * cd_slot_words<LPT>(), a3, g, HW, W, q, lane);
+        cd_commit();
+    }
+}
+
+// Scan of one direction by one warp: h of the plane into hb (plane layout, row stride Wp). The
+// ring already holds strips 0 .. NSL - 1 (issued by cd_prime).
+template <typename T, int LPT, bool LOCAL, int NSL>
+__device__ __forceinline__ void cd_scan(const float* z, float* hb, uint32_t* ring, const T* a3, const CdDir& g,
+                                        int HW, int W, int chunk, int lane) {
+    constexpr int K = CdGeom<T>::K;
+    constexpr int SLOT = cd_slot_words<LPT>();
+    const int L = g.L, M = g.M;
+    const int nq = (L + K - 1) / K;
+    float h[LPT];
+    bool on[LPT], hl[LPT], hr[LPT];
+    int pj[LPT];   // plane offset of (line 0, lane j)
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) {
+        const int j = e * 32 + lane;
+        h[e] = 0.f;
+        on[e] = j < M;
+        hl[e] = j > 0;
+        hr[e] = j < M - 1;
+        pj[e] = on[e] ? g.p0 + j * g.sj : 0;
+    }
+    int crem = first_chunk_len(g.asc, L, chunk);   // lines left in this chunk
+    const int clen = chunk > 0 ? chunk : L;
+    for (int q = 0; q < nq; ++q) {
+        cd_wait<NSL - 1>();
+        __syncwarp();
+        uint32_t* slot = ring + (q % NSL) * SLOT;
+        // normalised weights of the whole strip (independent of h)
+        float w0[K][LPT], w2[K][LPT];
+        bool shift = false;
+        {
+            float lg[3][K][LPT];
+            cd_strip_logits<T, LPT>(slot, g, lane, lg);
+#pragma unroll
+            for (int s = 0; s < K; ++s)
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) {
+                    const Wts w = lane_weights_fast_nocheck(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                    shift |= on[e] && q * K + s < L &&
+                             weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                    w0[s][e] = w.w0;
+                    w2[s][e] = w.w2;
+                }
+            if (__any_sync(0xffffffffu, shift)) {   // rare: some logit below the fast form's range
+#pragma unroll
+                for (int s = 0; s < K; ++s)
+#pragma unroll
+                    for (int e = 0; e < LPT; ++e)
+                        if (weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e])) {
+                            const Wts w = weights_shifted(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                            w0[s][e] = w.w0;
+                            w2[s][e] = w.w2;
+                        }
+            }
+        }
+        // the strip's logits are consumed: refill its slot now, NSL strips ahead of use
+        __syncwarp();
+        if (q + NSL < nq) cd_fetch<T, LPT>(slot, a3, g, HW, W, q + NSL, lane);
+        cd_commit();
+#pragma unroll
+        for (int s = 0; s < K; ++s) {
+            const int i = q * K + s;
+            if (i < L) {   // warp-uniform
+                const int di = i * g.si;
+                float zi[LPT];
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) zi[e] = z[on[e] ? pj[e] + di : 0];
+                // neighbours j - 1 and j + 1: rotate each element across the warp by one lane;
+                // lane 0 / 31 take the wrapped value of the previous / next element
+                float rl[LPT], rr[LPT];
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) {
+                    rl[e] = __shfl_sync(0xffffffffu, h[e], (lane + 31) & 31);
+                    rr[e] = __shfl_sync(0xffffffffu, h[e], (lane + 1) & 31);
+                }
+                bool restart = false;
+                if constexpr (LOCAL) {
+                    restart = --crem == 0;
+                    if (restart) crem = clen;
+                }
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) {
+                    const float left = lane > 0 ? rl[e] : (e > 0 ? rl[e - 1] : 0.f);
+                    const float right = lane < 31 ? rr[e] : (e < LPT - 1 ? rr[e + 1] : 0.f);
+                    const float a = w0[s][e], c = w2[s][e];
+                    const float v = fmaf(a, left, fmaf(1.f - a - c, h[e], fmaf(c, right, zi[e])));
+                    if (on[e]) hb[pj[e] + di] = v;
+                    h[e] = (on[e] && !restart) ? v : 0.f;
+                }
+            }
+        }
+    }
+}
+
+constexpr int kCdThreads = 128;   // one warp per direction
+
+template <typename T, int LPT, bool LOCAL, int NSL>
+__global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
+    extern __shared__ __align__(16) float sm[];
+    constexpr int UNR = 4;   // vectors of 4 per thread whose loads are in flight together
+    const int H = p.H, W = p.W, Wp = p.Wp;
+    const int HW = H * W, HWs = H * Wp;
+    const int nd = __popc(p.mask);
+    float* z = sm;
+    float* hb = z + HWs;                                        // nd planes, slot order
+    // nd rings of NSL strips, 16-byte aligned for the copies and the 16-byte reads
+    uint32_t* rings = reinterpret_cast<uint32_t*>(sm + cd_ring_offset(nd, HWs));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // this warp's direction: the warp-th set bit of the mask (its logit slot is warp)
+    unsigned dir = 0;
+    {
+        unsigned m = p.mask;
+        for (int k = 0; k < warp && m; ++k) m &= m - 1;
+        dir = m & (0u - m);
+    }
+    const CdDir geo = cd_dir(dir, H, W, Wp);
+    const bool scans = warp < nd;
+    uint32_t* ring = rings + warp * NSL * cd_slot_words<LPT>();
+    float* hw = hb + warp * HWs;
+    const int nplanes = p.N * p.C;
+    for (int plane = blockIdx.x; plane < nplanes; plane += gridDim.x) {
+        const int n = plane / p.C, c = plane % p.C;
+        const long long po = (long long)plane * HW;
+        const T* a3 = (const T*)p.a + (((long long)warp * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
+        // the first logit strips go out before z is formed
+        if (scans) cd_prime<T, LPT, NSL>(ring, a3, geo, HW, W, lane);
+        {
+            const T* x = (const T*)p.x + po;
+            const T* lam = (const T*)p.lam + po;
+            for (int e0 = tid * 4; e0 < HW; e0 += kCdThreads * 4 * UNR) {
+                float xv[UNR][4], lv[UNR][4];
+#pragma unroll
+                for (int r = 0; r < UNR; ++r) {
+                    const int e = e0 + r * kCdThreads * 4;
+                    if (e < HW) {
+                        ld_lanes<T, 4>(x + e, xv[r]);
+                        ld_lanes<T, 4>(lam + e, lv[r]);
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < UNR; ++r) {
+                    const int e = e0 + r * kCdThreads * 4;
+                    if (e < HW) {
+                        const int row = e / W, col = e - row * W;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) z[row * Wp + col + k] = lv[r][k] * xv[r][k];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (scans) cd_scan<T, LPT, LOCAL, NSL>(z, hw, ring, a3, geo, HW, W, p.chunk, lane);
+        __syncthreads();
+        // y = u * sum_d h^d, summed in slot order
+        {
+            const T* u = (const T*)p.u + po;
+            T* y = (T*)p.y + po;
+            for (int e0 = tid * 4; e0 < HW; e0 += kCdThreads * 4 * UNR) {
+                float uv[UNR][4];
+#pragma unroll
+                for (int r = 0; r < UNR; ++r) {
+                    const int e = e0 + r * kCdThreads * 4;
+                    if (e < HW) ld_lanes<T, 4>(u + e, uv[r]);
+                }
+#pragma unroll
+                for (int r = 0; r < UNR; ++r) {
+                    const int e = e0 + r * kCdThreads * 4;
+                    if (e < HW) {
+                        const int row = e / W, col = e - row * W;
+                        float v[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int q = row * Wp + col + k;
+                            float s = hb[q];
+                            for (int d = 1; d < nd; ++d) s += hb[d * HWs + q];
+                            v[k] = uv[r][k] * s;
+                        }
+                        st_lanes<T, 4>(y + e, v);
+                    }
+                }
+            }
+        }
+        // the next plane's z and h writes come after its first barrier, which every thread
+        // reaches only after this plane's sum
+    }
+}
+
 // ================================================================== backward (per-channel)
 struct PlaneBwdArgs {
     const void* x;
@@ -602,9 +922,49 @@ cudaError_t plane_fwd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t
     return cudaGetLastError();
 }
 
+size_t cd_smem(const Problem& P, int nsl, int lpt) {
+    const int nd = __builtin_popcount(P.mask);
+    const int slot = 384 * lpt;   // words per ring strip (cd_slot_words)
+    return (size_t)cd_ring_offset(nd, P.H * plane_wp(P)) * sizeof(float) + (size_t)nd * nsl * slot * 4;
+}
+// Ring depth of the concurrent-direction forward: three strips when two CTAs still fit on an SM,
+// else two; 0 when the kernel does not apply (per-direction lambda / u, rows not a multiple of
+// 4 elements, or the planes do not fit).
+int cd_ring_depth(const Problem& P) {
+    if (P.per_dir || P.W % (P.dtype == GSPN_F32 ? 4 : 8) != 0) return 0;   // rows of whole 16-byte chunks
+    const int lpt = plane_lanes(P);
+    if (cd_smem(P, 3, lpt) <= kPlaneSmemBudget / 2) return 3;
+    return cd_smem(P, 2, lpt) <= kPlaneSmemBudget ? 2 : 0;
+}
+
+template <typename T, int LPT, bool LOCAL, int NSL>
+cudaError_t plane_cd_launch4(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
+    const size_t smem = cd_smem(P, NSL, LPT);
+    auto kern = k_plane_fwd_cd<T, LPT, LOCAL, NSL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int per_sm = 1;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCdThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long want = (long long)std::max(1, per_sm) * device_sm_count();
+    const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
+    launch_begin(st);
+    kern<<<grid, kCdThreads, smem, st>>>(a);
+    launch_end(st);
+    return cudaGetLastError();
+}
+template <typename T, int LPT, bool LOCAL>
+cudaError_t plane_cd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
+    return cd_ring_depth(P) == 3 ? plane_cd_launch4<T, LPT, LOCAL, 3>(P, a, st)
+                                 : plane_cd_launch4<T, LPT, LOCAL, 2>(P, a, st);
+}
+
 // Local propagation has its own instantiations, so the global scans carry no chunk counters.
 template <typename T, int LPT>
 cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
+    if (cd_ring_depth(P) > 0)
+        return P.chunk > 0 ? plane_cd_launch3<T, LPT, true>(P, a, st) : plane_cd_launch3<T, LPT, false>(P, a, st);
     if (P.per_dir)
         return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true, true>(P, a, st)
                            : plane_fwd_launch3<T, LPT, false, true>(P, a, st);
