@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
 }
 
 // ====================================================== forward, directions scanned concurrently
-// One CTA per plane (persistent over planes), one warp per direction: after z = lambda x is in
+// fp32 storage. One CTA per plane (persistent over planes), one warp per direction: after z = lambda x is in
 // shared memory, the D directions of the mask are scanned at the same time, each warp writing
 // its h^d to a plane buffer of its own; y = u * (h^TB + h^BT + h^LR + h^RL) is then summed in
 // that fixed order, so the result does not depend on warp timing. Each scanning warp streams
@@ -371,6 +371,7 @@ __device__ __forceinline__ void cd_fetch(uint32_t* slot, const T* a3, const CdDi
 template <typename T, int LPT>
 __device__ __forceinline__ void cd_strip_logits(const uint32_t* slot, const CdDir& g, int lane,
                                                 float (&lg)[3][CdGeom<T>::K][LPT]) {
+    static_assert(sizeof(T) == 4, "the concurrent-direction forward runs fp32 storage");
     constexpr int K = CdGeom<T>::K;
     if (g.vert) {
         const T* src = reinterpret_cast<const T*>(slot);
@@ -387,18 +388,8 @@ __device__ __forceinline__ void cd_strip_logits(const uint32_t* slot, const CdDi
             for (int e = 0; e < LPT; ++e) {
                 const uint4 v = reinterpret_cast<const uint4*>(slot)[k * 32 * LPT + e * 32 + lane];
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                float f[K];   // columns in ascending order
-                if constexpr (sizeof(T) == 4) {
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) f[t] = __uint_as_float(w[t]);
-                } else {
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float2 p2 = unpack2<T>(w[t]);
-                        f[2 * t] = p2.x;
-                        f[2 * t + 1] = p2.y;
-                    }
-                }
+                const float f[K] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                                    __uint_as_float(v.w)};   // columns in ascending order
 #pragma unroll
                 for (int s = 0; s < K; ++s) lg[k][s][e] = g.asc ? f[s] : f[K - 1 - s];
             }
@@ -928,10 +919,12 @@ size_t cd_smem(const Problem& P, int nsl, int lpt) {
     return (size_t)cd_ring_offset(nd, P.H * plane_wp(P)) * sizeof(float) + (size_t)nd * nsl * slot * 4;
 }
 // Ring depth of the concurrent-direction forward: three strips when two CTAs still fit on an SM,
-// else two; 0 when the kernel does not apply (per-direction lambda / u, rows not a multiple of
-// 4 elements, or the planes do not fit).
+// else two; 0 when the kernel does not apply (bf16 storage, per-direction lambda / u, rows not a
+// multiple of 4 elements, or the planes do not fit). For bf16 planes the direction-serial kernel
+// measured faster (56 x 56 classifier maps: 1.39 ms against 1.46 ms per forward): half-size
+// planes let it keep four CTAs per SM where this kernel's fp32 h buffers allow two.
 int cd_ring_depth(const Problem& P) {
-    if (P.per_dir || P.W % (P.dtype == GSPN_F32 ? 4 : 8) != 0) return 0;   // rows of whole 16-byte chunks
+    if (P.dtype != GSPN_F32 || P.per_dir || P.W % 4 != 0) return 0;   // fp32 rows of whole 16-byte chunks
     const int lpt = plane_lanes(P);
     if (cd_smem(P, 3, lpt) <= kPlaneSmemBudget / 2) return 3;
     return cd_smem(P, 2, lpt) <= kPlaneSmemBudget ? 2 : 0;
@@ -963,8 +956,10 @@ cudaError_t plane_cd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t 
 // Local propagation has its own instantiations, so the global scans carry no chunk counters.
 template <typename T, int LPT>
 cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
-    if (cd_ring_depth(P) > 0)
-        return P.chunk > 0 ? plane_cd_launch3<T, LPT, true>(P, a, st) : plane_cd_launch3<T, LPT, false>(P, a, st);
+    if constexpr (sizeof(T) == 4) {
+        if (cd_ring_depth(P) > 0)
+            return P.chunk > 0 ? plane_cd_launch3<T, LPT, true>(P, a, st) : plane_cd_launch3<T, LPT, false>(P, a, st);
+    }
     if (P.per_dir)
         return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true, true>(P, a, st)
                            : plane_fwd_launch3<T, LPT, false, true>(P, a, st);

@@ -17,10 +17,9 @@ from _cases import assert_close, check_forward, f64, fwd_tol
 
 pytestmark = pytest.mark.gpu
 
-# rows of whole 16-byte chunks (W a multiple of 4 for fp32, 8 for bf16) run the concurrent-direction
-# forward (17 lines are not a whole number of 4- or 8-line strips; 1 x 8 and 3 x 8 are single-lane
-# and single-line scans; 100 x 16 and 60 x 96 use 4 lanes per thread; 36 is a whole number of
-# chunks for fp32 only); the others run the direction-serial forward
+# fp32 maps whose rows are a multiple of 4 run the concurrent-direction forward (17 lines are not a
+# whole number of 4-line strips; 1 x 8 and 3 x 8 are single-lane and single-line scans; 100 x 16
+# and 60 x 96 use 4 lanes per thread); bf16 maps and the other shapes run the direction-serial one
 SHAPES = [(1, 4, 16, 16), (2, 3, 17, 33), (1, 2, 1, 5), (1, 2, 5, 1), (2, 2, 31, 7), (1, 1, 64, 40), (1, 1, 1, 1),
           (2, 2, 56, 56), (1, 1, 128, 3), (3, 1, 33, 128), (2, 3, 17, 40), (2, 3, 17, 36), (1, 2, 1, 8),
           (1, 1, 3, 8), (1, 2, 100, 16), (2, 1, 60, 96)]
