@@ -285,16 +285,18 @@ __global__ void __launch_bounds__(kPlaneThreads) k_plane_fwd(PlaneArgs p) {
 }
 
 // ====================================================== forward, directions scanned concurrently
-// fp32 storage. One CTA per plane (persistent over planes), one warp per direction: after z = lambda x is in
-// shared memory, the D directions of the mask are scanned at the same time, each warp writing
-// its h^d to a plane buffer of its own; y = u * (h^TB + h^BT + h^LR + h^RL) is then summed in
-// that fixed order, so the result does not depend on warp timing. Each scanning warp streams
-// its three logit planes through a ring of NSL strips of K = 16 / sizeof(T) scan lines filled
-// with 16-byte cp.async copies that bypass L1, so the logits are read from HBM exactly once and
-// the transposed walks of the horizontal directions read one 16-byte run per lane and strip;
-// the weights of a whole strip are formed before its K recurrence steps, off the
-// h chain. Lane j of a scan line is held by thread j % 32 as its element j / 32 (interleaved),
-// which keeps every row and column walk of the odd-stride planes conflict-free.
+// fp32 storage. The four line scans of a plane are independent given z = lambda x and are only
+// added at the end ("GSPN-2: Efficient Parallel Sequence Modeling" paper notes, section "2D
+// spatial propagation review": one scan per direction, then the merge), so they run at the same
+// time here: one CTA per plane (persistent over planes), one warp per direction, each warp
+// writing its h^d to a plane buffer of its own; y = u * (h^TB + h^BT + h^LR + h^RL) is then
+// summed in that fixed order, so the result does not depend on warp timing. Each scanning warp
+// streams its three logit planes through a ring of NSL strips of K = 16 / sizeof(T) scan lines
+// filled with 16-byte cp.async copies that bypass L1: the logits are read from HBM exactly once,
+// and the transposed walks of the horizontal directions read one 16-byte run per lane and
+// strip. The weights of a whole strip are formed before its K recurrence steps, off the h chain.
+// Lane j of a scan line is held by thread j % 32 as its element j / 32 (interleaved), which keeps
+// every row and column walk of the odd-stride planes conflict-free.
 
 __device__ __forceinline__ uint32_t cd_saddr(const void* ptr) { return (uint32_t)__cvta_generic_to_shared(ptr); }
 __device__ __forceinline__ void cd_cp16(void* dst, const void* src) {
