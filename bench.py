@@ -43,7 +43,11 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="libgspn", choices=["libgspn", "reference"])
-    ap.add_argument("--workload", default="highres", choices=sorted(gspn_inputs.WORKLOADS))
+    ap.add_argument("--workload", default="highres", choices=sorted(gspn_inputs.WORKLOADS) + ["all"],
+                    help="'all': one line per workload, in the order tiny, classifier, highres, wide, train")
+    ap.add_argument("--shard", action="store_true",
+                    help="strong scaling: split the workload's planes over the ranks (batch blocks, else channel "
+                         "blocks) instead of giving every rank the whole workload")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-planes", type=int, default=24, help="planes of the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -77,7 +81,8 @@ def config_of(wl, world, chunk=0):
         "per_rank_batch": wl.N,
         "global_batch": wl.N * world,
         "parallelism": f"dp{world}" if world > 1 else "single",
-        "l2": "inputs larger than L2 (no flush)",
+        "l2": ("inputs larger than L2 (no flush)" if wl.compulsory_fwd_bytes() > 126 * 2 ** 20
+               else "inputs fit in L2: a parity-size case, not a bandwidth figure"),
         "chunk": chunk,
     }
 
@@ -103,11 +108,30 @@ def plane_bytes(wl):
     return (4 * wl.H * wl.W + (wl.D * 3 * wl.H * wl.W) // (wl.C if wl.wmode else 1)) * wl.elem_bytes
 
 
+def host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count(), model
+
+
 def run_reference(args):
     rank, _, world = env_rank()
-    wl = gspn_inputs.WORKLOADS[args.workload]
     if rank != 0:
         return
+    names = ["tiny", "classifier", "highres", "wide", "train"] if args.workload == "all" else [args.workload]
+    for name in names:
+        reference_line(args, gspn_inputs.WORKLOADS[name], world)
+
+
+def reference_line(args, wl, world):
     planes_per_step = 2
     times = []
     for s in range(args.warmup + args.steps):
@@ -117,17 +141,20 @@ def run_reference(args):
     tot = sum(times)
     nbytes = plane_bytes(wl) * planes_per_step * len(times)
     value = nbytes / tot / 1e9
-    ms_per_step = tot / len(times) * 1e3 * (wl.N * wl.C) / planes_per_step
+    ms_per_step = tot / len(times) * 1e3
+    nproc, model = host_cpu()
     line = {
         "impl": "reference",
         "metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "ms_per_full_forward_extrapolated": round(ms_per_step * (wl.N * wl.C) / planes_per_step, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": config_of(wl, world, args.chunk),
-        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{planes_per_step} of {wl.N * wl.C} planes per step, float64 C oracle, "
-                                   "one thread; ms_per_step extrapolated to the full batch"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "host_nproc": nproc,
+                         "cpu_model": model, "kind": "oracle",
+                         "sample": f"{planes_per_step} of {wl.N * wl.C} (n,c) planes per step (ms_per_step is "
+                                   "the measured time of that sample), float64 C oracle, one thread"},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -226,18 +253,55 @@ def committed_traffic(workload):
 def run_libgspn(args):
     import torch
     import torch.distributed as dist
-    import linear_spatial_propagation_gspn_b200 as g
 
     rank, local_rank, world = env_rank()
     torch.cuda.set_device(local_rank)
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
-    wl = gspn_inputs.WORKLOADS[args.workload]
+    names = ["tiny", "classifier", "highres", "wide", "train"] if args.workload == "all" else [args.workload]
+    for name in names:
+        line = bench_workload(args, name, rank, local_rank, world)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        torch.cuda.empty_cache()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _max_over_ranks(v, world, dev):
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return v
+    tt = torch.tensor([v], device=dev, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def bench_workload(args, name, rank, local_rank, world):
+    import torch
+    import torch.distributed as dist
+    import linear_spatial_propagation_gspn_b200 as g
+    from linear_spatial_propagation_gspn_b200 import sharding
+
+    wl = gspn_inputs.WORKLOADS[name]
     if args.batch:
         wl = wl.with_(N=args.batch)
     dev = torch.device("cuda", local_rank)
-    t = gspn_inputs.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
+    full_wl = wl
+    shard = None
+    if args.shard:
+        # strong scaling: every rank draws the same full inputs and keeps its plane shard
+        t = gspn_inputs.make_inputs(wl, device=dev)
+        shard = sharding.plan(wl.N, wl.C, world, rank)
+        shared = wl.wmode == 1
+        t = {k: (sharding.take(v, shard, logits=(k == "a"), shared=shared).contiguous()) for k, v in t.items()}
+        wl = wl.with_(N=t["x"].shape[0], C=t["x"].shape[1])
+        torch.cuda.empty_cache()
+    else:
+        t = gspn_inputs.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
     x, a, lam, u = t["x"], t["a"], t["lam"], t["u"]
     desc = g.desc_for(x, wl.wmode, wl.mask, chunk=args.chunk)
     algo = g.selected_algo(desc)
@@ -248,60 +312,57 @@ def run_libgspn(args):
     def step():
         g.forward(x, a, lam, u, wl.wmode, wl.mask, y=y, ws=ws, chunk=args.chunk)
 
-    for _ in range(args.warmup):
+    for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
     if g.device_status(ws) != g.GSPN_OK:
         raise RuntimeError("device status reports a timeout during warm-up")
 
-    # ---- timed region: K steps, events on the launching stream
+    # ---- timed region: K steps, one event per step boundary on the launching stream
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for k in range(args.steps):
         step()
-    e1.record(stream)
+        evs[k + 1].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms_total = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = _max_over_ranks(evs[0].elapsed_time(evs[-1]), world, dev)
+    per_step = [evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps)]
+    ms_median = _max_over_ranks(statistics.median(per_step), world, dev)
     ms_step = ms_total / args.steps
     comp = wl.compulsory_fwd_bytes()
-    value = comp * world / (ms_step * 1e-3) / 1e9
+    job_bytes = full_wl.compulsory_fwd_bytes() if args.shard else comp * world
+    job_elems = full_wl.numel if args.shard else wl.numel * world
+    value = job_bytes / (ms_step * 1e-3) / 1e9
 
     # ---- per-kernel timing pass (events recorded by the library around each launch)
     nk = 8
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]
-    for e in evs:
+    kevs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]
+    for e in kevs:
         e.record(stream)  # materialise the event handles
     torch.cuda.synchronize()
     reps = max(5, min(50, args.steps // 4))
     per = None
     launches = 0
     for _ in range(reps):
-        launches = g.forward_timed(x, a, lam, u, y, ws, desc, evs)
+        launches = g.forward_timed(x, a, lam, u, y, ws, desc, kevs)
         torch.cuda.synchronize()
-        d = [evs[2 * k].elapsed_time(evs[2 * k + 1]) for k in range(launches)]
+        d = [kevs[2 * k].elapsed_time(kevs[2 * k + 1]) for k in range(launches)]
         per = d if per is None else [p + q for p, q in zip(per, d)]
     per = [p / reps for p in per]
     peak, peak_kind = measured_peak()
     kern_ms = sum(per)
-    names = [n for n, bit in zip(("TB", "BT", "LR", "RL"), (1, 2, 4, 8)) if wl.mask & bit]
-    if launches == len(names) + 1:
-        names = ["weights"] + names
+    names = launch_names(wl, algo, launches)
     achieved = comp / (kern_ms * 1e-3) / 1e9
-    traffic, per_launch = committed_traffic(wl.name) if not args.batch else (None, None)
+    traffic, per_launch = committed_traffic(wl.name) if not (args.batch or args.shard) else (None, None)
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -314,7 +375,7 @@ def run_libgspn(args):
         # DRAM bytes each launch moves (ncu) over its event-timed duration
         roofline["kernels_dram_gbs"] = {n: round(b / (p * 1e-3) / 1e9, 1) for n, b, p in zip(names, per_launch, per)}
 
-    # ---- backward (A7): gradients of sum(dy * y), timed on its own over the same number of steps
+    # ---- backward (A7): gradients of sum(dy * y), timed on its own
     bwd = None
     if args.backward or wl.name == "train":
         dy = torch.randn(x.shape, generator=torch.Generator(device=dev).manual_seed(wl.seed + 7), device=dev,
@@ -333,22 +394,21 @@ def run_libgspn(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        b0 = torch.cuda.Event(enable_timing=True)
-        b1 = torch.cuda.Event(enable_timing=True)
-        b0.record(stream)
-        for _ in range(nb_steps):
+        bev = [torch.cuda.Event(enable_timing=True) for _ in range(nb_steps + 1)]
+        bev[0].record(stream)
+        for k in range(nb_steps):
             bstep()
-        b1.record(stream)
+            bev[k + 1].record(stream)
         torch.cuda.synchronize()
-        bms = b0.elapsed_time(b1) / nb_steps
-        if world > 1:
-            tt = torch.tensor([bms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            bms = float(tt.item())
+        bms = _max_over_ranks(bev[0].elapsed_time(bev[-1]) / nb_steps, world, dev)
+        bmed = _max_over_ranks(statistics.median(bev[k].elapsed_time(bev[k + 1]) for k in range(nb_steps)),
+                               world, dev)
         bcomp = wl.compulsory_bwd_bytes()
-        bgbs = bcomp * world / (bms * 1e-3) / 1e9
-        bwd = {"ms_per_step": round(bms, 4), "steps": nb_steps, "compulsory_bytes": bcomp,
-               "value": round(bgbs, 2), "unit": "GB/s", "frac": round(bgbs / world / peak, 4),
+        bjob = full_wl.compulsory_bwd_bytes() if args.shard else bcomp * world
+        bgbs = bjob / (bms * 1e-3) / 1e9
+        bwd = {"ms_per_step": round(bms, 4), "ms_median": round(bmed, 4), "steps": nb_steps,
+               "compulsory_bytes": bcomp, "value": round(bgbs, 2), "unit": "GB/s",
+               "frac": round(bcomp / (bms * 1e-3) / 1e9 / peak, 4),
                "algo": g.ALGO_NAMES.get(g.selected_algo(bdesc, True), "?"),
                "what": "reads dy, x, lambda, u, logits; writes dx, dlambda, du, dlogits (compulsory bytes)",
                "train_step_ms": round(ms_step + bms, 4)}
@@ -387,47 +447,56 @@ def run_libgspn(args):
             g.forward_host(desc, hx, ha, hl, hu, hy, dev_buf)
         q1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = q0.elapsed_time(q1) / args.e2e_steps
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = _max_over_ranks(q0.elapsed_time(q1) / args.e2e_steps, world, dev)
         h2d = sum(tt.numel() * tt.element_size() for tt in (hx, ha, hl, hu))
         d2h = hy.numel() * hy.element_size()
-        e2e = {"value": round(comp * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+        e2e = {"value": round(job_bytes / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "gspn_forward_host (pinned host buffers)"}
-        del dev_buf
+        del dev_buf, hx, ha, hl, hu, hy
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs = oracle_plane_seconds_only(wl, args.cpu_planes, args.chunk)
-        cpu = {"value": round(plane_bytes(wl) * args.cpu_planes / secs / 1e9, 6), "unit": "GB/s", "cores": 1,
-               "kind": "oracle",
-               "sample": f"{args.cpu_planes} of {wl.N * wl.C} (n,c) planes, float64 C oracle, one thread, "
+        planes = min(args.cpu_planes, wl.N * wl.C)
+        secs = oracle_plane_seconds_only(wl, planes, args.chunk)
+        nproc, model = host_cpu()
+        cpu = {"value": round(plane_bytes(wl) * planes / secs / 1e9, 6), "unit": "GB/s", "cores": 1,
+               "host_nproc": nproc, "cpu_model": model, "kind": "oracle",
+               "output_elements_per_s": round(planes * wl.H * wl.W / secs, 1),
+               "sample": f"{planes} of {wl.N * wl.C} (n,c) planes, float64 C oracle, one thread, "
                          f"{secs:.1f} s"}
 
+    del t, x, a, lam, u, y, ws
     if world > 1:
         dist.barrier()
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": dtype_name(wl), "data": "synthetic (seeded torch.randn/rand on device)",
-            "config": config_of(wl, world, args.chunk),
-            "algo": g.ALGO_NAMES.get(algo, str(algo)),
-            "roofline": roofline,
-            "copy_ceiling_gbs": round(copy_gbs, 1),
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "backward": bwd,
-            "gpu_launches": launches * args.steps,
-            "clocks": clocks,
-        }
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
+        "ms_median": round(ms_median, 4),
+        "output_elements_per_s": round(job_elems / (ms_step * 1e-3), 1),
+        "higher_is_better": True, "scaling": "strong" if args.shard else "weak", "vs_baseline": None,
+        "dtype": dtype_name(wl), "data": "synthetic (seeded torch.randn/rand on device)",
+        "config": dict(config_of(full_wl, 1 if args.shard else world, args.chunk),
+                       **({"shard": f"{shard.axis}[{shard.start}:{shard.stop}] on rank 0",
+                           "parallelism": f"{shard.axis.lower()}-shard{world}"} if args.shard else {})),
+        "algo": g.ALGO_NAMES.get(algo, str(algo)),
+        "roofline": roofline,
+        "copy_ceiling_gbs": round(copy_gbs, 1),
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "backward": bwd,
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks,
+    }
+
+
+def launch_names(wl, algo, launches):
+    dirs = [n for n, bit in zip(("TB", "BT", "LR", "RL"), (1, 2, 4, 8)) if wl.mask & bit]
+    if launches == len(dirs) + 1:
+        return ["weights"] + dirs
+    if launches == 1:
+        return ["plane" if algo == 2 else "forward"]
+    return [f"launch{k}" for k in range(launches)]
 
 
 def run_proxy(args):
@@ -506,6 +575,8 @@ def run_proxy(args):
 
 def main():
     args = parse_args()
+    if args.proxy and args.workload == "all":
+        raise SystemExit("--proxy runs one named workload")
     if args.impl == "reference":
         run_reference(args)
     elif args.proxy:

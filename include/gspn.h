@@ -151,7 +151,9 @@ GSPN_API size_t gspn_forward_host_buffer_size(const gspn_desc *desc);
 
 /* End-to-end forward from HOST buffers: copies x, a, lam, u from host memory (pinned memory
  * gives asynchronous copies) into the caller's device buffer `dev`, runs gspn_forward there,
- * copies y back to host memory `hy` and synchronises `stream`. Returns the first error. */
+ * copies y back to host memory `hy` and synchronises `stream`. Returns the first error; once a
+ * copy has been queued it synchronises `stream` before returning on every path, so the host
+ * buffers may be reused as soon as the call returns. */
 GSPN_API gspn_status gspn_forward_host(const gspn_desc *desc, const void *hx, const void *ha,
                               const void *hlam, const void *hu, void *hy, void *dev,
                               size_t dev_bytes, void *stream);
@@ -193,10 +195,12 @@ GSPN_API gspn_status gspn_proxy_forward(const gspn_desc *desc, int c_full, const
  * exists for callers that cannot allocate device memory at call time, e.g. code running under
  * another component's allocator or on a path where cudaMalloc/cudaFree would synchronise the
  * device). x, a, lam, u, y are device pointers on the current device; `stream` belongs to it.
- *   - Returns GSPN_ERR_WORKSPACE, before touching the device, if the descriptor needs more
- *     workspace than GSPN_NOALLOC_SCRATCH_BYTES (gspn_workspace_size(desc, 0) tells).
- *   - The first call on each device looks up the array's device address (once per device,
- *     with that device current); make that first call before any stream capture.
+ *   - Returns GSPN_ERR_INVALID_ARG for a malformed descriptor or a null pointer,
+ *     GSPN_ERR_UNSUPPORTED for a well-formed one no kernel family runs, and GSPN_ERR_WORKSPACE,
+ *     before touching the device, if the descriptor needs more workspace than
+ *     GSPN_NOALLOC_SCRATCH_BYTES (gspn_workspace_size(desc, 0) tells).
+ *   - Every call looks up the array's device address on the current device (a host-side query
+ *     that allocates nothing), so the address stays right across a cudaDeviceReset.
  *   - Every call on a device shares the one array, which keeps the last call's contents (each
  *     call rewrites what it reads): calls that overlap on the GPU, from any stream or thread,
  *     race on it. Serialise them.

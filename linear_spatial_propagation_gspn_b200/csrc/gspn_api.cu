@@ -95,6 +95,11 @@ thread_local Hooks g_hooks;
 
 }  // namespace
 
+bool desc_valid(const gspn_desc* d) {
+    Problem p;
+    return make_problem(d, &p);
+}
+
 void launch_begin(cudaStream_t st) {
     if (g_hooks.on && 2 * g_hooks.launches + 1 < g_hooks.n_ev) cudaEventRecord(g_hooks.ev[2 * g_hooks.launches], st);
 }
@@ -254,13 +259,19 @@ gspn_status gspn_forward_host(const gspn_desc* desc, const void* hx, const void*
     char* dws = da + align256(ab);
     const size_t wsb = dev_bytes - (size_t)(dws - base);
     cudaStream_t st = (cudaStream_t)stream;
-    if (cudaMemcpyAsync(dx, hx, ub, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(da, ha, ab, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(dlam, hlam, lb, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (cudaMemcpyAsync(du, hu, lb, cudaMemcpyHostToDevice, st) != cudaSuccess) return GSPN_ERR_CUDA;
+    // Once a copy is queued, every return waits for the stream first: the caller may free or
+    // reuse its host buffers as soon as this call returns, error or not.
+    auto fail = [&](gspn_status s) {
+        cudaStreamSynchronize(st);
+        return s;
+    };
+    if (cudaMemcpyAsync(dx, hx, ub, cudaMemcpyHostToDevice, st) != cudaSuccess) return fail(GSPN_ERR_CUDA);
+    if (cudaMemcpyAsync(da, ha, ab, cudaMemcpyHostToDevice, st) != cudaSuccess) return fail(GSPN_ERR_CUDA);
+    if (cudaMemcpyAsync(dlam, hlam, lb, cudaMemcpyHostToDevice, st) != cudaSuccess) return fail(GSPN_ERR_CUDA);
+    if (cudaMemcpyAsync(du, hu, lb, cudaMemcpyHostToDevice, st) != cudaSuccess) return fail(GSPN_ERR_CUDA);
     gspn_status s = gspn_forward(desc, dx, da, dlam, du, dyo, dws, wsb, stream);
-    if (s != GSPN_OK) return s;
-    if (cudaMemcpyAsync(hy, dyo, ub, cudaMemcpyDeviceToHost, st) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (s != GSPN_OK) return fail(s);
+    if (cudaMemcpyAsync(hy, dyo, ub, cudaMemcpyDeviceToHost, st) != cudaSuccess) return fail(GSPN_ERR_CUDA);
     if (cudaStreamSynchronize(st) != cudaSuccess) return GSPN_ERR_CUDA;
     return GSPN_OK;
 }

@@ -73,6 +73,9 @@ void launch_begin(cudaStream_t st);
 void launch_end(cudaStream_t st);
 
 // ---- misc ------------------------------------------------------------------------------
+// True when the descriptor is well formed (the checks gspn_forward reports as
+// GSPN_ERR_INVALID_ARG); says nothing about whether a kernel family supports it.
+bool desc_valid(const gspn_desc* d);
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_wait_probe(unsigned* status, const unsigned* flag, unsigned long long limit_ns,
                               cudaStream_t st);

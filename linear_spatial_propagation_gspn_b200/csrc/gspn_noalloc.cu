@@ -11,35 +11,23 @@
 //
 // The array is a file-scope __device__ variable: every GPU that loads this library holds
 // GSPN_NOALLOC_SCRATCH_BYTES of it until the process exits. In host code its name is only a
-// host-side stand-in, so the device address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) and handed to the kernels.
-#include <mutex>
-
+// host-side stand-in, so every call looks up the device address with cudaGetSymbolAddress (with
+// the target device current) and hands that to the kernels. The lookup is a host-side query that
+// allocates nothing; doing it per call (instead of caching it) keeps the address right even after
+// a cudaDeviceReset has reloaded the module at another address.
 #include "gspn.h"
 #include "gspn_internal.h"
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GSPN_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device; resolved on first use per device.
+// Device address of g_noalloc_scratch on the current device.
 gspn_status scratch_for_current_device(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return GSPN_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || p == nullptr) return GSPN_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return GSPN_ERR_CUDA;
+    *out = p;
     return GSPN_OK;
 }
 
@@ -47,10 +35,13 @@ gspn_status scratch_for_current_device(void** out) {
 
 extern "C" gspn_status gspn_forward_noalloc(const gspn_desc* desc, const void* x, const void* a, const void* lam,
                                             const void* u, void* y, void* stream) {
-    // Size check first: nothing touches the device for a problem that does not fit.
+    // Descriptor first (malformed: GSPN_ERR_INVALID_ARG, as gspn_forward reports it), then the
+    // size check: nothing touches the device for a problem that does not fit.
+    if (!gspn::desc_valid(desc)) return GSPN_ERR_INVALID_ARG;
     const size_t need = gspn_workspace_size(desc, 0);
-    if (need == 0) return desc ? GSPN_ERR_UNSUPPORTED : GSPN_ERR_INVALID_ARG;
+    if (need == 0) return GSPN_ERR_UNSUPPORTED;
     if (need > (size_t)GSPN_NOALLOC_SCRATCH_BYTES) return GSPN_ERR_WORKSPACE;
+    if (!x || !a || !lam || !u || !y) return GSPN_ERR_INVALID_ARG;
     void* scratch = nullptr;
     const gspn_status s = scratch_for_current_device(&scratch);
     if (s != GSPN_OK) return s;

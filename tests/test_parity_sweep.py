@@ -79,7 +79,7 @@ def test_full_size_sampled_planes(name):
     y2 = g.forward(t["x"], t["a"], t["lam"], t["u"], wl.wmode, wl.mask)
     torch.cuda.synchronize()
     assert torch.equal(y, y2), "two runs differ"
-    for (n, c) in _sample_planes(wl, 3, 123):
+    for (n, c) in _sample_planes(wl, 8, 123):
         cw = 0 if wl.wmode else c
         ref = oracle.forward(f64(t["x"][n:n + 1, c:c + 1]), f64(t["a"][:, n:n + 1, cw:cw + 1]),
                              f64(t["lam"][n:n + 1, c:c + 1]), f64(t["u"][n:n + 1, c:c + 1]), wl.wmode, wl.mask)
