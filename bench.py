@@ -58,6 +58,8 @@ def parse_args():
                     help="compressive channel proxy: project C channels to this many, propagate, project back")
     ap.add_argument("--chunk", type=int, default=0,
                     help="local propagation: lines per chunk along each scan axis (0 = global, the metric's)")
+    ap.add_argument("--algo", default="auto", choices=["auto", "generic", "plane", "sweep", "band"],
+                    help="kernel family (auto: the library's choice)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch N (small cases for profiler captures; not a bench line)")
     return ap.parse_args()
@@ -303,14 +305,16 @@ def bench_workload(args, name, rank, local_rank, world):
     else:
         t = gspn_inputs.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
     x, a, lam, u = t["x"], t["a"], t["lam"], t["u"]
-    desc = g.desc_for(x, wl.wmode, wl.mask, chunk=args.chunk)
+    algo_req = {"auto": g.ALGO_AUTO, "generic": g.ALGO_GENERIC, "plane": g.ALGO_PLANE, "sweep": g.ALGO_SWEEP,
+                "band": g.ALGO_BAND}[args.algo]
+    desc = g.desc_for(x, wl.wmode, wl.mask, algo=algo_req, chunk=args.chunk)
     algo = g.selected_algo(desc)
     ws = g.alloc_workspace(desc, False, dev)
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
 
     def step():
-        g.forward(x, a, lam, u, wl.wmode, wl.mask, y=y, ws=ws, chunk=args.chunk)
+        g.forward(x, a, lam, u, wl.wmode, wl.mask, algo=algo_req, y=y, ws=ws, chunk=args.chunk)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -491,6 +495,8 @@ def bench_workload(args, name, rank, local_rank, world):
 
 
 def launch_names(wl, algo, launches):
+    if algo == 4:   # band family
+        return ["weights", "TB-ckpt+z", "LR-ckpt", "BT+TB-recompute", "RL+LR-recompute"][:launches]
     dirs = [n for n, bit in zip(("TB", "BT", "LR", "RL"), (1, 2, 4, 8)) if wl.mask & bit]
     if launches == len(dirs) + 1:
         return ["weights"] + dirs

@@ -85,8 +85,12 @@ enum { GSPN_DIR_TB = 1, GSPN_DIR_BT = 2, GSPN_DIR_LR = 4, GSPN_DIR_RL = 8, GSPN_
  *   GENERIC: any shape; one CTA per plane and direction, hidden line in shared memory.
  *   PLANE:   small maps; the whole plane stays on chip and all directions run in one pass.
  *   SWEEP:   large maps (forward): persistent line sweeps fed by per-thread asynchronous copies,
- *            one launch per direction plus one for the weights. */
-enum { GSPN_ALGO_AUTO = 0, GSPN_ALGO_GENERIC = 1, GSPN_ALGO_PLANE = 2, GSPN_ALGO_SWEEP = 3 };
+ *            one launch per direction plus one for the weights.
+ *   BAND:    1024 x 1024 maps, all four directions, forward only, never chosen by AUTO: the
+ *            ascending scans keep a checkpoint of their line every 8 lines and the descending
+ *            scans recompute them band by band, so partial sums never cross HBM between the two
+ *            scans of a pair (fewer DRAM bytes than SWEEP, but more rows streamed per SM). */
+enum { GSPN_ALGO_AUTO = 0, GSPN_ALGO_GENERIC = 1, GSPN_ALGO_PLANE = 2, GSPN_ALGO_SWEEP = 3, GSPN_ALGO_BAND = 4 };
 
 /* chunk: 0 = global propagation over the whole map. K > 0 = local propagation: the map is cut
  * along each direction's scan axis into chunks of K lines aligned to image line 0 (rows for

@@ -30,8 +30,8 @@ GSPN_ERR_WORKSPACE, GSPN_ERR_CUDA, GSPN_ERR_DEVICE_TIMEOUT = 4, 5, 6
 F32, BF16 = 0, 1
 PER_CHANNEL, SHARED = 0, 1
 DIR_TB, DIR_BT, DIR_LR, DIR_RL, DIR_ALL = 1, 2, 4, 8, 15
-ALGO_AUTO, ALGO_GENERIC, ALGO_PLANE, ALGO_SWEEP = 0, 1, 2, 3
-ALGO_NAMES = {ALGO_GENERIC: "generic", ALGO_PLANE: "plane", ALGO_SWEEP: "sweep"}
+ALGO_AUTO, ALGO_GENERIC, ALGO_PLANE, ALGO_SWEEP, ALGO_BAND = 0, 1, 2, 3, 4
+ALGO_NAMES = {ALGO_GENERIC: "generic", ALGO_PLANE: "plane", ALGO_SWEEP: "sweep", ALGO_BAND: "band"}
 
 
 class GspnDesc(ctypes.Structure):

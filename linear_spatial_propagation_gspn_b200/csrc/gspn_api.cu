@@ -18,7 +18,7 @@ bool make_problem(const gspn_desc* d, Problem* p) {
     if (d->wmode != GSPN_W_PER_CHANNEL && d->wmode != GSPN_W_SHARED) return false;
     if (d->dir_mask < 1u || d->dir_mask > 15u) return false;
     if (d->dtype != GSPN_F32 && d->dtype != GSPN_BF16) return false;
-    if (d->algo < GSPN_ALGO_AUTO || d->algo > GSPN_ALGO_SWEEP) return false;
+    if (d->algo < GSPN_ALGO_AUTO || d->algo > GSPN_ALGO_BAND) return false;
     if (d->chunk < 0) return false;
     if (d->per_dir != 0 && d->per_dir != 1) return false;
     if ((long long)d->N * d->C > 0x7fffffffLL) return false;
@@ -45,6 +45,7 @@ int select_algo(const gspn_desc* d, const Problem& p, bool bwd) {
     case GSPN_ALGO_GENERIC: return generic_supports(p, bwd) ? GSPN_ALGO_GENERIC : -1;
     case GSPN_ALGO_PLANE: return plane_supports(p, bwd) ? GSPN_ALGO_PLANE : -1;
     case GSPN_ALGO_SWEEP: return sweep_supports(p, bwd) ? GSPN_ALGO_SWEEP : -1;
+    case GSPN_ALGO_BAND: return (!bwd && band_supports(p)) ? GSPN_ALGO_BAND : -1;
     default:
         if (plane_supports(p, bwd)) return GSPN_ALGO_PLANE;
         if (!p.per_dir && sweep_supports(p, bwd)) return GSPN_ALGO_SWEEP;
@@ -58,6 +59,7 @@ size_t ws_for(int algo, const Problem& p, bool bwd) {
     case GSPN_ALGO_GENERIC: return generic_ws_bytes(p, bwd);
     case GSPN_ALGO_PLANE: return plane_ws_bytes(p, bwd);
     case GSPN_ALGO_SWEEP: return sweep_ws_bytes(p, bwd);
+    case GSPN_ALGO_BAND: return bwd ? 0 : band_ws_bytes(p);
     default: return 0;
     }
 }
@@ -189,6 +191,7 @@ gspn_status gspn_forward(const gspn_desc* desc, const void* x, const void* a, co
     switch (algo) {
     case GSPN_ALGO_PLANE: e = plane_forward(p, x, a, lam, u, y, ws, st); break;
     case GSPN_ALGO_SWEEP: e = sweep_forward(p, x, a, lam, u, y, ws, st); break;
+    case GSPN_ALGO_BAND: e = band_forward(p, x, a, lam, u, y, ws, st); break;
     default: e = generic_forward(p, x, a, lam, u, y, ws, st); break;
     }
     return to_status(e);

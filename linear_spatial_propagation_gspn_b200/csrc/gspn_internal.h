@@ -66,6 +66,17 @@ cudaError_t sweep_backward(const Problem& p, const void* x, const void* a, const
                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws,
                            cudaStream_t st);
 
+// Weight table of the line sweeps: for every direction slot and (n, cw) plane, the outer weights
+// (w0, w2) of each normalised tridiagonal row, in TableT of the storage dtype (fp32, or fp16 for
+// bf16 storage). Slots from tslot0 on are written transposed ([W][H] per plane).
+cudaError_t launch_weight_table(const Problem& P, const void* a, void* table, int tslot0, cudaStream_t st);
+
+// ---- band family (large square maps): checkpointed scans with band recompute ----------------
+bool band_supports(const Problem& p);
+size_t band_ws_bytes(const Problem& p);
+cudaError_t band_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u, void* y,
+                         void* ws, cudaStream_t st);
+
 // ---- per-launch timing hooks (gspn_forward_timed) ---------------------------------------
 // Kernel families call launch_begin / launch_end around every kernel launch. When a timed
 // call is active on this host thread they record the caller's events on the launch stream.
