@@ -183,9 +183,10 @@ GSPN_API gspn_status gspn_copy_ceiling(const void *src, void *dst, size_t bytes,
  * per pixel, with P_in a C_proxy x C and P_out a C x C_proxy matrix (row-major, storage dtype).
  * `desc` describes the proxy-space propagation: desc->C = C_proxy, and the logits a, lam and u
  * are in proxy space (shapes as for gspn_forward with C = C_proxy). x and y: N x c_full x H x W.
- * The projections are strided batched GEMMs on the tensor cores (cuBLAS; bf16 storage: bf16
- * operands with fp32 accumulation; fp32 storage: exact fp32), xp and yp live in the workspace in
- * the storage dtype. All pointers are device pointers. */
+ * The projections are the library's own GEMM kernels: for bf16 storage with C and C_proxy
+ * multiples of 8 and H*W a multiple of 8, tcgen05 tensor-core MMAs on TMA-loaded tiles (bf16
+ * operands, fp32 accumulation); otherwise an exact fp32 GEMM on the CUDA cores. xp and yp live in
+ * the workspace in the storage dtype. All pointers are device pointers. */
 GSPN_API size_t gspn_proxy_workspace_size(const gspn_desc *desc, int c_full);
 GSPN_API gspn_status gspn_proxy_forward(const gspn_desc *desc, int c_full, const void *x, const void *p_in,
                                const void *a, const void *lam, const void *u, const void *p_out,

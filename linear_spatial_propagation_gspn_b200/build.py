@@ -53,10 +53,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         if p.wait() != 0:
             raise RuntimeError(f"nvcc failed on {src}")
     tmp = LIB + f".tmp{os.getpid()}"
-    # cuBLAS for the channel-proxy projections (plain GEMMs); rpath to the toolkit's copy
-    cuda_lib = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64")
-    subprocess.check_call([nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
-                           "-L", cuda_lib, "-lcublas", "-Xlinker", f"-rpath={cuda_lib}"])
+    subprocess.check_call([nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 

@@ -177,6 +177,13 @@ int gspn_selected_algo(const gspn_desc* desc, int for_backward) {
 
 gspn_status gspn_forward(const gspn_desc* desc, const void* x, const void* a, const void* lam, const void* u, void* y,
                          void* ws, size_t ws_bytes, void* stream) {
+    return gspn::forward_internal(desc, x, a, lam, u, y, ws, ws_bytes, stream, true);
+}
+
+}  // extern "C"
+
+gspn_status gspn::forward_internal(const gspn_desc* desc, const void* x, const void* a, const void* lam, const void* u,
+                                   void* y, void* ws, size_t ws_bytes, void* stream, bool clear_status) {
     Problem p;
     if (!make_problem(desc, &p)) return GSPN_ERR_INVALID_ARG;
     if (!x || !a || !lam || !u || !y || !ws) return GSPN_ERR_INVALID_ARG;
@@ -186,7 +193,7 @@ gspn_status gspn_forward(const gspn_desc* desc, const void* x, const void* a, co
     if (algo < 0) return GSPN_ERR_UNSUPPORTED;
     if (ws_bytes < ws_for(algo, p, false)) return GSPN_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(unsigned), st);
+    cudaError_t e = clear_status ? cudaMemsetAsync(ws, 0, sizeof(unsigned), st) : cudaSuccess;
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
     switch (algo) {
     case GSPN_ALGO_PLANE: e = plane_forward(p, x, a, lam, u, y, ws, st); break;
@@ -196,6 +203,8 @@ gspn_status gspn_forward(const gspn_desc* desc, const void* x, const void* a, co
     }
     return to_status(e);
 }
+
+extern "C" {
 
 gspn_status gspn_forward_timed(const gspn_desc* desc, const void* x, const void* a, const void* lam, const void* u,
                                void* y, void* ws, size_t ws_bytes, void* stream, void* const* events, int n_events,

@@ -77,6 +77,18 @@ size_t band_ws_bytes(const Problem& p);
 cudaError_t band_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u, void* y,
                          void* ws, cudaStream_t st);
 
+// gspn_forward with the option of keeping the device status word (callers that launched their own
+// kernels on the same workspace first clear it themselves).
+gspn_status forward_internal(const gspn_desc* desc, const void* x, const void* a, const void* lam, const void* u,
+                             void* y, void* ws, size_t ws_bytes, void* stream, bool clear_status);
+
+// ---- channel projections of the compressive proxy (k_proj.cu) -----------------------------
+// Y[n] (Mo x HW) = P (Mo x K) . X[n] (K x HW) for n < batch, row-major, storage dtype: a tcgen05
+// GEMM for bf16 with 16-byte rows (K and HW multiples of 8), an exact fp32 SIMT GEMM otherwise.
+bool proj_uses_tc(int dtype, int Mo, int K, long long HW);
+cudaError_t launch_projection(int dtype, int Mo, int K, long long HW, int batch, const void* P, const void* X, void* Y,
+                              unsigned* status, cudaStream_t st);
+
 // ---- per-launch timing hooks (gspn_forward_timed) ---------------------------------------
 // Kernel families call launch_begin / launch_end around every kernel launch. When a timed
 // call is active on this host thread they record the caller's events on the launch stream.

@@ -56,3 +56,25 @@ def test_proxy_rejects_bad_shapes():
     x, p_in, a, lam, u, p_out = _inputs(1, 8, 2, 16, 16, 15, 1, "f32", seed=1)
     with pytest.raises(ValueError):
         g.proxy_forward(x, p_out, a, lam, u, p_in, 1, 15)
+
+
+# bf16 shapes whose projections run on the tensor cores (C, C_proxy and H*W multiples of 8):
+# several pixel tiles and a ragged last one, output-row tiles with padding (C_proxy 24 -> 32 rows,
+# 1152 -> 5 tiles of 240), contraction lengths below, at and far above one 64-wide stage, and
+# more than one batch item.
+TC_SHAPES = [(1, 24, 8, 64, 1024), (2, 64, 16, 32, 40), (1, 256, 48, 16, 72), (2, 320, 24, 8, 24),
+             (1, 1152, 144, 16, 64), (3, 136, 64, 24, 24)]
+
+
+@pytest.mark.parametrize("shape", TC_SHAPES)
+@pytest.mark.parametrize("wmode", [0, 1])
+def test_proxy_tensor_core_projections(shape, wmode):
+    N, C, Cp, H, W = shape
+    x, p_in, a, lam, u, p_out = _inputs(N, C, Cp, H, W, 15, wmode, "bf16", seed=3 * sum(shape) + wmode)
+    y = g.proxy_forward(x, p_in, a, lam, u, p_out, wmode, 15)
+    torch.cuda.synchronize()
+    ref = oracle.proxy_forward(f64(x), f64(p_in), f64(a), f64(lam), f64(u), f64(p_out), wmode, 15)
+    assert_close(f64(y), ref, fwd_tol("bf16", ref), f"proxy tensor-core {shape}")
+    y2 = g.proxy_forward(x, p_in, a, lam, u, p_out, wmode, 15)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2), "two runs differ"
