@@ -223,7 +223,7 @@ def measured_peak():
 
 # Sources of the kernels the traffic summary describes (the sweep family and its device
 # helpers); host-side entry points and the other families do not change their traffic.
-SWEEP_SOURCES = ("gspn_common.cuh", "k_sweep.cu")
+SWEEP_SOURCES = ("gspn_common.cuh", "sweep_io.cuh", "k_sweep.cu")
 
 
 def kernel_source_sha():

@@ -89,12 +89,23 @@ __global__ void k_gen_fwd(GenArgs p) {
     }
 }
 
+// Channel-shared logit gradients are sums over channels accumulated with atomics from many CTAs.
+// They are summed as 64-bit fixed-point integers (2^32 units): integer addition does not depend on
+// the order, so the result is the same on every run. A term is an fp32 value scaled by a power of
+// two (exact) and rounded to 2^-32; it is clamped to |v| <= 2^19 so that 2048 terms cannot overflow.
+constexpr float kFixScale = 4294967296.f;   // 2^32
+__device__ __forceinline__ unsigned long long to_fixed(float v) {
+    v = fminf(fmaxf(v, -524288.f), 524288.f);
+    return (unsigned long long)__float2ll_rn(v * kFixScale);
+}
+__device__ __forceinline__ float from_fixed(unsigned long long q) { return (float)(long long)q * (1.f / kFixScale); }
+
 struct GenBwdArgs {
     const void* a;
     const void* u;
     const void* dy;
     void* da;            // per-channel mode: written directly (storage dtype)
-    float* dacc;         // shared mode: fp32 sum over channels (zeroed before)
+    unsigned long long* dacc;   // shared mode: fixed-point sum over channels (zeroed before)
     float* dz;           // fp32, N*C*H*W
     const float* hstore; // h of this direction, image coordinates, fp32
     int N, C, H, W, Cw;
@@ -125,7 +136,7 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
     const long long abase = (((long long)p.slot * p.N + n) * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
     const T* a3 = (const T*)p.a + abase;
     T* da3 = p.da ? (T*)p.da + abase : nullptr;
-    float* dacc3 = p.dacc ? p.dacc + (((long long)p.slot * p.N + n) * 3) * HW : nullptr;
+    unsigned long long* dacc3 = p.dacc ? p.dacc + (((long long)p.slot * p.N + n) * 3) * HW : nullptr;
     float* dz = p.dz + plane * HW;
     const float* hs = p.hstore + plane * HW;
     // [delta prev | delta cur | w(prev buffer) x3 | w(cur buffer) x3]
@@ -172,9 +183,9 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
                     Io<T>::st(da3 + HW + q, g1);
                     Io<T>::st(da3 + 2 * HW + q, g2);
                 } else {
-                    atomicAdd(dacc3 + q, g0);
-                    atomicAdd(dacc3 + HW + q, g1);
-                    atomicAdd(dacc3 + 2 * HW + q, g2);
+                    atomicAdd(dacc3 + q, to_fixed(g0));
+                    atomicAdd(dacc3 + HW + q, to_fixed(g1));
+                    atomicAdd(dacc3 + 2 * HW + q, to_fixed(g2));
                 }
                 wcur[j] = J.w0;
                 wcur[M + j] = J.w1;
@@ -209,6 +220,52 @@ __global__ void k_f32_to(const float* src, T* dst, long long n) {
         Io<T>::st(dst + e, src[e]);
 }
 
+template <typename T>
+__global__ void k_fixed_to(const unsigned long long* src, T* dst, long long n) {
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+        Io<T>::st(dst + e, from_fixed(src[e]));
+}
+
+// Batched transpose dst[b][c][r] (+)= src[b][r][c] for b < B (R x Cc planes), through 32 x 32
+// shared-memory tiles (coalesced both ways). Src: storage type, fp32 or 64-bit fixed point.
+template <typename S> __device__ __forceinline__ float ld_any(const S* p) { return Io<S>::ld(p); }
+template <> __device__ __forceinline__ float ld_any<unsigned long long>(const unsigned long long* p) {
+    return from_fixed(*p);
+}
+template <typename S, typename D, bool ADD>
+__global__ void k_transpose(const S* __restrict__ src, D* __restrict__ dst, int R, int Cc) {
+    __shared__ float tile[32][33];
+    const long long b = blockIdx.z;
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    const S* sp = src + b * (long long)R * Cc;
+    D* dp = dst + b * (long long)R * Cc;
+    for (int k = threadIdx.y; k < 32; k += 8) {
+        const int r = r0 + k, c = c0 + threadIdx.x;
+        if (r < R && c < Cc) tile[k][threadIdx.x] = ld_any(sp + (long long)r * Cc + c);
+    }
+    __syncthreads();
+    for (int k = threadIdx.y; k < 32; k += 8) {
+        const int c = c0 + k, r = r0 + threadIdx.x;
+        if (r < R && c < Cc) {
+            D* q = dp + (long long)c * R + r;
+            const float v = tile[threadIdx.x][k];
+            Io<D>::st(q, ADD ? Io<D>::ld(q) + v : v);
+        }
+    }
+}
+template <typename S, typename D, bool ADD>
+cudaError_t launch_transpose(const S* src, D* dst, long long B, int R, int Cc, cudaStream_t st) {
+    const long long plane = (long long)R * Cc;
+    for (long long b0 = 0; b0 < B; b0 += 65535) {   // grid z is limited to 65535
+        const long long nb = std::min<long long>(65535, B - b0);
+        dim3 grid((unsigned)((Cc + 31) / 32), (unsigned)((R + 31) / 32), (unsigned)nb);
+        k_transpose<S, D, ADD><<<grid, dim3(32, 8), 0, st>>>(src + b0 * plane, dst + b0 * plane, R, Cc);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 int gen_threads(int M) { return std::min(1024, std::max(32, ((M + 31) / 32) * 32)); }
 
 template <typename T>
@@ -235,53 +292,156 @@ cudaError_t gen_forward_t(const Problem& P, const void* x, const void* a, const 
     return cudaSuccess;
 }
 
+// Direction-serial backward with the per-direction lam / u of the learnable merge: every direction
+// on the image-layout buffers (horizontal directions walk columns).
 template <typename T>
-cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
-                           const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
+cudaError_t gen_backward_perdir(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
+                                const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
     WsCarver wc(ws);
     float* acc = wc.take<float>(P.U);
     float* dz = wc.take<float>(P.U);
     float* hstore = wc.take<float>(P.U);
-    float* dacc = P.wmode == GSPN_W_SHARED ? wc.take<float>(P.A) : nullptr;
+    unsigned long long* dacc = P.wmode == GSPN_W_SHARED ? wc.take<unsigned long long>(P.A) : nullptr;
     cudaError_t e;
-    if (dacc) {
-        e = cudaMemsetAsync(dacc, 0, P.A * sizeof(float), st);
-        if (e != cudaSuccess) return e;
-    }
-    int slot = 0, seen = 0;
+    if (dacc && (e = cudaMemsetAsync(dacc, 0, P.A * sizeof(unsigned long long), st)) != cudaSuccess) return e;
+    int slot = 0;
     for (unsigned d = kTB; d <= kRL; d <<= 1) {
         if (!(P.mask & d)) continue;
         const int M = is_vertical(d) ? P.W : P.H;
-        // 1) recompute this direction's h (image coordinates) and accumulate sum_d h for du
-        GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, false,
+        GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, slot == 0, false,
                   P.chunk, P.per_dir};
-        if (P.D == 1) g.first = 1;
         size_t smem = 2 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_gen_fwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(g);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        // 2) reverse scan
-        GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, P.H, P.W, P.Cw, d, slot, seen == 0,
+        GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, P.H, P.W, P.Cw, d, slot, slot == 0,
                      P.chunk, P.per_dir, x, lam, dlam, du};
         smem = 8 * (size_t)M * sizeof(float);
         cudaFuncSetAttribute(k_gen_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_gen_bwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(b);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         ++slot;
-        ++seen;
     }
     const int blocks = (int)std::max<long long>(1, std::min<long long>(4096, (P.U + 255) / 256));
-    if (P.per_dir) {
-        k_f32_to<T><<<blocks, 256, 0, st>>>(dz, (T*)dx, P.U);   // dlam_d, du_d written per direction
-    } else {
-        k_gen_bwd_final<T><<<blocks, 256, 0, st>>>((const T*)x, (const T*)lam, (const T*)dy, dz, acc, (T*)dx,
-                                                   (T*)dlam, (T*)du, P.U);
-    }
+    k_f32_to<T><<<blocks, 256, 0, st>>>(dz, (T*)dx, P.U);   // dlam_d, du_d written per direction
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (dacc) {
         const int ab = (int)std::max<long long>(1, std::min<long long>(4096, (P.A + 255) / 256));
-        k_f32_to<T><<<ab, 256, 0, st>>>(dacc, (T*)da, P.A);
+        k_fixed_to<T><<<ab, 256, 0, st>>>(dacc, (T*)da, P.A);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+// Recompute + reverse scan of one direction, which runs as a vertical scan (TB or BT) of the
+// problem with H x W lanes given: the image itself for the vertical directions, its transpose for
+// the horizontal ones.
+template <typename T>
+cudaError_t gen_direction_bwd(const Problem& P, int H, int W, unsigned vdir, int slot, bool first, const void* x,
+                              const void* a, const void* lam, const void* u, const void* dy, void* da,
+                              unsigned long long* dacc, float* acc, float* dz, float* hstore, cudaStream_t st) {
+    const int M = W;
+    GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, H, W, P.Cw, P.D, vdir, slot, first, false, P.chunk, 0};
+    size_t smem = 2 * (size_t)M * sizeof(float);
+    cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_gen_fwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(g);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, H, W, P.Cw, vdir, slot, first,
+                 P.chunk, 0, x, lam, nullptr, nullptr};
+    smem = 8 * (size_t)M * sizeof(float);
+    cudaFuncSetAttribute(k_gen_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_gen_bwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(b);
+    return cudaGetLastError();
+}
+
+int n_vert(const Problem& P) { return ((P.mask & kTB) ? 1 : 0) + ((P.mask & kBT) ? 1 : 0); }
+int n_horz(const Problem& P) { return P.D - n_vert(P); }
+
+// Backward with lam and u shared by the directions. The vertical directions scan the image-layout
+// buffers; the horizontal ones scan transposed copies of x, lam, u, dy and of their logit slots
+// (left->right is then top->bottom of the transpose, right->left bottom->top), so every scan reads
+// and writes whole rows. Their sums over directions and their logit gradients are transposed back.
+template <typename T>
+cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
+                           const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
+    if (P.per_dir) return gen_backward_perdir<T>(P, x, a, lam, u, dy, dx, da, dlam, du, ws, st);
+    const bool shared = P.wmode == GSPN_W_SHARED;
+    const int nV = n_vert(P), nH = n_horz(P);
+    const long long slotA = (long long)P.N * P.Cw * 3 * P.HW;   // logits of one direction slot
+    const long long slotD = (long long)P.N * 3 * P.HW;          // shared-mode gradient of one slot
+    WsCarver wc(ws);
+    float* acc = wc.take<float>(P.U);
+    float* dz = wc.take<float>(P.U);
+    float* hstore = wc.take<float>(P.U);
+    unsigned long long* dacc = shared ? wc.take<unsigned long long>((size_t)P.D * slotD) : nullptr;
+    float *accT = nullptr, *dzT = nullptr;
+    T *xT = nullptr, *lamT = nullptr, *uT = nullptr, *dyT = nullptr, *aT = nullptr, *daT = nullptr;
+    if (nH > 0) {
+        accT = wc.take<float>(P.U);
+        dzT = wc.take<float>(P.U);
+        xT = wc.take<T>(P.U);
+        lamT = wc.take<T>(P.U);
+        uT = wc.take<T>(P.U);
+        dyT = wc.take<T>(P.U);
+        aT = wc.take<T>((size_t)nH * slotA);
+        if (!shared) daT = wc.take<T>((size_t)nH * slotA);
+    }
+    cudaError_t e;
+    if (dacc && (e = cudaMemsetAsync(dacc, 0, (size_t)P.D * slotD * sizeof(unsigned long long), st)) != cudaSuccess)
+        return e;
+    const long long planes = (long long)P.N * P.C;
+    if (nH > 0) {
+        if ((e = launch_transpose<T, T, false>((const T*)x, xT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        if ((e = launch_transpose<T, T, false>((const T*)lam, lamT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        if ((e = launch_transpose<T, T, false>((const T*)u, uT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        if ((e = launch_transpose<T, T, false>((const T*)dy, dyT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        // the horizontal slots follow the vertical ones: one batch of nH * N * Cw * 3 planes
+        if ((e = launch_transpose<T, T, false>((const T*)a + nV * slotA, aT, (long long)nH * P.N * P.Cw * 3, P.H,
+                                               P.W, st)) != cudaSuccess)
+            return e;
+    }
+    int v = 0, h = 0;
+    for (unsigned d = kTB; d <= kRL; d <<= 1) {
+        if (!(P.mask & d)) continue;
+        if (is_vertical(d)) {
+            e = gen_direction_bwd<T>(P, P.H, P.W, d, v, v == 0, x, a, lam, u, dy, da, dacc, acc, dz, hstore, st);
+            ++v;
+        } else {
+            e = gen_direction_bwd<T>(P, P.W, P.H, d == kLR ? kTB : kBT, h, h == 0, xT, aT, lamT, uT, dyT, daT,
+                                     dacc ? dacc + nV * slotD : nullptr, accT, dzT, hstore, st);
+            ++h;
+        }
+        if (e != cudaSuccess) return e;
+    }
+    if (nH > 0) {   // sums of the horizontal directions back to the image layout
+        if (nV > 0) {
+            if ((e = launch_transpose<float, float, true>(accT, acc, planes, P.W, P.H, st)) != cudaSuccess) return e;
+            if ((e = launch_transpose<float, float, true>(dzT, dz, planes, P.W, P.H, st)) != cudaSuccess) return e;
+        } else {
+            if ((e = launch_transpose<float, float, false>(accT, acc, planes, P.W, P.H, st)) != cudaSuccess) return e;
+            if ((e = launch_transpose<float, float, false>(dzT, dz, planes, P.W, P.H, st)) != cudaSuccess) return e;
+        }
+    }
+    const int blocks = (int)std::max<long long>(1, std::min<long long>(4096, (P.U + 255) / 256));
+    k_gen_bwd_final<T><<<blocks, 256, 0, st>>>((const T*)x, (const T*)lam, (const T*)dy, dz, acc, (T*)dx, (T*)dlam,
+                                               (T*)du, P.U);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (shared) {
+        if (nV > 0) {
+            const long long nv = (long long)nV * slotD;
+            const int ab = (int)std::max<long long>(1, std::min<long long>(4096, (nv + 255) / 256));
+            k_fixed_to<T><<<ab, 256, 0, st>>>(dacc, (T*)da, nv);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (nH > 0 &&
+            (e = launch_transpose<unsigned long long, T, false>(dacc + nV * slotD, (T*)da + nV * slotA,
+                                                                (long long)nH * P.N * 3, P.W, P.H, st)) != cudaSuccess)
+            return e;
+    } else if (nH > 0) {
+        if ((e = launch_transpose<T, T, false>(daT, (T*)da + nV * slotA, (long long)nH * P.N * P.Cw * 3, P.W, P.H,
+                                               st)) != cudaSuccess)
+            return e;
     }
     return cudaSuccess;
 }
@@ -300,7 +460,14 @@ size_t generic_ws_bytes(const Problem& p, bool bwd) {
         return b;
     }
     b += 3 * align256(p.U * sizeof(float));
-    if (p.wmode == GSPN_W_SHARED) b += align256(p.A * sizeof(float));
+    if (p.wmode == GSPN_W_SHARED) b += align256(p.A * sizeof(unsigned long long));
+    const int nh = ((p.mask & kLR) ? 1 : 0) + ((p.mask & kRL) ? 1 : 0);
+    if (!p.per_dir && nh > 0) {
+        const size_t es = p.esize();
+        const size_t slot_a = (size_t)p.N * p.Cw * 3 * p.HW;
+        b += 2 * align256(p.U * sizeof(float)) + 4 * align256(p.U * es) + align256(nh * slot_a * es);
+        if (p.wmode != GSPN_W_SHARED) b += align256(nh * slot_a * es);
+    }
     return b;
 }
 

@@ -872,6 +872,258 @@ __global__ void __launch_bounds__(kPlaneBwdThreads) k_plane_bwd(PlaneBwdArgs p) 
     }
 }
 
+// ====================================================== backward, directions scanned concurrently
+// fp32 storage, per-channel weights. Warp d takes the d-th direction of the mask: it recomputes
+// that direction's h into a plane of its own (cd_scan, the forward's strip scan), then runs the
+// reverse scan delta_i = g_i + w_{i+1}^T delta_{i+1} into a second plane of its own, streaming the
+// direction's logits through its ring again, strips in reverse order. The directions' scans are
+// independent given z and g, so the D warps run them at the same time. Afterwards all threads form
+// every direction's logit gradients from its delta and h planes (coalesced, image order) and
+// dx = lam dz, dlam = x dz, du = dy sum_d h^d with dz = sum_d delta^d, both sums in slot order, so
+// the result does not depend on warp timing.
+
+// Primes the ring with the last NSL strips, last first (one commit group per strip).
+template <typename T, int LPT, int NSL>
+__device__ __forceinline__ void cd_prime_rev(uint32_t* ring, const T* a3, const CdDir& g, int HW, int W, int lane) {
+    constexpr int K = CdGeom<T>::K;
+    const int nq = (g.L + K - 1) / K;
+#pragma unroll
+    for (int q = 0; q < NSL; ++q) {
+        if (q < nq) cd_fetch<T, LPT>(ring + q * cd_slot_words<LPT>(), a3, g, HW, W, nq - 1 - q, lane);
+        cd_commit();
+    }
+}
+
+// Reverse scan of one direction by one warp over the lines L-1 .. 0: delta into db (plane layout).
+// (w_{i+1}^T delta)[j] = w_{i+1}[j-1][2] delta[j-1] + w_{i+1}[j][1] delta[j] + w_{i+1}[j+1][0] delta[j+1];
+// no delta flows back through the first line of a chunk (its weights multiply h = 0).
+template <typename T, int LPT, bool LOCAL, int NSL>
+__device__ __forceinline__ void cd_reverse(const float* gz, float* db, uint32_t* ring, const T* a3, const CdDir& g,
+                                           int HW, int W, int chunk, int lane) {
+    constexpr int K = CdGeom<T>::K;
+    constexpr int SLOT = cd_slot_words<LPT>();
+    const int L = g.L, M = g.M;
+    const int nq = (L + K - 1) / K;
+    float del[LPT], pw0[LPT], pw1[LPT], pw2[LPT];   // delta and weights of line i + 1
+    bool on[LPT], hl[LPT], hr[LPT];
+    int pj[LPT];
+#pragma unroll
+    for (int e = 0; e < LPT; ++e) {
+        const int j = e * 32 + lane;
+        del[e] = pw0[e] = pw1[e] = pw2[e] = 0.f;
+        on[e] = j < M;
+        hl[e] = j > 0;
+        hr[e] = j < M - 1;
+        pj[e] = on[e] ? g.p0 + j * g.sj : 0;
+    }
+    for (int qr = 0; qr < nq; ++qr) {
+        const int q = nq - 1 - qr;
+        cd_wait<NSL - 1>();
+        __syncwarp();
+        uint32_t* slot = ring + (qr % NSL) * SLOT;
+        float w0[K][LPT], w2[K][LPT];
+        bool shift = false;
+        {
+            float lg[3][K][LPT];
+            cd_strip_logits<T, LPT>(slot, g, lane, lg);
+#pragma unroll
+            for (int s = 0; s < K; ++s)
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) {
+                    const Wts w = lane_weights_fast_nocheck(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                    shift |= on[e] && q * K + s < L &&
+                             weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                    w0[s][e] = w.w0;
+                    w2[s][e] = w.w2;
+                }
+            if (__any_sync(0xffffffffu, shift)) {   // rare: some logit below the fast form's range
+#pragma unroll
+                for (int s = 0; s < K; ++s)
+#pragma unroll
+                    for (int e = 0; e < LPT; ++e)
+                        if (weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e])) {
+                            const Wts w = weights_shifted(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                            w0[s][e] = w.w0;
+                            w2[s][e] = w.w2;
+                        }
+            }
+        }
+        __syncwarp();
+        if (qr + NSL < nq) cd_fetch<T, LPT>(slot, a3, g, HW, W, nq - 1 - (qr + NSL), lane);
+        cd_commit();
+#pragma unroll
+        for (int s = K - 1; s >= 0; --s) {
+            const int i = q * K + s;
+            if (i < L) {   // warp-uniform
+                const int di = i * g.si;
+                float tl[LPT], tr[LPT], rl[LPT], rr[LPT];
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) {
+                    tl[e] = pw2[e] * del[e];   // lane j's term for lane j + 1
+                    tr[e] = pw0[e] * del[e];   // lane j's term for lane j - 1
+                }
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) {
+                    rl[e] = __shfl_sync(0xffffffffu, tl[e], (lane + 31) & 31);
+                    rr[e] = __shfl_sync(0xffffffffu, tr[e], (lane + 1) & 31);
+                }
+                bool live = i != 0;
+                if constexpr (LOCAL) live = !chunk_start(g.asc, L, chunk, i);
+#pragma unroll
+                for (int e = 0; e < LPT; ++e) {
+                    const float left = lane > 0 ? rl[e] : (e > 0 ? rl[e - 1] : 0.f);
+                    const float right = lane < 31 ? rr[e] : (e < LPT - 1 ? rr[e + 1] : 0.f);
+                    const float gi = gz[on[e] ? pj[e] + di : 0];
+                    const float d = on[e] ? fmaf(pw1[e], del[e], gi) + left + right : 0.f;
+                    if (on[e]) db[pj[e] + di] = d;
+                    del[e] = d;
+                    const bool keep = on[e] && live;
+                    pw0[e] = keep ? w0[s][e] : 0.f;
+                    pw2[e] = keep ? w2[s][e] : 0.f;
+                    pw1[e] = keep ? 1.f - w0[s][e] - w2[s][e] : 0.f;
+                }
+            }
+        }
+    }
+}
+
+// Logit gradients of direction D from its delta and h planes, weights formed again from the logits
+// (all threads, image order, vector loads and stores; W % 4 == 0): at scan position (i, j), i > 0,
+//   dw_k = delta_i[j] h_{i-1}[j+k-1],  da_k = w_k sigmoid(-a_k) (dw_k - sum_k' w_k' dw_k')
+// (zero for out-of-range k and for the first line of a chunk).
+template <typename T, unsigned D, int NT>
+__device__ __forceinline__ void cd_logit_grads(const T* a3, T* da3, const float* hb, const float* db, int H, int W,
+                                               int Wp, int chunk, int tid) {
+    constexpr bool V = D == kTB || D == kBT;
+    const int M = V ? W : H;
+    const int HW = H * W;
+    for (int e0 = tid * 4; e0 < HW; e0 += NT * 4) {
+        const int r = e0 / W, c0 = e0 - r * W;
+        float a0[4], a1[4], a2[4], g0[4], g1[4], g2[4];
+        ld_lanes<T, 4>(a3 + e0, a0);
+        ld_lanes<T, 4>(a3 + HW + e0, a1);
+        ld_lanes<T, 4>(a3 + 2 * HW + e0, a2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int c = c0 + k;
+            const int i = D == kTB ? r : D == kBT ? H - 1 - r : D == kLR ? c : W - 1 - c;
+            const int j = V ? c : r;
+            g0[k] = g1[k] = g2[k] = 0.f;
+            if (!chunk_start(scan_ascending(D), V ? H : W, chunk, i)) {
+                const bool hasl = j > 0, hasr = j < M - 1;
+                const LaneJac J = lane_jacobian(a0[k], a1[k], a2[k], hasl, hasr);
+                const float d = db[r * Wp + c];
+                const float h0 = hasl ? hb[plane_pix<D>(H, W, Wp, i - 1, j - 1)] : 0.f;
+                const float h1 = hb[plane_pix<D>(H, W, Wp, i - 1, j)];
+                const float h2 = hasr ? hb[plane_pix<D>(H, W, Wp, i - 1, j + 1)] : 0.f;
+                const float dw0 = d * h0, dw1 = d * h1, dw2 = d * h2;
+                const float sdw = J.w0 * dw0 + J.w1 * dw1 + J.w2 * dw2;
+                g0[k] = J.g0 * (dw0 - sdw);
+                g1[k] = J.g1 * (dw1 - sdw);
+                g2[k] = J.g2 * (dw2 - sdw);
+            }
+        }
+        st_lanes<T, 4>(da3 + e0, g0);
+        st_lanes<T, 4>(da3 + HW + e0, g1);
+        st_lanes<T, 4>(da3 + 2 * HW + e0, g2);
+    }
+}
+
+// Shared memory of the concurrent-direction backward (floats): z, g, then nd h planes and nd delta
+// planes, then nd rings of NSL strips (16-byte aligned).
+__host__ __device__ constexpr int cdb_ring_offset(int nd, int HWs) { return ((2 + 2 * nd) * HWs + 3) & ~3; }
+// One warp per direction scans; all eight warps share the parallel phases (loads, logit gradients,
+// the final products), which are latency-bound at one CTA per SM.
+constexpr int kCdbThreads = 256;
+
+template <typename T, int LPT, bool LOCAL, int NSL>
+__global__ void __launch_bounds__(kCdbThreads) k_plane_bwd_cd(PlaneBwdArgs p) {
+    extern __shared__ __align__(16) float sm[];
+    const int H = p.H, W = p.W, Wp = p.Wp;
+    const int HW = H * W, HWs = H * Wp;
+    const int nd = __popc(p.mask);
+    float* z = sm;
+    float* gpl = z + HWs;
+    float* hb = gpl + HWs;          // nd planes, slot order
+    float* db = hb + nd * HWs;      // nd planes, slot order
+    uint32_t* rings = reinterpret_cast<uint32_t*>(sm + cdb_ring_offset(nd, HWs));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    unsigned dir = 0;   // this warp's direction: the warp-th set bit of the mask (its slot is warp)
+    {
+        unsigned m = p.mask;
+        for (int k = 0; k < warp && m; ++k) m &= m - 1;
+        dir = m & (0u - m);
+    }
+    const CdDir geo = cd_dir(dir, H, W, Wp);
+    const bool scans = warp < nd;
+    uint32_t* ring = rings + warp * NSL * cd_slot_words<LPT>();
+    float* hw = hb + warp * HWs;
+    float* dw = db + warp * HWs;
+    const int nplanes = p.N * p.C;
+    for (int plane = blockIdx.x; plane < nplanes; plane += gridDim.x) {
+        const int n = plane / p.C, c = plane % p.C;
+        const long long po = (long long)plane * HW;
+        auto aoff = [&](int s) { return (((long long)s * p.N + n) * p.C + c) * 3 * HW; };
+        const T* a3 = (const T*)p.a + aoff(warp);
+        const T *x = (const T*)p.x + po, *lam = (const T*)p.lam + po, *u = (const T*)p.u + po;
+        const T* dy = (const T*)p.dy + po;
+        if (scans) cd_prime<T, LPT, NSL>(ring, a3, geo, HW, W, lane);
+        for (int e0 = tid * 4; e0 < HW; e0 += kCdbThreads * 4) {   // z = lam x, g = u dy
+            float xv[4], lv[4], uv[4], dv[4];
+            ld_lanes<T, 4>(x + e0, xv);
+            ld_lanes<T, 4>(lam + e0, lv);
+            ld_lanes<T, 4>(u + e0, uv);
+            ld_lanes<T, 4>(dy + e0, dv);
+            const int row = e0 / W, col = e0 - row * W;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                z[row * Wp + col + k] = lv[k] * xv[k];
+                gpl[row * Wp + col + k] = uv[k] * dv[k];
+            }
+        }
+        __syncthreads();
+        if (scans) {
+            cd_scan<T, LPT, LOCAL, NSL>(z, hw, ring, a3, geo, HW, W, p.chunk, lane);
+            __syncwarp();   // every lane has read its last strip before the ring is refilled
+            cd_prime_rev<T, LPT, NSL>(ring, a3, geo, HW, W, lane);
+            cd_reverse<T, LPT, LOCAL, NSL>(gpl, dw, ring, a3, geo, HW, W, p.chunk, lane);
+        }
+        __syncthreads();
+        // logit gradients, one direction after another (slot order)
+        {
+            int slot = 0;
+            if (p.mask & kTB) { const long long o = aoff(slot); cd_logit_grads<T, kTB, kCdbThreads>((const T*)p.a + o, (T*)p.da + o, hb + slot * HWs, db + slot * HWs, H, W, Wp, p.chunk, tid); ++slot; }
+            if (p.mask & kBT) { const long long o = aoff(slot); cd_logit_grads<T, kBT, kCdbThreads>((const T*)p.a + o, (T*)p.da + o, hb + slot * HWs, db + slot * HWs, H, W, Wp, p.chunk, tid); ++slot; }
+            if (p.mask & kLR) { const long long o = aoff(slot); cd_logit_grads<T, kLR, kCdbThreads>((const T*)p.a + o, (T*)p.da + o, hb + slot * HWs, db + slot * HWs, H, W, Wp, p.chunk, tid); ++slot; }
+            if (p.mask & kRL) { const long long o = aoff(slot); cd_logit_grads<T, kRL, kCdbThreads>((const T*)p.a + o, (T*)p.da + o, hb + slot * HWs, db + slot * HWs, H, W, Wp, p.chunk, tid); ++slot; }
+        }
+        // dx = lam dz, dlam = x dz, du = dy sum_d h^d (sums in slot order)
+        for (int e0 = tid * 4; e0 < HW; e0 += kCdbThreads * 4) {
+            float xv[4], lv[4], dv[4], ox[4], ol[4], ou[4];
+            ld_lanes<T, 4>(x + e0, xv);
+            ld_lanes<T, 4>(lam + e0, lv);
+            ld_lanes<T, 4>(dy + e0, dv);
+            const int row = e0 / W, col = e0 - row * W;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int q = row * Wp + col + k;
+                float dz = db[q], hs = hb[q];
+                for (int d = 1; d < nd; ++d) {
+                    dz += db[d * HWs + q];
+                    hs += hb[d * HWs + q];
+                }
+                ox[k] = lv[k] * dz;
+                ol[k] = xv[k] * dz;
+                ou[k] = dv[k] * hs;
+            }
+            st_lanes<T, 4>((T*)p.dx + po + e0, ox);
+            st_lanes<T, 4>((T*)p.dlam + po + e0, ol);
+            st_lanes<T, 4>((T*)p.du + po + e0, ou);
+        }
+        __syncthreads();   // the next plane overwrites z, g and the planes
+    }
+}
+
 int plane_wp(const Problem& P) { return P.W % 2 == 0 ? P.W + 1 : P.W; }
 size_t plane_smem(const Problem& P) { return 4 * (size_t)P.H * plane_wp(P) * sizeof(float); }
 int plane_lanes(const Problem& P) {
@@ -968,8 +1220,47 @@ cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t 
     return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true, false>(P, a, st)
                        : plane_fwd_launch3<T, LPT, false, false>(P, a, st);
 }
+size_t cdb_smem(const Problem& P, int nsl, int lpt) {
+    const int nd = __builtin_popcount(P.mask);
+    return (size_t)cdb_ring_offset(nd, P.H * plane_wp(P)) * sizeof(float) + (size_t)nd * nsl * 384 * lpt * 4;
+}
+// Ring depth of the concurrent-direction backward (fp32, rows of whole 16-byte chunks): 3 strips if
+// they fit, else 2; 0 when the kernel does not apply.
+int cdb_ring_depth(const Problem& P) {
+    if (P.dtype != GSPN_F32 || P.per_dir || P.W % 4 != 0 || P.wmode != GSPN_W_PER_CHANNEL) return 0;
+    const int lpt = plane_lanes(P);
+    if (cdb_smem(P, 3, lpt) <= kPlaneSmemBudget) return 3;
+    return cdb_smem(P, 2, lpt) <= kPlaneSmemBudget ? 2 : 0;
+}
+template <typename T, int LPT, bool LOCAL, int NSL>
+cudaError_t plane_bwd_cd_launch4(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
+    const size_t smem = cdb_smem(P, NSL, LPT);
+    auto kern = k_plane_bwd_cd<T, LPT, LOCAL, NSL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    int per_sm = 1;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kCdbThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long want = (long long)std::max(1, per_sm) * device_sm_count();
+    const int grid = (int)std::min<long long>(want, (long long)P.N * P.C);
+    launch_begin(st);
+    kern<<<grid, kCdbThreads, smem, st>>>(a);
+    launch_end(st);
+    return cudaGetLastError();
+}
+template <typename T, int LPT, bool LOCAL>
+cudaError_t plane_bwd_cd_launch3(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
+    return cdb_ring_depth(P) == 3 ? plane_bwd_cd_launch4<T, LPT, LOCAL, 3>(P, a, st)
+                                  : plane_bwd_cd_launch4<T, LPT, LOCAL, 2>(P, a, st);
+}
 template <typename T, int LPT>
 cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream_t st) {
+    if constexpr (sizeof(T) == 4) {
+        if (cdb_ring_depth(P) > 0)
+            return P.chunk > 0 ? plane_bwd_cd_launch3<T, LPT, true>(P, a, st)
+                               : plane_bwd_cd_launch3<T, LPT, false>(P, a, st);
+    }
     return P.chunk > 0 ? plane_bwd_launch3<T, LPT, true>(P, a, st) : plane_bwd_launch3<T, LPT, false>(P, a, st);
 }
 
