@@ -248,6 +248,33 @@ __device__ __forceinline__ LaneJac lane_jacobian(float a0, float a1, float a2, b
     return J;
 }
 
+// Fast forms for the scans whose step cost is instruction issue (the generic family): MUFU
+// exponentials and divisions (relative error a few ulp, normalised after the approximations) when
+// every in-range logit is >= kShiftBelow, else the accurate shifted form. Out-of-range logits are
+// clamped before the exponential so that they cannot produce inf * 0.
+__device__ __forceinline__ Wts lane_weights_fast(float a0, float a1, float a2, bool has_l, bool has_r) {
+    if (weights_need_shift(a0, a1, a2, has_l, has_r)) return weights_shifted(a0, a1, a2, has_l, has_r);
+    return lane_weights_fast_nocheck(a0, a1, a2, has_l, has_r);
+}
+__device__ __forceinline__ LaneJac lane_jacobian_fast(float a0, float a1, float a2, bool has_l, bool has_r) {
+    if (weights_need_shift(a0, a1, a2, has_l, has_r)) return lane_jacobian(a0, a1, a2, has_l, has_r);
+    const float e0 = __expf(-fmaxf(a0, kShiftBelow));
+    const float e1 = __expf(-fmaxf(a1, kShiftBelow));
+    const float e2 = __expf(-fmaxf(a2, kShiftBelow));
+    const float p0 = 1.f + e0, p1 = 1.f + e1, p2 = 1.f + e2;
+    const Wts q = weights_from_p(p0, p1, p2, has_l, has_r);
+    const float inv = __fdividef(1.f, q.w0 + q.w1 + q.w2);
+    LaneJac J;
+    J.w0 = q.w0 * inv;
+    J.w1 = q.w1 * inv;
+    J.w2 = q.w2 * inv;
+    // s_k (1 - s_k) / S = w_k sigmoid(-a_k) = w_k e_k / p_k (0 out of range, where w_k = 0)
+    J.g0 = J.w0 * __fdividef(e0, p0);
+    J.g1 = J.w1 * __fdividef(e1, p1);
+    J.g2 = J.w2 * __fdividef(e2, p2);
+    return J;
+}
+
 // ------------------------------------------------------------------ status word and waits
 // Workspace bytes [0, 256) hold the device status; kernels only ever OR bits into word 0.
 constexpr size_t kStatusBytes = 256;

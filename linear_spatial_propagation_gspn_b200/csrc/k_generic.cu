@@ -35,16 +35,24 @@ struct GenArgs {
     int per_dir;        // lam and u carry a direction axis: this direction's are at slot * U
 };
 
+// The scans are latency-bound: every step's loads depend on nothing but the step index, so each
+// thread asks L2 for its lanes' elements kPrefetch steps ahead (one prefetch per array; the lanes
+// of a warp share one request per line). Only vertical scans do this: their lines are rows, so a
+// warp's prefetches cover whole lines (horizontal scans here only occur on the per-direction path,
+// whose columns would cost a request per lane).
+constexpr int kPrefetch = 8;
+__device__ __forceinline__ void pf_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // Forward scan of one direction for plane blockIdx.x. Writes y (last direction), the fp32
 // partial sum (other directions) and, when hstore is set, this direction's h.
-template <typename T>
+template <typename T, unsigned DIR>
 __global__ void k_gen_fwd(GenArgs p) {
     extern __shared__ float sh[];
     const int plane = blockIdx.x;
     const int n = plane / p.C, c = plane % p.C;
     const long long HW = (long long)p.H * p.W;
-    const int L = is_vertical(p.dir) ? p.H : p.W;
-    const int M = is_vertical(p.dir) ? p.W : p.H;
+    const int L = is_vertical(DIR) ? p.H : p.W;
+    const int M = is_vertical(DIR) ? p.W : p.H;
     const long long lu = p.per_dir ? (long long)p.slot * p.N * p.C * HW : 0;   // this direction's lam / u
     const T* x = (const T*)p.x + plane * HW;
     const T* lam = (const T*)p.lam + lu + plane * HW;
@@ -55,17 +63,27 @@ __global__ void k_gen_fwd(GenArgs p) {
     float* hst = p.hstore ? p.hstore + plane * HW : nullptr;
     float* hp = sh;
     float* hc = sh + M;
+    const bool pf = is_vertical(DIR);
     for (int i = 0; i < L; ++i) {
         for (int j = threadIdx.x; j < M; j += blockDim.x) {
-            const long long q = scan_pixel(p.dir, p.H, p.W, i, j);
+            const long long q = scan_pixel(DIR, p.H, p.W, i, j);
+            if (pf && i + kPrefetch < L) {
+                const long long f = scan_pixel(DIR, p.H, p.W, i + kPrefetch, j);
+                pf_l2(x + f);
+                pf_l2(lam + f);
+                pf_l2(a3 + f);
+                pf_l2(a3 + HW + f);
+                pf_l2(a3 + 2 * HW + f);
+                if (acc && !p.first) pf_l2(acc + f);
+                if (p.per_dir || (p.last && !hst)) pf_l2(u + f);
+            }
             float h = Io<T>::ld(lam + q) * Io<T>::ld(x + q);
-            if (!chunk_start(scan_ascending(p.dir), L, p.chunk, i)) {
-                float w0, w1, w2;
-                lane_weights(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q), Io<T>::ld(a3 + 2 * HW + q), j > 0,
-                             j < M - 1, w0, w1, w2);
-                if (j > 0) h = fmaf(w0, hp[j - 1], h);
-                h = fmaf(w1, hp[j], h);
-                if (j < M - 1) h = fmaf(w2, hp[j + 1], h);
+            if (!chunk_start(scan_ascending(DIR), L, p.chunk, i)) {
+                const Wts w = lane_weights_fast(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q),
+                                                Io<T>::ld(a3 + 2 * HW + q), j > 0, j < M - 1);
+                if (j > 0) h = fmaf(w.w0, hp[j - 1], h);
+                h = fmaf(w.w1, hp[j], h);
+                if (j < M - 1) h = fmaf(w.w2, hp[j + 1], h);
             }
             hc[j] = h;
             if (hst) hst[q] = h;
@@ -122,14 +140,14 @@ struct GenBwdArgs {
 
 // Reverse scan of one direction for plane blockIdx.x:
 //   delta_i = u dy + w_{i+1}^T delta_{i+1};  dz (+)= delta;  da from dw_i[j][k] = delta_i[j] h_{i-1}[j+k-1].
-template <typename T>
+template <typename T, unsigned DIR>
 __global__ void k_gen_bwd(GenBwdArgs p) {
     extern __shared__ float sh[];
     const int plane = blockIdx.x;
     const int n = plane / p.C, c = plane % p.C;
     const long long HW = (long long)p.H * p.W;
-    const int L = is_vertical(p.dir) ? p.H : p.W;
-    const int M = is_vertical(p.dir) ? p.W : p.H;
+    const int L = is_vertical(DIR) ? p.H : p.W;
+    const int M = is_vertical(DIR) ? p.W : p.H;
     const long long lu = p.per_dir ? (long long)p.slot * p.N * p.C * HW : 0;   // this direction's lam / u
     const T* u = (const T*)p.u + lu + plane * HW;
     const T* dy = (const T*)p.dy + plane * HW;
@@ -144,12 +162,33 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
     float* dcur = sh + M;
     float* wprev = sh + 2 * M;
     float* wcur = sh + 5 * M;
+    const bool pf = is_vertical(DIR);
     for (int i = L - 1; i >= 0; --i) {
         for (int j = threadIdx.x; j < M; j += blockDim.x) {
-            const long long q = scan_pixel(p.dir, p.H, p.W, i, j);
+            const long long q = scan_pixel(DIR, p.H, p.W, i, j);
+            if (pf && i - kPrefetch >= 1) {
+                const long long f = scan_pixel(DIR, p.H, p.W, i - kPrefetch, j);
+                pf_l2(u + f);
+                pf_l2(dy + f);
+                pf_l2(a3 + f);
+                pf_l2(a3 + HW + f);
+                pf_l2(a3 + 2 * HW + f);
+                pf_l2(hs + scan_pixel(DIR, p.H, p.W, i - kPrefetch - 1, j));
+                if (!p.first) pf_l2(dz + f);
+                if (dacc3) {
+                    pf_l2(dacc3 + f);
+                    pf_l2(dacc3 + HW + f);
+                    pf_l2(dacc3 + 2 * HW + f);
+                }
+                if (p.per_dir) {
+                    const long long pq = lu + plane * HW + f;
+                    pf_l2((const T*)p.lam + pq);
+                    pf_l2((const T*)p.x + plane * HW + f);
+                }
+            }
             float del = Io<T>::ld(u + q) * Io<T>::ld(dy + q);
             // no delta flows back through the first line of a chunk (it does not see h_{i-1})
-            if (i < L - 1 && !chunk_start(scan_ascending(p.dir), L, p.chunk, i + 1)) {
+            if (i < L - 1 && !chunk_start(scan_ascending(DIR), L, p.chunk, i + 1)) {
                 // (w_{i+1}^T delta_{i+1})[j] = w[j-1][2] d[j-1] + w[j][1] d[j] + w[j+1][0] d[j+1]
                 if (j > 0) del = fmaf(wprev[2 * M + j - 1], dprev[j - 1], del);
                 del = fmaf(wprev[M + j], dprev[j], del);
@@ -168,13 +207,13 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
                 if (p.first) dz[q] = del;
                 else dz[q] += del;
             }
-            if (!chunk_start(scan_ascending(p.dir), L, p.chunk, i)) {
+            if (!chunk_start(scan_ascending(DIR), L, p.chunk, i)) {
                 const bool hl = j > 0, hr = j < M - 1;
-                LaneJac J = lane_jacobian(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q), Io<T>::ld(a3 + 2 * HW + q),
-                                          hl, hr);
-                const float h0 = hl ? hs[scan_pixel(p.dir, p.H, p.W, i - 1, j - 1)] : 0.f;
-                const float h1 = hs[scan_pixel(p.dir, p.H, p.W, i - 1, j)];
-                const float h2 = hr ? hs[scan_pixel(p.dir, p.H, p.W, i - 1, j + 1)] : 0.f;
+                const LaneJac J = lane_jacobian_fast(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q),
+                                                     Io<T>::ld(a3 + 2 * HW + q), hl, hr);
+                const float h0 = hl ? hs[scan_pixel(DIR, p.H, p.W, i - 1, j - 1)] : 0.f;
+                const float h1 = hs[scan_pixel(DIR, p.H, p.W, i - 1, j)];
+                const float h2 = hr ? hs[scan_pixel(DIR, p.H, p.W, i - 1, j + 1)] : 0.f;
                 const float dw0 = del * h0, dw1 = del * h1, dw2 = del * h2;
                 const float s = J.w0 * dw0 + J.w1 * dw1 + J.w2 * dw2;
                 const float g0 = J.g0 * (dw0 - s), g1 = J.g1 * (dw1 - s), g2 = J.g2 * (dw2 - s);
@@ -268,6 +307,47 @@ cudaError_t launch_transpose(const S* src, D* dst, long long B, int R, int Cc, c
 
 int gen_threads(int M) { return std::min(1024, std::max(32, ((M + 31) / 32) * 32)); }
 
+// One launch of the forward / reverse scan of direction d (the direction is a template argument,
+// so the pixel indexing folds to a row base plus the lane).
+template <typename T, unsigned D>
+cudaError_t gen_fwd_launch_d(const GenArgs& g, int M, cudaStream_t st) {
+    const size_t smem = 2 * (size_t)M * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(k_gen_fwd<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    launch_begin(st);
+    k_gen_fwd<T, D><<<g.N * g.C, gen_threads(M), smem, st>>>(g);
+    launch_end(st);
+    return cudaGetLastError();
+}
+template <typename T>
+cudaError_t gen_fwd_launch(const GenArgs& g, int M, cudaStream_t st) {
+    switch (g.dir) {
+    case kTB: return gen_fwd_launch_d<T, kTB>(g, M, st);
+    case kBT: return gen_fwd_launch_d<T, kBT>(g, M, st);
+    case kLR: return gen_fwd_launch_d<T, kLR>(g, M, st);
+    default: return gen_fwd_launch_d<T, kRL>(g, M, st);
+    }
+}
+template <typename T, unsigned D>
+cudaError_t gen_bwd_launch_d(const GenBwdArgs& b, int M, cudaStream_t st) {
+    const size_t smem = 8 * (size_t)M * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(k_gen_bwd<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    launch_begin(st);
+    k_gen_bwd<T, D><<<b.N * b.C, gen_threads(M), smem, st>>>(b);
+    launch_end(st);
+    return cudaGetLastError();
+}
+template <typename T>
+cudaError_t gen_bwd_launch(const GenBwdArgs& b, int M, cudaStream_t st) {
+    switch (b.dir) {
+    case kTB: return gen_bwd_launch_d<T, kTB>(b, M, st);
+    case kBT: return gen_bwd_launch_d<T, kBT>(b, M, st);
+    case kLR: return gen_bwd_launch_d<T, kLR>(b, M, st);
+    default: return gen_bwd_launch_d<T, kRL>(b, M, st);
+    }
+}
+
 template <typename T>
 cudaError_t gen_forward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
                           void* ws, cudaStream_t st) {
@@ -278,13 +358,7 @@ cudaError_t gen_forward_t(const Problem& P, const void* x, const void* a, const 
         if (!(P.mask & d)) continue;
         GenArgs g{x, a, lam, u, y, acc, nullptr, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, seen == 0, seen == P.D - 1,
                   P.chunk, P.per_dir};
-        const int M = is_vertical(d) ? P.W : P.H;
-        const size_t smem = 2 * (size_t)M * sizeof(float);
-        cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        launch_begin(st);
-        k_gen_fwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(g);
-        launch_end(st);
-        cudaError_t e = cudaGetLastError();
+        const cudaError_t e = gen_fwd_launch<T>(g, is_vertical(d) ? P.W : P.H, st);
         if (e != cudaSuccess) return e;
         ++slot;
         ++seen;
@@ -310,16 +384,10 @@ cudaError_t gen_backward_perdir(const Problem& P, const void* x, const void* a, 
         const int M = is_vertical(d) ? P.W : P.H;
         GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, P.H, P.W, P.Cw, P.D, d, slot, slot == 0, false,
                   P.chunk, P.per_dir};
-        size_t smem = 2 * (size_t)M * sizeof(float);
-        cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gen_fwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(g);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = gen_fwd_launch<T>(g, M, st)) != cudaSuccess) return e;
         GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, P.H, P.W, P.Cw, d, slot, slot == 0,
                      P.chunk, P.per_dir, x, lam, dlam, du};
-        smem = 8 * (size_t)M * sizeof(float);
-        cudaFuncSetAttribute(k_gen_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_gen_bwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(b);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = gen_bwd_launch<T>(b, M, st)) != cudaSuccess) return e;
         ++slot;
     }
     const int blocks = (int)std::max<long long>(1, std::min<long long>(4096, (P.U + 255) / 256));
@@ -342,17 +410,11 @@ cudaError_t gen_direction_bwd(const Problem& P, int H, int W, unsigned vdir, int
                               unsigned long long* dacc, float* acc, float* dz, float* hstore, cudaStream_t st) {
     const int M = W;
     GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, H, W, P.Cw, P.D, vdir, slot, first, false, P.chunk, 0};
-    size_t smem = 2 * (size_t)M * sizeof(float);
-    cudaFuncSetAttribute(k_gen_fwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_gen_fwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(g);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = gen_fwd_launch<T>(g, M, st);
     if (e != cudaSuccess) return e;
     GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, H, W, P.Cw, vdir, slot, first,
                  P.chunk, 0, x, lam, nullptr, nullptr};
-    smem = 8 * (size_t)M * sizeof(float);
-    cudaFuncSetAttribute(k_gen_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_gen_bwd<T><<<P.N * P.C, gen_threads(M), smem, st>>>(b);
-    return cudaGetLastError();
+    return gen_bwd_launch<T>(b, M, st);
 }
 
 int n_vert(const Problem& P) { return ((P.mask & kTB) ? 1 : 0) + ((P.mask & kBT) ? 1 : 0); }

@@ -880,8 +880,7 @@ RoleInfo role_info(int role) {
     case R_SZ: return role_info_t<R_SZ>();
     case R_SA: return role_info_t<R_SA>();
     case R_SZA: return role_info_t<R_SZA>();
-    case R_SY: return role_info_t<R_SY>();
-    default: return role_info_t<R_ZSA>();
+    default: return role_info_t<R_SY>();
     }
 }
 
@@ -899,7 +898,6 @@ int mode_of(int v, int D) {
 constexpr int kFixedLanes = 1024;
 int v_lanes(const Problem& P) {
     if (P.W % 8 != 0) return 4;
-    if (const char* e = getenv("GSPN_VLPT")) return atoi(e) == 4 ? 4 : 8;
     if (P.W == kFixedLanes && P.H % 32 == 0 && (long long)P.N * P.C <= device_sm_count()) return 4;
     return 8;
 }
@@ -956,13 +954,7 @@ VCfg v_config(const Problem& P, int role) {
 }
 
 // ---- horizontal geometry: threads, rows per thread (as instantiated), padded rows, ring depth
-int h_pref_rows() {
-    if (const char* e = getenv("GSPN_HROWS")) {
-        const int g = atoi(e);
-        if (g == 1 || g == 2 || g == 4) return g;
-    }
-    return 1;
-}
+int h_pref_rows() { return 1; }
 int h_threads(const Problem& P) {
     const int t = ((P.H + h_pref_rows() - 1) / h_pref_rows() + 31) / 32 * 32;
     return std::min(1024, std::max(t, ((P.H + 3) / 4 + 31) / 32 * 32));
@@ -1056,8 +1048,6 @@ cudaError_t launch_v3(const Problem& P, const SweepArgs& a, const VCfg& c, cudaS
 // Fixed-width kernel: 1024-lane lines (the 1024 x 1024 maps in both scan orientations), scan
 // lengths a multiple of 32.
 bool use_fixed(const Problem& P) {
-    if (const char* e = getenv("GSPN_NOFIXED"))
-        if (atoi(e) != 0) return false;
     return P.W == kFixedLanes && P.H % 32 == 0 && P.H >= 32;
 }
 
@@ -1109,7 +1099,6 @@ cudaError_t launch_role(bool asc, const Problem& P, const SweepArgs& a, int role
     case R_SA: return asc ? cudaErrorNotSupported : launch_v<T, kBT, R_SA>(P, a, st);
     case R_SZA: return asc ? launch_v<T, kTB, R_SZA>(P, a, st) : launch_v<T, kBT, R_SZA>(P, a, st);
     case R_SY: return asc ? launch_v<T, kTB, R_SY>(P, a, st) : launch_v<T, kBT, R_SY>(P, a, st);
-    case R_ZSA: return asc ? cudaErrorNotSupported : launch_v<T, kBT, R_ZSA>(P, a, st);
     default: return cudaErrorNotSupported;
     }
 }
@@ -1140,22 +1129,16 @@ bool tpath_geometry(const Problem& P) {
 }
 int n_vertical(const Problem& P) { return ((P.mask & kTB) ? 1 : 0) + ((P.mask & kBT) ? 1 : 0); }
 
-// How the vertical sweeps hand their results to the horizontal ones on the transposed path:
-//  1: TB writes the partial sum scan-major and z lane-major; BT recomputes z from x and lambda,
-//     adds its scan and writes the partial sum lane-major (one staged output each);
-//  2: TB writes z and the partial sum scan-major; BT reads both and writes both lane-major.
-// With one vertical direction it writes both lane-major.
-int tplan() {
-    if (const char* e = getenv("GSPN_TPLAN")) return atoi(e) == 2 ? 2 : 1;
-    return 1;
-}
+// How the vertical sweeps hand their results to the horizontal ones on the transposed path: TB
+// writes the partial sum scan-major and z lane-major; BT recomputes z from x and lambda, adds its
+// scan and writes the partial sum lane-major (one staged output each). With one vertical
+// direction it writes both lane-major.
 
 // Role of visit v (direction d).
 int visit_role(const Problem& P, unsigned d, int v, bool tp) {
     if (!tp) return mode_of(v, P.D);   // R_FIRST..R_LAST coincide with M_FIRST..M_LAST
     if (is_vertical(d)) {
         if (n_vertical(P) == 1) return R_SZA;
-        if (tplan() == 2) return v == 0 ? R_FIRST : R_ZSA;
         return v == 0 ? R_SZ : R_SA;
     }
     return v == P.D - 1 ? R_SY : R_MID;
@@ -1185,7 +1168,6 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
     WT* table = wc.take<WT>(table_elems(P));
     void *z = nullptr, *acc = nullptr, *zt = nullptr, *acct = nullptr;
     if (tp) {
-        if (nV == 2 && tplan() == 2) z = wc.take<T>(P.U);
         if (nV == 2) acc = wc.take<T>(P.U);
         zt = wc.take<T>(P.U);
         acct = wc.take<T>(P.U);
@@ -1195,25 +1177,9 @@ cudaError_t sweep_forward_t(const Problem& P, const void* x, const void* a, cons
     }
     // A1: weight formation for every direction, once per (n, cw) plane, in one launch; on the
     // transposed path the horizontal slots (which follow the vertical ones) are written [W][H]
-    WeightArgs wa{a, table, P.N, P.Cw, P.H, P.W, P.D, tp ? nV : P.D, {0u, 0u, 0u, 0u}};
-    for (int v = 0, k = 0; k < 4; ++k)
-        if (P.mask & (1u << k)) wa.dirs[v++] = 1u << k;
+    cudaError_t e = launch_weight_table(P, a, table, tp ? nV : P.D, st);
+    if (e != cudaSuccess) return e;
     const int per_slot = P.N * P.Cw;
-    {
-        const int tiles_x = (P.W + kWTileC - 1) / kWTileC, tiles_y = (P.H + kWTileR - 1) / kWTileR;
-        const long long ntiles = (long long)P.D * per_slot * tiles_x * tiles_y;
-        int per_sm = 1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_weights<T>, kWThreads, 0) != cudaSuccess ||
-            per_sm < 1)
-            per_sm = 1;
-        const int grid = (int)std::min<long long>(ntiles, (long long)per_sm * device_sm_count());
-        launch_begin(st);
-        k_weights<T><<<grid, kWThreads, 0, st>>>(wa, tiles_x, tiles_y, (int)ntiles);
-        launch_end(st);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    cudaError_t e;
     // A2-A6: one sweep per direction
     const size_t slot_elems = (size_t)per_slot * 2 * (size_t)P.HW;
     const Problem PS = swapped(P);
@@ -1291,7 +1257,7 @@ size_t sweep_ws_bytes(const Problem& P, bool bwd) {
     if (bwd) return 0;
     size_t b = 256 + align256(table_elems(P) * table_esize(P));
     const size_t ub = align256((size_t)P.U * P.esize());
-    if (tpath(P)) b += (n_vertical(P) == 2 ? (tplan() == 2 ? 4 : 3) : 2) * ub;
+    if (tpath(P)) b += (n_vertical(P) == 2 ? 3 : 2) * ub;
     else if (P.D > 1) b += 2 * ub;
     return b;
 }

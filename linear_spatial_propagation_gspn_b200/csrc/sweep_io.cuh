@@ -126,17 +126,16 @@ enum {
     R_SA = 5,      // x, lam, partial -> partial (lane-major)
     R_SZA = 6,     // x, lam -> z and partial (lane-major)
     R_SY = 7,      // z, partial -> y (lane-major, u applied while writing)
-    R_ZSA = 8,     // z, partial -> z and partial (lane-major)
 };
 template <int ROLE> struct RoleT {
     static constexpr bool XL = ROLE == R_FIRST || ROLE == R_ONLY || ROLE == R_SZ || ROLE == R_SA || ROLE == R_SZA;
-    static constexpr bool ACCIN = ROLE == R_MID || ROLE == R_LAST || ROLE == R_SA || ROLE == R_SY || ROLE == R_ZSA;
+    static constexpr bool ACCIN = ROLE == R_MID || ROLE == R_LAST || ROLE == R_SA || ROLE == R_SY;
     static constexpr bool URING = ROLE == R_ONLY || ROLE == R_LAST;   // u through the ring
     static constexpr bool ZNAT = ROLE == R_FIRST;
     static constexpr bool ANAT = ROLE == R_FIRST || ROLE == R_MID || ROLE == R_SZ;
     static constexpr bool YNAT = ROLE == R_ONLY || ROLE == R_LAST;
-    static constexpr bool ZSTG = ROLE == R_SZ || ROLE == R_SZA || ROLE == R_ZSA;
-    static constexpr bool ASTG = ROLE == R_SA || ROLE == R_SZA || ROLE == R_SY || ROLE == R_ZSA;
+    static constexpr bool ZSTG = ROLE == R_SZ || ROLE == R_SZA;
+    static constexpr bool ASTG = ROLE == R_SA || ROLE == R_SZA || ROLE == R_SY;
     static constexpr bool YSTG = ROLE == R_SY;
     // storage-dtype tensors per ring stage: x lam | z, [partial], [u]  (plus two fp32 weight rows)
     static constexpr int NTEN = (XL ? 2 : 1) + (ACCIN ? 1 : 0) + (URING ? 1 : 0);
