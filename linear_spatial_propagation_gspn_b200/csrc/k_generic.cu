@@ -35,6 +35,37 @@ struct GenArgs {
     int per_dir;        // lam and u carry a direction axis: this direction's are at slot * U
 };
 
+// Weights and Jacobian factors of one lane (see lane_jacobian) with one reciprocal: with
+// p_k = 1 + e_k, e_k = exp(-a_k), the in-range numerators q_k (products of the other two p's),
+// D = q0 + q1 + q2, P = the product of the in-range p's and r = 1 / (P D): w_k = q_k P r and
+// sigmoid(a_k) = 1 / p_k = q_k D r, so g_k = w_k (1 - sigmoid(a_k)) = w_k e_k q_k D r. P D stays
+// finite while every in-range logit is >= kJacBelow; otherwise the accurate form is used. w1 is
+// taken as 1 - w0 - w2.
+constexpr float kJacBelow = -17.f;
+__device__ __forceinline__ LaneJac lane_jacobian_1r(float a0, float a1, float a2, bool has_l, bool has_r) {
+    const float amin = fminf(a1, fminf(has_l ? a0 : a1, has_r ? a2 : a1));
+    if (amin < kJacBelow) return lane_jacobian(a0, a1, a2, has_l, has_r);
+    // out-of-range logits are clamped so that they cannot produce inf * 0
+    const float e0 = __expf(-fmaxf(a0, kJacBelow));
+    const float e1 = __expf(-fmaxf(a1, kJacBelow));
+    const float e2 = __expf(-fmaxf(a2, kJacBelow));
+    const float p0 = 1.f + e0, p1 = 1.f + e1, p2 = 1.f + e2;
+    const Wts q = weights_from_p(p0, p1, p2, has_l, has_r);
+    const float Dn = q.w0 + q.w1 + q.w2;
+    const float P = (has_l ? p0 : 1.f) * p1 * (has_r ? p2 : 1.f);
+    const float r = __fdividef(1.f, P * Dn);
+    const float inv = P * r, dr = Dn * r;
+    LaneJac J;
+    J.w0 = q.w0 * inv;
+    J.w2 = q.w2 * inv;
+    // the row sums to one exactly (a single in-range neighbour gets w1 = 1 and no gradient)
+    J.w1 = 1.f - J.w0 - J.w2;
+    J.g0 = J.w0 * e0 * (q.w0 * dr);
+    J.g1 = J.w1 * e1 * (q.w1 * dr);
+    J.g2 = J.w2 * e2 * (q.w2 * dr);
+    return J;
+}
+
 // The scans are latency-bound: every step's loads depend on nothing but the step index, so each
 // thread asks L2 for its lanes' elements kPrefetch steps ahead (one prefetch per array; the lanes
 // of a warp share one request per line). Only vertical scans do this: their lines are rows, so a
@@ -209,7 +240,7 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
             }
             if (!chunk_start(scan_ascending(DIR), L, p.chunk, i)) {
                 const bool hl = j > 0, hr = j < M - 1;
-                const LaneJac J = lane_jacobian_fast(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q),
+                const LaneJac J = lane_jacobian_1r(Io<T>::ld(a3 + q), Io<T>::ld(a3 + HW + q),
                                                      Io<T>::ld(a3 + 2 * HW + q), hl, hr);
                 const float h0 = hl ? hs[scan_pixel(DIR, p.H, p.W, i - 1, j - 1)] : 0.f;
                 const float h1 = hs[scan_pixel(DIR, p.H, p.W, i - 1, j)];
@@ -238,6 +269,313 @@ __global__ void k_gen_bwd(GenBwdArgs p) {
         __syncthreads();
         float* t = dprev; dprev = dcur; dcur = t;
         t = wprev; wprev = wcur; wcur = t;
+    }
+}
+
+// ---- Concurrent backward for lam and u shared by the directions: every direction of every plane
+// in one launch (grid y = direction), the horizontal directions as top->bottom / bottom->top scans
+// of transposed copies, so every line is a row. Each direction writes its own slots of h, of the
+// partial sum and of the adjoint (no read-modify-write across directions), which lets the SMs hold
+// CTAs of several planes and directions at once and hide one plane's step latency behind another's.
+// A thread owns LPT lanes strided by the block size (lane j = thread + k * blockDim), so every
+// warp-wide load, store and fixed-point atomic touches consecutive addresses. The loads of the next
+// step are issued before the current step's arithmetic (they do not depend on it), and rows
+// kPrefetch steps ahead are requested from L2. The lines in shared memory carry kPad zero lanes on
+// each side, so edge lanes read zeros. Same arithmetic and summation order per lane as k_gen_fwd /
+// k_gen_bwd.
+constexpr int kPad = 4;
+constexpr int kTT = 64;   // tile edge of the transposes
+constexpr int kGenvLPT = 4;
+constexpr int kGenvMaxLanes = 1024;
+
+struct GenvDir {         // one direction's buffers, in the layout it scans (image or transposed)
+    const void* x;
+    const void* lam;
+    const void* u;
+    const void* dy;
+    const void* a;       // this direction's logit slot: N x Cw x 3 x H x W
+    float* hs;           // h of this direction (recompute -> reverse scan; summed by the final kernel)
+    float* dz;           // adjoint delta of this direction
+    void* da;            // per-channel mode: this direction's logit-gradient slot
+    unsigned long long* dacc;   // shared mode: fixed-point sum over channels, N x 3 x H x W
+    int H, W;            // scan length, lanes
+    int asc;             // top->bottom (1) or bottom->top (0)
+};
+struct GenvArgs {
+    GenvDir d[4];
+    int N, C, Cw, chunk;
+};
+
+// One 128-byte line of a row per thread: a warp's prefetches of a row cover it once.
+template <typename E>
+__device__ __forceinline__ void pf_row(const E* row, int W, int t) {
+    if (t * 128 < W * (int)sizeof(E)) pf_l2((const char*)row + t * 128);
+}
+
+template <typename T, int LPT>
+__global__ void __launch_bounds__(kGenvMaxLanes / LPT, 2) k_genv_fwd(GenvArgs p) {
+    constexpr int NT = kGenvMaxLanes / LPT;
+    extern __shared__ float sh[];
+    const GenvDir& D = p.d[blockIdx.y];
+    const bool asc = D.asc != 0;
+    const int plane = blockIdx.x;
+    const int n = plane / p.C, c = plane % p.C;
+    const int H = D.H, W = D.W, LW = W + 2 * kPad;
+    const long long HW = (long long)H * W;
+    const T* x = (const T*)D.x + plane * HW;
+    const T* lam = (const T*)D.lam + plane * HW;
+    const T* a0p = (const T*)D.a + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
+    const T* a1p = a0p + HW;
+    const T* a2p = a1p + HW;
+    float* hst = D.hs + plane * HW;
+    float* hp = sh;
+    float* hc = sh + LW;
+    for (int e = threadIdx.x; e < 2 * LW; e += NT) sh[e] = 0.f;
+    const int t = threadIdx.x;
+    auto rowo = [&](int i) { return (asc ? i : H - 1 - i) * W; };   // row offset in the plane
+    float nx[LPT], nl[LPT], n0[LPT], n1[LPT], n2[LPT];
+    auto fetch = [&](int i) {
+        const int o = rowo(i) + t;
+#pragma unroll
+        for (int k = 0; k < LPT; ++k) {
+            if (t + k * NT >= W) break;
+            nx[k] = Io<T>::ld(x + o + k * NT);
+            nl[k] = Io<T>::ld(lam + o + k * NT);
+            n0[k] = Io<T>::ld(a0p + o + k * NT);
+            n1[k] = Io<T>::ld(a1p + o + k * NT);
+            n2[k] = Io<T>::ld(a2p + o + k * NT);
+        }
+    };
+    fetch(0);
+    __syncthreads();
+    for (int i = 0; i < H; ++i) {
+        float cx[LPT], cl[LPT], c0[LPT], c1[LPT], c2[LPT];
+#pragma unroll
+        for (int k = 0; k < LPT; ++k) {
+            cx[k] = nx[k]; cl[k] = nl[k]; c0[k] = n0[k]; c1[k] = n1[k]; c2[k] = n2[k];
+        }
+        if (i + 1 < H) fetch(i + 1);
+        if (i + kPrefetch < H) {
+            const int f = rowo(i + kPrefetch);
+            pf_row(x + f, W, t);
+            pf_row(lam + f, W, t);
+            pf_row(a0p + f, W, t);
+            pf_row(a1p + f, W, t);
+            pf_row(a2p + f, W, t);
+        }
+        const int o = rowo(i) + t;
+        const bool cs = chunk_start(asc, H, p.chunk, i);
+#pragma unroll
+        for (int k = 0; k < LPT; ++k) {
+            const int j = t + k * NT;
+            if (j >= W) break;
+            float h = cl[k] * cx[k];
+            if (!cs) {
+                const Wts w = lane_weights_fast(c0[k], c1[k], c2[k], j > 0, j < W - 1);
+                if (j > 0) h = fmaf(w.w0, hp[kPad + j - 1], h);
+                h = fmaf(w.w1, hp[kPad + j], h);
+                if (j < W - 1) h = fmaf(w.w2, hp[kPad + j + 1], h);
+            }
+            hc[kPad + j] = h;
+            hst[o + k * NT] = h;
+        }
+        __syncthreads();
+        float* tt = hp;
+        hp = hc;
+        hc = tt;
+    }
+}
+
+template <typename T, bool SHARED, int LPT>
+__global__ void __launch_bounds__(kGenvMaxLanes / LPT, 2) k_genv_bwd(GenvArgs p) {
+    constexpr int NT = kGenvMaxLanes / LPT;
+    extern __shared__ float sh[];
+    const GenvDir& D = p.d[blockIdx.y];
+    const bool asc = D.asc != 0;
+    const int plane = blockIdx.x;
+    const int n = plane / p.C, c = plane % p.C;
+    const int H = D.H, W = D.W, LW = W + 2 * kPad;
+    const long long HW = (long long)H * W;
+    const T* u = (const T*)D.u + plane * HW;
+    const T* dy = (const T*)D.dy + plane * HW;
+    const long long abase = ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
+    const T* a0p = (const T*)D.a + abase;
+    const T* a1p = a0p + HW;
+    const T* a2p = a1p + HW;
+    T* da0 = SHARED ? nullptr : (T*)D.da + abase;
+    unsigned long long* dq0 = SHARED ? D.dacc + (long long)n * 3 * HW : nullptr;
+    float* dz = D.dz + plane * HW;
+    const float* hs = D.hs + plane * HW;
+    // [delta prev | delta cur | w prev x3 | w cur x3 | h of line i-1, two buffers], each padded
+    float* dprev = sh;
+    float* dcur = sh + LW;
+    float* wprev = sh + 2 * LW;
+    float* wcur = sh + 5 * LW;
+    float* hb = sh + 8 * LW;
+    for (int e = threadIdx.x; e < 10 * LW; e += NT) sh[e] = 0.f;
+    const int t = threadIdx.x;
+    auto rowo = [&](int i) { return (asc ? i : H - 1 - i) * W; };
+    float nu[LPT], ndy[LPT], n0[LPT], n1[LPT], n2[LPT], nh[LPT];
+    // the loads of step i: u, dy, logits of line i and h of line i - 1 (its neighbours are read
+    // from the shared copy that step i's predecessor writes, one barrier later)
+    auto fetch = [&](int i) {
+        const int o = rowo(i) + t;
+        const int o1 = i > 0 ? rowo(i - 1) + t : 0;
+#pragma unroll
+        for (int k = 0; k < LPT; ++k) {
+            if (t + k * NT >= W) break;
+            nu[k] = Io<T>::ld(u + o + k * NT);
+            ndy[k] = Io<T>::ld(dy + o + k * NT);
+            n0[k] = Io<T>::ld(a0p + o + k * NT);
+            n1[k] = Io<T>::ld(a1p + o + k * NT);
+            n2[k] = Io<T>::ld(a2p + o + k * NT);
+            nh[k] = i > 0 ? hs[o1 + k * NT] : 0.f;
+        }
+    };
+    fetch(H - 1);
+    int hbuf = 0;
+    {   // h of line H - 2 into the shared copy for the first step
+        float* hl = hb + kPad;
+#pragma unroll
+        for (int k = 0; k < LPT; ++k)
+            if (t + k * NT < W) hl[t + k * NT] = nh[k];
+    }
+    __syncthreads();
+    for (int i = H - 1; i >= 0; --i) {
+        float cu[LPT], cdy[LPT], c0[LPT], c1[LPT], c2[LPT];
+#pragma unroll
+        for (int k = 0; k < LPT; ++k) {
+            cu[k] = nu[k]; cdy[k] = ndy[k]; c0[k] = n0[k]; c1[k] = n1[k]; c2[k] = n2[k];
+        }
+        const float* hl = hb + hbuf * LW + kPad;   // h of line i - 1 (all lanes, from the previous step)
+        if (i > 0) {
+            fetch(i - 1);
+            // h of line i - 2 for the next step, into the other buffer
+            float* hn = hb + (hbuf ^ 1) * LW + kPad;
+#pragma unroll
+            for (int k = 0; k < LPT; ++k)
+                if (t + k * NT < W) hn[t + k * NT] = nh[k];
+        }
+        if (i - kPrefetch >= 1) {
+            const int f = rowo(i - kPrefetch);
+            pf_row(u + f, W, t);
+            pf_row(dy + f, W, t);
+            pf_row(a0p + f, W, t);
+            pf_row(a1p + f, W, t);
+            pf_row(a2p + f, W, t);
+            pf_row(hs + rowo(i - kPrefetch - 1), W, t);
+            if (SHARED) {
+                pf_row(dq0 + f, W, t);
+                pf_row(dq0 + HW + f, W, t);
+                pf_row(dq0 + 2 * HW + f, W, t);
+            }
+        }
+        const int o = rowo(i) + t;
+        // no delta flows back through the first line of a chunk (it does not see h_{i-1})
+        const bool back = i < H - 1 && !chunk_start(asc, H, p.chunk, i + 1);
+        const bool cs = chunk_start(asc, H, p.chunk, i);
+        const float* dpv = dprev + kPad;
+        const float* w0v = wprev + kPad;
+        const float* w1v = wprev + LW + kPad;
+        const float* w2v = wprev + 2 * LW + kPad;
+#pragma unroll
+        for (int k = 0; k < LPT; ++k) {
+            const int j = t + k * NT;
+            if (j >= W) break;
+            float d = cu[k] * cdy[k];
+            if (back) {
+                // (w_{i+1}^T delta_{i+1})[j] = w[j-1][2] d[j-1] + w[j][1] d[j] + w[j+1][0] d[j+1]
+                if (j > 0) d = fmaf(w2v[j - 1], dpv[j - 1], d);
+                d = fmaf(w1v[j], dpv[j], d);
+                if (j < W - 1) d = fmaf(w0v[j + 1], dpv[j + 1], d);
+            }
+            dcur[kPad + j] = d;
+            dz[o + k * NT] = d;
+            float g0 = 0.f, g1 = 0.f, g2 = 0.f;
+            if (!cs) {
+                const LaneJac J = lane_jacobian_1r(c0[k], c1[k], c2[k], j > 0, j < W - 1);
+                const float dw0 = d * hl[j - 1], dw1 = d * hl[j], dw2 = d * hl[j + 1];
+                const float sm = J.w0 * dw0 + J.w1 * dw1 + J.w2 * dw2;
+                g0 = J.g0 * (dw0 - sm);
+                g1 = J.g1 * (dw1 - sm);
+                g2 = J.g2 * (dw2 - sm);
+                wcur[kPad + j] = J.w0;
+                wcur[LW + kPad + j] = J.w1;
+                wcur[2 * LW + kPad + j] = J.w2;
+                if constexpr (SHARED) {
+                    atomicAdd(dq0 + o + k * NT, to_fixed(g0));
+                    atomicAdd(dq0 + HW + o + k * NT, to_fixed(g1));
+                    atomicAdd(dq0 + 2 * HW + o + k * NT, to_fixed(g2));
+                }
+            }
+            if constexpr (!SHARED) {
+                Io<T>::st(da0 + o + k * NT, g0);
+                Io<T>::st(da0 + HW + o + k * NT, g1);
+                Io<T>::st(da0 + 2 * HW + o + k * NT, g2);
+            }
+        }
+        __syncthreads();
+        float* tt = dprev; dprev = dcur; dcur = tt;
+        tt = wprev; wprev = wcur; wcur = tt;
+        hbuf ^= 1;
+    }
+}
+
+// dx = lam dz, dlam = x dz, du = dy acc with dz and acc the sums of the directions' slots: up to
+// two image-layout slots (the vertical directions) and up to two transposed ones ([W][H] per plane,
+// the horizontal directions), the latter read through a 64 x 64 shared-memory transpose per tile
+// (coalesced on both sides). Null slots are absent directions. Per element the sum is taken as
+// (horizontal 0 + horizontal 1) + vertical 0 + vertical 1.
+struct GenvFinal {
+    const float *accV0, *accV1, *dzV0, *dzV1;   // image layout
+    const float *accH0, *accH1, *dzH0, *dzH1;   // transposed layout
+};
+template <typename T>
+__global__ void __launch_bounds__(256) k_genv_final(GenvFinal f, const T* __restrict__ x, const T* __restrict__ lam,
+                                                    const T* __restrict__ dy, T* dx, T* dlam, T* du, int H, int W) {
+    __shared__ float ta[kTT][kTT + 1];
+    __shared__ float tz[kTT][kTT + 1];
+    const long long HW = (long long)H * W, pb = blockIdx.z * HW;
+    const int r0 = blockIdx.y * kTT, c0 = blockIdx.x * kTT;
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+    if (f.accH0) {
+        // transposed slots: image (r, c) at [c][r]; this thread reads rows c0 + ty + 4k, column r0 + tx
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+            const int c = c0 + ty + 4 * k, r = r0 + tx;
+            float va = 0.f, vz = 0.f;
+            if (r < H && c < W) {
+                const long long q = pb + (long long)c * H + r;
+                va = f.accH0[q];
+                vz = f.dzH0[q];
+                if (f.accH1) {
+                    va += f.accH1[q];
+                    vz += f.dzH1[q];
+                }
+            }
+            ta[ty + 4 * k][tx] = va;
+            tz[ty + 4 * k][tx] = vz;
+        }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int k = 0; k < 16; ++k) {
+        const int r = r0 + ty + 4 * k, c = c0 + tx;
+        if (r >= H || c >= W) continue;
+        const long long e = pb + (long long)r * W + c;
+        float a = f.accH0 ? ta[tx][ty + 4 * k] : 0.f;
+        float z = f.accH0 ? tz[tx][ty + 4 * k] : 0.f;
+        if (f.accV0) {
+            a += f.accV0[e];
+            z += f.dzV0[e];
+        }
+        if (f.accV1) {
+            a += f.accV1[e];
+            z += f.dzV1[e];
+        }
+        Io<T>::st(dx + e, Io<T>::ld(lam + e) * z);
+        Io<T>::st(dlam + e, Io<T>::ld(x + e) * z);
+        Io<T>::st(du + e, Io<T>::ld(dy + e) * a);
     }
 }
 
@@ -271,24 +609,33 @@ template <typename S> __device__ __forceinline__ float ld_any(const S* p) { retu
 template <> __device__ __forceinline__ float ld_any<unsigned long long>(const unsigned long long* p) {
     return from_fixed(*p);
 }
+// Batched transpose of R x Cc planes through 64 x 64 shared tiles; a thread moves 16 elements and
+// issues all 16 loads before the first shared-memory store (enough bytes in flight per SM to keep
+// HBM busy). ADD adds the transposed values onto dst.
 template <typename S, typename D, bool ADD>
-__global__ void k_transpose(const S* __restrict__ src, D* __restrict__ dst, int R, int Cc) {
-    __shared__ float tile[32][33];
+__global__ void __launch_bounds__(256) k_transpose(const S* __restrict__ src, D* __restrict__ dst, int R, int Cc) {
+    __shared__ float tile[kTT][kTT + 1];
     const long long b = blockIdx.z;
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    const int r0 = blockIdx.y * kTT, c0 = blockIdx.x * kTT;
     const S* sp = src + b * (long long)R * Cc;
     D* dp = dst + b * (long long)R * Cc;
-    for (int k = threadIdx.y; k < 32; k += 8) {
-        const int r = r0 + k, c = c0 + threadIdx.x;
-        if (r < R && c < Cc) tile[k][threadIdx.x] = ld_any(sp + (long long)r * Cc + c);
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;   // 64 x 4 threads
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int r = r0 + ty + 4 * k, c = c0 + tx;
+        v[k] = (r < R && c < Cc) ? ld_any(sp + (long long)r * Cc + c) : 0.f;
     }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) tile[ty + 4 * k][tx] = v[k];
     __syncthreads();
-    for (int k = threadIdx.y; k < 32; k += 8) {
-        const int c = c0 + k, r = r0 + threadIdx.x;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int c = c0 + ty + 4 * k, r = r0 + tx;
         if (r < R && c < Cc) {
             D* q = dp + (long long)c * R + r;
-            const float v = tile[threadIdx.x][k];
-            Io<D>::st(q, ADD ? Io<D>::ld(q) + v : v);
+            const float t = tile[tx][ty + 4 * k];
+            Io<D>::st(q, ADD ? Io<D>::ld(q) + t : t);
         }
     }
 }
@@ -297,8 +644,8 @@ cudaError_t launch_transpose(const S* src, D* dst, long long B, int R, int Cc, c
     const long long plane = (long long)R * Cc;
     for (long long b0 = 0; b0 < B; b0 += 65535) {   // grid z is limited to 65535
         const long long nb = std::min<long long>(65535, B - b0);
-        dim3 grid((unsigned)((Cc + 31) / 32), (unsigned)((R + 31) / 32), (unsigned)nb);
-        k_transpose<S, D, ADD><<<grid, dim3(32, 8), 0, st>>>(src + b0 * plane, dst + b0 * plane, R, Cc);
+        dim3 grid((unsigned)((Cc + kTT - 1) / kTT), (unsigned)((R + kTT - 1) / kTT), (unsigned)nb);
+        k_transpose<S, D, ADD><<<grid, 256, 0, st>>>(src + b0 * plane, dst + b0 * plane, R, Cc);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -410,15 +757,138 @@ cudaError_t gen_direction_bwd(const Problem& P, int H, int W, unsigned vdir, int
                               unsigned long long* dacc, float* acc, float* dz, float* hstore, cudaStream_t st) {
     const int M = W;
     GenArgs g{x, a, lam, u, nullptr, acc, hstore, P.N, P.C, H, W, P.Cw, P.D, vdir, slot, first, false, P.chunk, 0};
-    cudaError_t e = gen_fwd_launch<T>(g, M, st);
-    if (e != cudaSuccess) return e;
     GenBwdArgs b{a, u, dy, dacc ? nullptr : da, dacc, dz, hstore, P.N, P.C, H, W, P.Cw, vdir, slot, first,
                  P.chunk, 0, x, lam, nullptr, nullptr};
+    cudaError_t e = gen_fwd_launch<T>(g, M, st);
+    if (e != cudaSuccess) return e;
     return gen_bwd_launch<T>(b, M, st);
 }
 
 int n_vert(const Problem& P) { return ((P.mask & kTB) ? 1 : 0) + ((P.mask & kBT) ? 1 : 0); }
 int n_horz(const Problem& P) { return P.D - n_vert(P); }
+
+// The concurrent backward runs lam / u shared by the directions with at most kGenvMaxLanes lanes
+// per scanned line.
+bool genv_ok(const Problem& P) {
+    auto lanes_ok = [](int L) { return L <= kGenvMaxLanes; };
+    return !P.per_dir && P.HW < (1LL << 31) && (n_vert(P) == 0 || lanes_ok(P.W)) && (n_horz(P) == 0 || lanes_ok(P.H));
+}
+
+template <typename T>
+cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
+                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
+    const bool shared = P.wmode == GSPN_W_SHARED;
+    const int nV = n_vert(P), nH = n_horz(P);
+    const long long slotA = (long long)P.N * P.Cw * 3 * P.HW;   // logits of one direction slot
+    const long long slotD = (long long)P.N * 3 * P.HW;          // shared-mode gradient of one slot
+    const long long planes = (long long)P.N * P.C;
+    WsCarver wc(ws);
+    float* hs = wc.take<float>((size_t)P.D * P.U);   // h per direction: also the terms of du
+    float* dz = wc.take<float>((size_t)P.D * P.U);
+    unsigned long long* dacc = shared ? wc.take<unsigned long long>((size_t)P.D * slotD) : nullptr;
+    T *xT = nullptr, *lamT = nullptr, *uT = nullptr, *dyT = nullptr, *aT = nullptr, *daT = nullptr;
+    if (nH > 0) {
+        xT = wc.take<T>(P.U);
+        lamT = wc.take<T>(P.U);
+        uT = wc.take<T>(P.U);
+        dyT = wc.take<T>(P.U);
+        aT = wc.take<T>((size_t)nH * slotA);
+        if (!shared) daT = wc.take<T>((size_t)nH * slotA);
+    }
+    cudaError_t e;
+    if (dacc && (e = cudaMemsetAsync(dacc, 0, (size_t)P.D * slotD * sizeof(unsigned long long), st)) != cudaSuccess)
+        return e;
+    if (nH > 0) {
+        if ((e = launch_transpose<T, T, false>((const T*)x, xT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        if ((e = launch_transpose<T, T, false>((const T*)lam, lamT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        if ((e = launch_transpose<T, T, false>((const T*)u, uT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        if ((e = launch_transpose<T, T, false>((const T*)dy, dyT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        // the horizontal slots follow the vertical ones: one batch of nH * N * Cw * 3 planes
+        if ((e = launch_transpose<T, T, false>((const T*)a + nV * slotA, aT, (long long)nH * P.N * P.Cw * 3, P.H,
+                                               P.W, st)) != cudaSuccess)
+            return e;
+    }
+    GenvArgs g;
+    g.N = P.N;
+    g.C = P.C;
+    g.Cw = P.Cw;
+    g.chunk = P.chunk;
+    int v = 0, h = 0, k = 0, lanes = 0;
+    for (unsigned d = kTB; d <= kRL; d <<= 1) {
+        if (!(P.mask & d)) continue;
+        GenvDir& G = g.d[k];
+        G.hs = hs + (size_t)k * P.U;
+        G.dz = dz + (size_t)k * P.U;
+        if (is_vertical(d)) {
+            G.x = x; G.lam = lam; G.u = u; G.dy = dy;
+            G.a = (const T*)a + v * slotA;
+            G.da = shared ? nullptr : (void*)((T*)da + v * slotA);
+            G.dacc = shared ? dacc + v * slotD : nullptr;
+            G.H = P.H; G.W = P.W; G.asc = d == kTB;
+            ++v;
+        } else {
+            G.x = xT; G.lam = lamT; G.u = uT; G.dy = dyT;
+            G.a = aT + h * slotA;
+            G.da = shared ? nullptr : (void*)(daT + h * slotA);
+            G.dacc = shared ? dacc + (nV + h) * slotD : nullptr;
+            G.H = P.W; G.W = P.H; G.asc = d == kLR;
+            ++h;
+        }
+        lanes = std::max(lanes, G.W);
+        ++k;
+    }
+    const int threads = kGenvMaxLanes / kGenvLPT;   // the kernels' lane stride
+    const size_t lw = (size_t)lanes + 2 * kPad;
+    const dim3 grid((unsigned)planes, (unsigned)P.D);
+    if ((e = cudaFuncSetAttribute(k_genv_fwd<T, kGenvLPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(2 * lw * sizeof(float)))) != cudaSuccess)
+        return e;
+    launch_begin(st);
+    k_genv_fwd<T, kGenvLPT><<<grid, threads, 2 * lw * sizeof(float), st>>>(g);
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    auto kb = shared ? k_genv_bwd<T, true, kGenvLPT> : k_genv_bwd<T, false, kGenvLPT>;
+    if ((e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(10 * lw * sizeof(float)))) !=
+        cudaSuccess)
+        return e;
+    launch_begin(st);
+    kb<<<grid, threads, 10 * lw * sizeof(float), st>>>(g);
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    for (long long b0 = 0; b0 < planes; b0 += 65535) {   // grid z is limited to 65535
+        const long long nb = std::min<long long>(65535, planes - b0);
+        const size_t off = (size_t)b0 * P.HW;
+        auto slot = [&](float* base, int i) -> const float* { return base + (size_t)i * P.U + off; };
+        GenvFinal f{};
+        if (nV > 0) { f.accV0 = slot(hs, 0); f.dzV0 = slot(dz, 0); }
+        if (nV > 1) { f.accV1 = slot(hs, 1); f.dzV1 = slot(dz, 1); }
+        if (nH > 0) { f.accH0 = slot(hs, nV); f.dzH0 = slot(dz, nV); }
+        if (nH > 1) { f.accH1 = slot(hs, nV + 1); f.dzH1 = slot(dz, nV + 1); }
+        const dim3 fg((unsigned)((P.W + kTT - 1) / kTT), (unsigned)((P.H + kTT - 1) / kTT), (unsigned)nb);
+        launch_begin(st);
+        k_genv_final<T><<<fg, 256, 0, st>>>(f, (const T*)x + off, (const T*)lam + off, (const T*)dy + off,
+                                            (T*)dx + off, (T*)dlam + off, (T*)du + off, P.H, P.W);
+        launch_end(st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (shared) {
+        if (nV > 0) {
+            const long long nv = (long long)nV * slotD;
+            const int ab = (int)std::max<long long>(1, std::min<long long>(4096, (nv + 255) / 256));
+            k_fixed_to<T><<<ab, 256, 0, st>>>(dacc, (T*)da, nv);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (nH > 0 &&
+            (e = launch_transpose<unsigned long long, T, false>(dacc + nV * slotD, (T*)da + nV * slotA,
+                                                                (long long)nH * P.N * 3, P.W, P.H, st)) != cudaSuccess)
+            return e;
+    } else if (nH > 0) {
+        if ((e = launch_transpose<T, T, false>(daT, (T*)da + nV * slotA, (long long)nH * P.N * P.Cw * 3, P.W, P.H,
+                                               st)) != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
 
 // Backward with lam and u shared by the directions. The vertical directions scan the image-layout
 // buffers; the horizontal ones scan transposed copies of x, lam, u, dy and of their logit slots
@@ -428,6 +898,7 @@ template <typename T>
 cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
     if (P.per_dir) return gen_backward_perdir<T>(P, x, a, lam, u, dy, dx, da, dlam, du, ws, st);
+    if (genv_ok(P)) return gen_backward_cc<T>(P, x, a, lam, u, dy, dx, da, dlam, du, ws, st);
     const bool shared = P.wmode == GSPN_W_SHARED;
     const int nV = n_vert(P), nH = n_horz(P);
     const long long slotA = (long long)P.N * P.Cw * 3 * P.HW;   // logits of one direction slot
@@ -521,9 +992,20 @@ size_t generic_ws_bytes(const Problem& p, bool bwd) {
         if (p.D > 1) b += align256(p.U * sizeof(float));
         return b;
     }
+    const int nh = ((p.mask & kLR) ? 1 : 0) + ((p.mask & kRL) ? 1 : 0);
+    if (genv_ok(p)) {   // the layout gen_backward_cc carves
+        const size_t es = p.esize();
+        const size_t slot_a = (size_t)p.N * p.Cw * 3 * p.HW, slot_d = (size_t)p.N * 3 * p.HW;
+        b += 2 * align256((size_t)p.D * p.U * sizeof(float));
+        if (p.wmode == GSPN_W_SHARED) b += align256((size_t)p.D * slot_d * sizeof(unsigned long long));
+        if (nh > 0) {
+            b += 4 * align256(p.U * es) + align256(nh * slot_a * es);
+            if (p.wmode != GSPN_W_SHARED) b += align256(nh * slot_a * es);
+        }
+        return b;
+    }
     b += 3 * align256(p.U * sizeof(float));
     if (p.wmode == GSPN_W_SHARED) b += align256(p.A * sizeof(unsigned long long));
-    const int nh = ((p.mask & kLR) ? 1 : 0) + ((p.mask & kRL) ? 1 : 0);
     if (!p.per_dir && nh > 0) {
         const size_t es = p.esize();
         const size_t slot_a = (size_t)p.N * p.Cw * 3 * p.HW;
