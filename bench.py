@@ -62,6 +62,8 @@ def parse_args():
                     help="kernel family (auto: the library's choice)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch N (small cases for profiler captures; not a bench line)")
+    ap.add_argument("--height", type=int, default=0,
+                    help="override the workload's map height H (small cases for profiler captures; not a bench line)")
     return ap.parse_args()
 
 
@@ -291,6 +293,8 @@ def bench_workload(args, name, rank, local_rank, world):
     wl = gspn_inputs.WORKLOADS[name]
     if args.batch:
         wl = wl.with_(N=args.batch)
+    if args.height:
+        wl = wl.with_(H=args.height)
     dev = torch.device("cuda", local_rank)
     full_wl = wl
     shard = None
@@ -366,7 +370,8 @@ def bench_workload(args, name, rank, local_rank, world):
     kern_ms = sum(per)
     names = launch_names(wl, algo, launches)
     achieved = comp / (kern_ms * 1e-3) / 1e9
-    traffic, per_launch = committed_traffic(wl.name) if not (args.batch or args.shard) else (None, None)
+    traffic, per_launch = (committed_traffic(wl.name) if not (args.batch or args.height or args.shard)
+                           else (None, None))
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
         "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -517,6 +522,8 @@ def run_proxy(args):
     wl = gspn_inputs.WORKLOADS[args.workload]
     if args.batch:
         wl = wl.with_(N=args.batch)
+    if args.height:
+        wl = wl.with_(H=args.height)
     Cp = args.proxy
     pw = wl.with_(C=Cp)
     t = gspn_inputs.make_inputs(wl, device=dev)
