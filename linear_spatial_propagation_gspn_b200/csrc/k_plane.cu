@@ -307,6 +307,12 @@ template <int N> __device__ __forceinline__ void cd_wait() { asm volatile("cp.as
 
 // Float offset of the rings in shared memory: after z and the nd h planes, rounded up to 16 bytes.
 __host__ __device__ constexpr int cd_ring_offset(int nd, int HWs) { return ((1 + nd) * HWs + 3) & ~3; }
+// The same for h planes of hbytes per element (the forward keeps them in the storage type: bf16
+// planes take half the shared memory, so more CTAs fit on an SM; the sum over directions is then
+// formed from h rounded to bf16, well inside the bf16 output's tolerance).
+__host__ __device__ constexpr int cd_ring_offset_h(int nd, int HWs, int hbytes) {
+    return ((HWs * 4 + nd * HWs * hbytes + 15) / 16) * 4;
+}
 
 template <typename T> struct CdGeom {
     static constexpr int K = 16 / (int)sizeof(T);   // scan lines per ring strip = elements per 16 bytes
@@ -369,20 +375,21 @@ __device__ __forceinline__ void cd_fetch(uint32_t* slot, const T* a3, const CdDi
     }
 }
 
-// All logits of the strip for this thread's lanes: lg[k][s][e] = logit k of line s, lane e 32 + lane.
-template <typename T, int LPT>
-__device__ __forceinline__ void cd_strip_logits(const uint32_t* slot, const CdDir& g, int lane,
-                                                float (&lg)[3][CdGeom<T>::K][LPT]) {
-    static_assert(sizeof(T) == 4, "the concurrent-direction forward runs fp32 storage");
+// Logits of KH lines of the strip (lines s0 .. s0 + KH - 1) for this thread's lanes:
+// lg[k][s][e] = logit k of line s0 + s, lane e 32 + lane.
+template <typename T, int LPT, int KH>
+__device__ __forceinline__ void cd_strip_logits(const uint32_t* slot, const CdDir& g, int lane, int s0,
+                                                float (&lg)[3][KH][LPT]) {
     constexpr int K = CdGeom<T>::K;
     if (g.vert) {
         const T* src = reinterpret_cast<const T*>(slot);
 #pragma unroll
         for (int k = 0; k < 3; ++k)
 #pragma unroll
-            for (int s = 0; s < K; ++s)
+            for (int s = 0; s < KH; ++s)
 #pragma unroll
-                for (int e = 0; e < LPT; ++e) lg[k][s][e] = Io<T>::ld(src + (k * K + s) * 32 * LPT + e * 32 + lane);
+                for (int e = 0; e < LPT; ++e)
+                    lg[k][s][e] = Io<T>::ld(src + (k * K + s0 + s) * 32 * LPT + e * 32 + lane);
     } else {
 #pragma unroll
         for (int k = 0; k < 3; ++k)
@@ -390,10 +397,20 @@ __device__ __forceinline__ void cd_strip_logits(const uint32_t* slot, const CdDi
             for (int e = 0; e < LPT; ++e) {
                 const uint4 v = reinterpret_cast<const uint4*>(slot)[k * 32 * LPT + e * 32 + lane];
                 const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const float f[K] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
-                                    __uint_as_float(v.w)};   // columns in ascending order
+                float f[K];   // columns in ascending order
+                if constexpr (sizeof(T) == 4) {
 #pragma unroll
-                for (int s = 0; s < K; ++s) lg[k][s][e] = g.asc ? f[s] : f[K - 1 - s];
+                    for (int q = 0; q < 4; ++q) f[q] = __uint_as_float(w[q]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 t = unpack2<T>(w[q]);
+                        f[2 * q] = t.x;
+                        f[2 * q + 1] = t.y;
+                    }
+                }
+#pragma unroll
+                for (int s = 0; s < KH; ++s) lg[k][s][e] = g.asc ? f[s0 + s] : f[K - 1 - s0 - s];
             }
     }
 }
@@ -412,8 +429,8 @@ __device__ __forceinline__ void cd_prime(uint32_t* ring, const T* a3, const CdDi
 
 // Scan of one direction by one warp: h of the plane into hb (plane layout, row stride Wp). The
 // ring already holds strips 0 .. NSL - 1 (issued by cd_prime).
-template <typename T, int LPT, bool LOCAL, int NSL>
-__device__ __forceinline__ void cd_scan(const float* z, float* hb, uint32_t* ring, const T* a3, const CdDir& g,
+template <typename T, int LPT, bool LOCAL, int NSL, typename HB = float>
+__device__ __forceinline__ void cd_scan(const float* z, HB* hb, uint32_t* ring, const T* a3, const CdDir& g,
                                         int HW, int W, int chunk, int lane) {
     constexpr int K = CdGeom<T>::K;
     constexpr int SLOT = cd_slot_words<LPT>();
@@ -433,71 +450,77 @@ __device__ __forceinline__ void cd_scan(const float* z, float* hb, uint32_t* rin
     }
     int crem = first_chunk_len(g.asc, L, chunk);   // lines left in this chunk
     const int clen = chunk > 0 ? chunk : L;
+    constexpr int KH = 4;                // lines whose weights are formed together
     for (int q = 0; q < nq; ++q) {
         cd_wait<NSL - 1>();
         __syncwarp();
         uint32_t* slot = ring + (q % NSL) * SLOT;
-        // normalised weights of the whole strip (independent of h)
-        float w0[K][LPT], w2[K][LPT];
-        bool shift = false;
-        {
-            float lg[3][K][LPT];
-            cd_strip_logits<T, LPT>(slot, g, lane, lg);
 #pragma unroll
-            for (int s = 0; s < K; ++s)
+        for (int s0 = 0; s0 < K; s0 += KH) {
+            // normalised weights of KH lines of the strip (independent of h)
+            float w0[KH][LPT], w2[KH][LPT];
+            bool shift = false;
+            {
+                float lg[3][KH][LPT];
+                cd_strip_logits<T, LPT, KH>(slot, g, lane, s0, lg);
 #pragma unroll
-                for (int e = 0; e < LPT; ++e) {
-                    const Wts w = lane_weights_fast_nocheck(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
-                    shift |= on[e] && q * K + s < L &&
-                             weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
-                    w0[s][e] = w.w0;
-                    w2[s][e] = w.w2;
+                for (int s = 0; s < KH; ++s)
+#pragma unroll
+                    for (int e = 0; e < LPT; ++e) {
+                        const Wts w = lane_weights_fast_nocheck(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                        shift |= on[e] && q * K + s0 + s < L &&
+                                 weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                        w0[s][e] = w.w0;
+                        w2[s][e] = w.w2;
+                    }
+                if (__any_sync(0xffffffffu, shift)) {   // rare: some logit below the fast form's range
+#pragma unroll
+                    for (int s = 0; s < KH; ++s)
+#pragma unroll
+                        for (int e = 0; e < LPT; ++e)
+                            if (weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e])) {
+                                const Wts w = weights_shifted(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
+                                w0[s][e] = w.w0;
+                                w2[s][e] = w.w2;
+                            }
                 }
-            if (__any_sync(0xffffffffu, shift)) {   // rare: some logit below the fast form's range
-#pragma unroll
-                for (int s = 0; s < K; ++s)
-#pragma unroll
-                    for (int e = 0; e < LPT; ++e)
-                        if (weights_need_shift(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e])) {
-                            const Wts w = weights_shifted(lg[0][s][e], lg[1][s][e], lg[2][s][e], hl[e], hr[e]);
-                            w0[s][e] = w.w0;
-                            w2[s][e] = w.w2;
-                        }
             }
-        }
-        // the strip's logits are consumed: refill its slot now, NSL strips ahead of use
-        __syncwarp();
-        if (q + NSL < nq) cd_fetch<T, LPT>(slot, a3, g, HW, W, q + NSL, lane);
-        cd_commit();
+            if (s0 + KH == K) {
+                // the strip's logits are consumed: refill its slot now, NSL strips ahead of use
+                __syncwarp();
+                if (q + NSL < nq) cd_fetch<T, LPT>(slot, a3, g, HW, W, q + NSL, lane);
+                cd_commit();
+            }
 #pragma unroll
-        for (int s = 0; s < K; ++s) {
-            const int i = q * K + s;
-            if (i < L) {   // warp-uniform
-                const int di = i * g.si;
-                float zi[LPT];
+            for (int s = 0; s < KH; ++s) {
+                const int i = q * K + s0 + s;
+                if (i < L) {   // warp-uniform
+                    const int di = i * g.si;
+                    float zi[LPT];
 #pragma unroll
-                for (int e = 0; e < LPT; ++e) zi[e] = z[on[e] ? pj[e] + di : 0];
-                // neighbours j - 1 and j + 1: rotate each element across the warp by one lane;
-                // lane 0 / 31 take the wrapped value of the previous / next element
-                float rl[LPT], rr[LPT];
+                    for (int e = 0; e < LPT; ++e) zi[e] = z[on[e] ? pj[e] + di : 0];
+                    // neighbours j - 1 and j + 1: rotate each element across the warp by one lane;
+                    // lane 0 / 31 take the wrapped value of the previous / next element
+                    float rl[LPT], rr[LPT];
 #pragma unroll
-                for (int e = 0; e < LPT; ++e) {
-                    rl[e] = __shfl_sync(0xffffffffu, h[e], (lane + 31) & 31);
-                    rr[e] = __shfl_sync(0xffffffffu, h[e], (lane + 1) & 31);
-                }
-                bool restart = false;
-                if constexpr (LOCAL) {
-                    restart = --crem == 0;
-                    if (restart) crem = clen;
-                }
+                    for (int e = 0; e < LPT; ++e) {
+                        rl[e] = __shfl_sync(0xffffffffu, h[e], (lane + 31) & 31);
+                        rr[e] = __shfl_sync(0xffffffffu, h[e], (lane + 1) & 31);
+                    }
+                    bool restart = false;
+                    if constexpr (LOCAL) {
+                        restart = --crem == 0;
+                        if (restart) crem = clen;
+                    }
 #pragma unroll
-                for (int e = 0; e < LPT; ++e) {
-                    const float left = lane > 0 ? rl[e] : (e > 0 ? rl[e - 1] : 0.f);
-                    const float right = lane < 31 ? rr[e] : (e < LPT - 1 ? rr[e + 1] : 0.f);
-                    const float a = w0[s][e], c = w2[s][e];
-                    const float v = fmaf(a, left, fmaf(1.f - a - c, h[e], fmaf(c, right, zi[e])));
-                    if (on[e]) hb[pj[e] + di] = v;
-                    h[e] = (on[e] && !restart) ? v : 0.f;
+                    for (int e = 0; e < LPT; ++e) {
+                        const float left = lane > 0 ? rl[e] : (e > 0 ? rl[e - 1] : 0.f);
+                        const float right = lane < 31 ? rr[e] : (e < LPT - 1 ? rr[e + 1] : 0.f);
+                        const float a = w0[s][e], c = w2[s][e];
+                        const float v = fmaf(a, left, fmaf(1.f - a - c, h[e], fmaf(c, right, zi[e])));
+                        if (on[e]) Io<HB>::st(hb + pj[e] + di, v);
+                        h[e] = (on[e] && !restart) ? v : 0.f;
+                    }
                 }
             }
         }
@@ -514,9 +537,9 @@ __global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
     const int HW = H * W, HWs = H * Wp;
     const int nd = __popc(p.mask);
     float* z = sm;
-    float* hb = z + HWs;                                        // nd planes, slot order
+    T* hb = reinterpret_cast<T*>(z + HWs);                      // nd planes (storage type), slot order
     // nd rings of NSL strips, 16-byte aligned for the copies and the 16-byte reads
-    uint32_t* rings = reinterpret_cast<uint32_t*>(sm + cd_ring_offset(nd, HWs));
+    uint32_t* rings = reinterpret_cast<uint32_t*>(sm + cd_ring_offset_h(nd, HWs, (int)sizeof(T)));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // this warp's direction: the warp-th set bit of the mask (its logit slot is warp)
     unsigned dir = 0;
@@ -528,7 +551,7 @@ __global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
     const CdDir geo = cd_dir(dir, H, W, Wp);
     const bool scans = warp < nd;
     uint32_t* ring = rings + warp * NSL * cd_slot_words<LPT>();
-    float* hw = hb + warp * HWs;
+    T* hw = hb + warp * HWs;
     const int nplanes = p.N * p.C;
     for (int plane = blockIdx.x; plane < nplanes; plane += gridDim.x) {
         const int n = plane / p.C, c = plane % p.C;
@@ -561,7 +584,7 @@ __global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
             }
         }
         __syncthreads();
-        if (scans) cd_scan<T, LPT, LOCAL, NSL>(z, hw, ring, a3, geo, HW, W, p.chunk, lane);
+        if (scans) cd_scan<T, LPT, LOCAL, NSL, T>(z, hw, ring, a3, geo, HW, W, p.chunk, lane);
         __syncthreads();
         // y = u * sum_d h^d, summed in slot order
         {
@@ -583,8 +606,8 @@ __global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int q = row * Wp + col + k;
-                            float s = hb[q];
-                            for (int d = 1; d < nd; ++d) s += hb[d * HWs + q];
+                            float s = Io<T>::ld(hb + q);
+                            for (int d = 1; d < nd; ++d) s += Io<T>::ld(hb + d * HWs + q);
                             v[k] = uv[r][k] * s;
                         }
                         st_lanes<T, 4>(y + e, v);
@@ -925,7 +948,7 @@ __device__ __forceinline__ void cd_reverse(const float* gz, float* db, uint32_t*
         bool shift = false;
         {
             float lg[3][K][LPT];
-            cd_strip_logits<T, LPT>(slot, g, lane, lg);
+            cd_strip_logits<T, LPT, K>(slot, g, lane, 0, lg);
 #pragma unroll
             for (int s = 0; s < K; ++s)
 #pragma unroll
@@ -1170,15 +1193,17 @@ cudaError_t plane_fwd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t
 size_t cd_smem(const Problem& P, int nsl, int lpt) {
     const int nd = __builtin_popcount(P.mask);
     const int slot = 384 * lpt;   // words per ring strip (cd_slot_words)
-    return (size_t)cd_ring_offset(nd, P.H * plane_wp(P)) * sizeof(float) + (size_t)nd * nsl * slot * 4;
+    return (size_t)cd_ring_offset_h(nd, P.H * plane_wp(P), (int)P.esize()) * sizeof(float) + (size_t)nd * nsl * slot * 4;
 }
 // Ring depth of the concurrent-direction forward: three strips when two CTAs still fit on an SM,
-// else two; 0 when the kernel does not apply (bf16 storage, per-direction lambda / u, rows not a
-// multiple of 4 elements, or the planes do not fit). For bf16 planes the direction-serial kernel
-// measured faster (56 x 56 classifier maps: 1.39 ms against 1.46 ms per forward): half-size
-// planes let it keep four CTAs per SM where this kernel's fp32 h buffers allow two.
+// else two; 0 when the kernel does not apply (per-direction lambda / u, rows not a whole number of
+// 16-byte chunks, or the planes do not fit). bf16 storage keeps its h planes in bf16 (half the
+// shared memory of fp32 ones) and forms the weights of a strip four lines at a time (160
+// registers instead of 255), which made it faster than the direction-serial kernel on the
+// 56 x 56 classifier maps (1.30 ms against 1.43 ms per forward).
 int cd_ring_depth(const Problem& P) {
-    if (P.dtype != GSPN_F32 || P.per_dir || P.W % 4 != 0) return 0;   // fp32 rows of whole 16-byte chunks
+    // rows of whole 16-byte chunks: 4 fp32 or 8 bf16 elements
+    if (P.per_dir || P.W % (P.dtype == GSPN_F32 ? 4 : 8) != 0) return 0;
     const int lpt = plane_lanes(P);
     if (cd_smem(P, 3, lpt) <= kPlaneSmemBudget / 2) return 3;
     return cd_smem(P, 2, lpt) <= kPlaneSmemBudget ? 2 : 0;
@@ -1210,10 +1235,8 @@ cudaError_t plane_cd_launch3(const Problem& P, const PlaneArgs& a, cudaStream_t 
 // Local propagation has its own instantiations, so the global scans carry no chunk counters.
 template <typename T, int LPT>
 cudaError_t plane_fwd_launch(const Problem& P, const PlaneArgs& a, cudaStream_t st) {
-    if constexpr (sizeof(T) == 4) {
-        if (cd_ring_depth(P) > 0)
-            return P.chunk > 0 ? plane_cd_launch3<T, LPT, true>(P, a, st) : plane_cd_launch3<T, LPT, false>(P, a, st);
-    }
+    if (cd_ring_depth(P) > 0)
+        return P.chunk > 0 ? plane_cd_launch3<T, LPT, true>(P, a, st) : plane_cd_launch3<T, LPT, false>(P, a, st);
     if (P.per_dir)
         return P.chunk > 0 ? plane_fwd_launch3<T, LPT, true, true>(P, a, st)
                            : plane_fwd_launch3<T, LPT, false, true>(P, a, st);
