@@ -579,6 +579,63 @@ __global__ void __launch_bounds__(256) k_genv_final(GenvFinal f, const T* __rest
     }
 }
 
+// Per-direction lambda / u (the learnable merge): y = sum_d u_d h_d with h_d driven by lambda_d x,
+// so dx = sum_d lambda_d delta_d, dlambda_d = x delta_d and du_d = dy h_d. Same tiling as
+// k_genv_final; slot d of h and delta is image layout (vertical) or transposed (horizontal), and
+// slot d of lambda, dlambda and du is image layout at d * U. dx sums the slots in direction order.
+struct GenvFinalPD {
+    const float* hs[4];
+    const float* dz[4];
+    int vert[4];
+    int D;
+    long long U;
+};
+template <typename T>
+__global__ void __launch_bounds__(256) k_genv_final_pd(GenvFinalPD f, const T* __restrict__ x, const T* __restrict__ lam,
+                                                       const T* __restrict__ dy, T* dx, T* dlam, T* du, int H, int W) {
+    __shared__ float th[kTT][kTT + 1];
+    __shared__ float tz[kTT][kTT + 1];
+    const long long HW = (long long)H * W, pb = blockIdx.z * HW;
+    const int r0 = blockIdx.y * kTT, c0 = blockIdx.x * kTT;
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+    float sx[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) sx[k] = 0.f;
+    for (int d = 0; d < f.D; ++d) {
+        const float* hsd = f.hs[d] + pb;
+        const float* dzd = f.dz[d] + pb;
+        const bool vert = f.vert[d] != 0;
+        if (!vert) {   // transposed slot: image (r, c) at [c][r]
+#pragma unroll 4
+            for (int k = 0; k < 16; ++k) {
+                const int c = c0 + ty + 4 * k, r = r0 + tx;
+                const bool in = r < H && c < W;
+                th[ty + 4 * k][tx] = in ? hsd[(long long)c * H + r] : 0.f;
+                tz[ty + 4 * k][tx] = in ? dzd[(long long)c * H + r] : 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+            const int r = r0 + ty + 4 * k, c = c0 + tx;
+            if (r >= H || c >= W) continue;
+            const long long e = pb + (long long)r * W + c;
+            const float hv = vert ? hsd[e - pb] : th[tx][ty + 4 * k];
+            const float zv = vert ? dzd[e - pb] : tz[tx][ty + 4 * k];
+            const long long ed = d * f.U + e;
+            sx[k] += Io<T>::ld(lam + ed) * zv;
+            Io<T>::st(dlam + ed, Io<T>::ld(x + e) * zv);
+            Io<T>::st(du + ed, Io<T>::ld(dy + e) * hv);
+        }
+        __syncthreads();
+    }
+#pragma unroll 4
+    for (int k = 0; k < 16; ++k) {
+        const int r = r0 + ty + 4 * k, c = c0 + tx;
+        if (r < H && c < W) Io<T>::st(dx + pb + (long long)r * W + c, sx[k]);
+    }
+}
+
 // dx = lam dz, dlam = x dz, du = dy acc.
 template <typename T>
 __global__ void k_gen_bwd_final(const T* x, const T* lam, const T* dy, const float* dz, const float* acc, T* dx,
@@ -767,11 +824,10 @@ cudaError_t gen_direction_bwd(const Problem& P, int H, int W, unsigned vdir, int
 int n_vert(const Problem& P) { return ((P.mask & kTB) ? 1 : 0) + ((P.mask & kBT) ? 1 : 0); }
 int n_horz(const Problem& P) { return P.D - n_vert(P); }
 
-// The concurrent backward runs lam / u shared by the directions with at most kGenvMaxLanes lanes
-// per scanned line.
+// The concurrent backward runs lines of at most kGenvMaxLanes lanes.
 bool genv_ok(const Problem& P) {
     auto lanes_ok = [](int L) { return L <= kGenvMaxLanes; };
-    return !P.per_dir && P.HW < (1LL << 31) && (n_vert(P) == 0 || lanes_ok(P.W)) && (n_horz(P) == 0 || lanes_ok(P.H));
+    return P.HW < (1LL << 31) && (n_vert(P) == 0 || lanes_ok(P.W)) && (n_horz(P) == 0 || lanes_ok(P.H));
 }
 
 template <typename T>
@@ -787,10 +843,11 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
     float* dz = wc.take<float>((size_t)P.D * P.U);
     unsigned long long* dacc = shared ? wc.take<unsigned long long>((size_t)P.D * slotD) : nullptr;
     T *xT = nullptr, *lamT = nullptr, *uT = nullptr, *dyT = nullptr, *aT = nullptr, *daT = nullptr;
+    const int nlu = P.per_dir ? nH : 1;   // lambda / u planes sets the horizontal scans read
     if (nH > 0) {
         xT = wc.take<T>(P.U);
-        lamT = wc.take<T>(P.U);
-        uT = wc.take<T>(P.U);
+        lamT = wc.take<T>((size_t)nlu * P.U);
+        uT = wc.take<T>((size_t)nlu * P.U);
         dyT = wc.take<T>(P.U);
         aT = wc.take<T>((size_t)nH * slotA);
         if (!shared) daT = wc.take<T>((size_t)nH * slotA);
@@ -800,8 +857,12 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
         return e;
     if (nH > 0) {
         if ((e = launch_transpose<T, T, false>((const T*)x, xT, planes, P.H, P.W, st)) != cudaSuccess) return e;
-        if ((e = launch_transpose<T, T, false>((const T*)lam, lamT, planes, P.H, P.W, st)) != cudaSuccess) return e;
-        if ((e = launch_transpose<T, T, false>((const T*)u, uT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        // per-direction lambda / u: the horizontal slots follow the vertical ones
+        const size_t lu0 = P.per_dir ? (size_t)nV * P.U : 0;
+        if ((e = launch_transpose<T, T, false>((const T*)lam + lu0, lamT, nlu * planes, P.H, P.W, st)) != cudaSuccess)
+            return e;
+        if ((e = launch_transpose<T, T, false>((const T*)u + lu0, uT, nlu * planes, P.H, P.W, st)) != cudaSuccess)
+            return e;
         if ((e = launch_transpose<T, T, false>((const T*)dy, dyT, planes, P.H, P.W, st)) != cudaSuccess) return e;
         // the horizontal slots follow the vertical ones: one batch of nH * N * Cw * 3 planes
         if ((e = launch_transpose<T, T, false>((const T*)a + nV * slotA, aT, (long long)nH * P.N * P.Cw * 3, P.H,
@@ -820,14 +881,16 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
         G.hs = hs + (size_t)k * P.U;
         G.dz = dz + (size_t)k * P.U;
         if (is_vertical(d)) {
-            G.x = x; G.lam = lam; G.u = u; G.dy = dy;
+            const size_t lu = P.per_dir ? (size_t)v * P.U : 0;
+            G.x = x; G.lam = (const T*)lam + lu; G.u = (const T*)u + lu; G.dy = dy;
             G.a = (const T*)a + v * slotA;
             G.da = shared ? nullptr : (void*)((T*)da + v * slotA);
             G.dacc = shared ? dacc + v * slotD : nullptr;
             G.H = P.H; G.W = P.W; G.asc = d == kTB;
             ++v;
         } else {
-            G.x = xT; G.lam = lamT; G.u = uT; G.dy = dyT;
+            const size_t lu = P.per_dir ? (size_t)h * P.U : 0;
+            G.x = xT; G.lam = lamT + lu; G.u = uT + lu; G.dy = dyT;
             G.a = aT + h * slotA;
             G.da = shared ? nullptr : (void*)(daT + h * slotA);
             G.dacc = shared ? dacc + (nV + h) * slotD : nullptr;
@@ -859,12 +922,28 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
         const long long nb = std::min<long long>(65535, planes - b0);
         const size_t off = (size_t)b0 * P.HW;
         auto slot = [&](float* base, int i) -> const float* { return base + (size_t)i * P.U + off; };
+        const dim3 fg((unsigned)((P.W + kTT - 1) / kTT), (unsigned)((P.H + kTT - 1) / kTT), (unsigned)nb);
+        if (P.per_dir) {
+            GenvFinalPD f{};
+            f.D = P.D;
+            f.U = (long long)P.U;
+            for (int i = 0; i < P.D; ++i) {
+                f.hs[i] = slot(hs, i);
+                f.dz[i] = slot(dz, i);
+                f.vert[i] = i < nV;
+            }
+            launch_begin(st);
+            k_genv_final_pd<T><<<fg, 256, 0, st>>>(f, (const T*)x + off, (const T*)lam + off, (const T*)dy + off,
+                                                   (T*)dx + off, (T*)dlam + off, (T*)du + off, P.H, P.W);
+            launch_end(st);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            continue;
+        }
         GenvFinal f{};
         if (nV > 0) { f.accV0 = slot(hs, 0); f.dzV0 = slot(dz, 0); }
         if (nV > 1) { f.accV1 = slot(hs, 1); f.dzV1 = slot(dz, 1); }
         if (nH > 0) { f.accH0 = slot(hs, nV); f.dzH0 = slot(dz, nV); }
         if (nH > 1) { f.accH1 = slot(hs, nV + 1); f.dzH1 = slot(dz, nV + 1); }
-        const dim3 fg((unsigned)((P.W + kTT - 1) / kTT), (unsigned)((P.H + kTT - 1) / kTT), (unsigned)nb);
         launch_begin(st);
         k_genv_final<T><<<fg, 256, 0, st>>>(f, (const T*)x + off, (const T*)lam + off, (const T*)dy + off,
                                             (T*)dx + off, (T*)dlam + off, (T*)du + off, P.H, P.W);
@@ -897,8 +976,8 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
 template <typename T>
 cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
-    if (P.per_dir) return gen_backward_perdir<T>(P, x, a, lam, u, dy, dx, da, dlam, du, ws, st);
     if (genv_ok(P)) return gen_backward_cc<T>(P, x, a, lam, u, dy, dx, da, dlam, du, ws, st);
+    if (P.per_dir) return gen_backward_perdir<T>(P, x, a, lam, u, dy, dx, da, dlam, du, ws, st);
     const bool shared = P.wmode == GSPN_W_SHARED;
     const int nV = n_vert(P), nH = n_horz(P);
     const long long slotA = (long long)P.N * P.Cw * 3 * P.HW;   // logits of one direction slot
@@ -999,7 +1078,8 @@ size_t generic_ws_bytes(const Problem& p, bool bwd) {
         b += 2 * align256((size_t)p.D * p.U * sizeof(float));
         if (p.wmode == GSPN_W_SHARED) b += align256((size_t)p.D * slot_d * sizeof(unsigned long long));
         if (nh > 0) {
-            b += 4 * align256(p.U * es) + align256(nh * slot_a * es);
+            const size_t nlu = p.per_dir ? nh : 1;
+            b += 2 * align256(p.U * es) + 2 * align256(nlu * p.U * es) + align256(nh * slot_a * es);
             if (p.wmode != GSPN_W_SHARED) b += align256(nh * slot_a * es);
         }
         return b;

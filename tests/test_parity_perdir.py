@@ -66,3 +66,21 @@ def test_per_direction_large_map_forward():
     torch.cuda.synchronize()
     ref = oracle.forward(f64(x), f64(a), f64(lam), f64(u), 1, 15, per_dir=1)
     assert_close(f64(y), ref, fwd_tol("f32", ref), "per-direction large map")
+
+
+@pytest.mark.parametrize("shape,mask,wmode,dtype", [((1, 2, 1024, 1024), 15, 1, "f32"),
+                                                    ((2, 1, 96, 1024), 9, 0, "f32"),
+                                                    ((1, 2, 128, 264), 15, 0, "bf16")])
+def test_per_direction_large_map_backward(shape, mask, wmode, dtype):
+    """The large-map backward (all directions at once, horizontal directions on transposed copies
+    of x, dy and each direction's lam / u) with per-direction lam / u, against the oracle's
+    backward: a full 1024 x 1024 map, a map wider than tall with a subset of directions, bf16."""
+    wl = small_case(*shape, mask=mask, wmode=wmode, dtype=dtype, seed=sum(shape) + mask)
+    x, a, lam, u, dy = _inputs(wl, seed=5 + mask)
+    got = g.backward(x, a, lam, u, dy, wmode, mask, per_dir=1)
+    again = g.backward(x, a, lam, u, dy, wmode, mask, per_dir=1)
+    torch.cuda.synchronize()
+    ref = oracle.backward(f64(x), f64(a), f64(lam), f64(u), f64(dy), wmode, mask, per_dir=1)
+    for name, gg, g2, rr in zip(("dx", "da", "dlam", "du"), got, again, ref):
+        assert torch.equal(gg, g2), f"per-direction large-map backward {name}: two runs differ"
+        assert_close(f64(gg), rr, grad_tol(dtype, rr), f"per-direction large-map backward {name}")
