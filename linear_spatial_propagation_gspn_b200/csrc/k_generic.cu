@@ -636,6 +636,49 @@ __global__ void __launch_bounds__(256) k_genv_final_pd(GenvFinalPD f, const T* _
     }
 }
 
+// Forward output from the per-direction h slots: y = sum_d u_d h_d (per-direction u, slot d of u
+// at d * U) or y = u sum_d h_d (shared u), the slots summed in direction order; horizontal slots
+// read through a 64 x 64 shared-memory transpose per tile.
+template <typename T>
+__global__ void __launch_bounds__(256) k_genv_y(GenvFinalPD f, const T* __restrict__ u, T* y, int H, int W,
+                                                int per_dir) {
+    __shared__ float th[kTT][kTT + 1];
+    const long long HW = (long long)H * W, pb = blockIdx.z * HW;
+    const int r0 = blockIdx.y * kTT, c0 = blockIdx.x * kTT;
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+    float sy[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) sy[k] = 0.f;
+    for (int d = 0; d < f.D; ++d) {
+        const float* hsd = f.hs[d] + pb;
+        const bool vert = f.vert[d] != 0;
+        if (!vert) {   // transposed slot: image (r, c) at [c][r]
+#pragma unroll 4
+            for (int k = 0; k < 16; ++k) {
+                const int c = c0 + ty + 4 * k, r = r0 + tx;
+                th[ty + 4 * k][tx] = (r < H && c < W) ? hsd[(long long)c * H + r] : 0.f;
+            }
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+            const int r = r0 + ty + 4 * k, c = c0 + tx;
+            if (r >= H || c >= W) continue;
+            const long long e = (long long)r * W + c;
+            const float hv = vert ? hsd[e] : th[tx][ty + 4 * k];
+            sy[k] += per_dir ? Io<T>::ld(u + d * f.U + pb + e) * hv : hv;
+        }
+        __syncthreads();
+    }
+#pragma unroll 4
+    for (int k = 0; k < 16; ++k) {
+        const int r = r0 + ty + 4 * k, c = c0 + tx;
+        if (r >= H || c >= W) continue;
+        const long long e = pb + (long long)r * W + c;
+        Io<T>::st(y + e, per_dir ? sy[k] : Io<T>::ld(u + e) * sy[k]);
+    }
+}
+
 // dx = lam dz, dlam = x dz, du = dy acc.
 template <typename T>
 __global__ void k_gen_bwd_final(const T* x, const T* lam, const T* dy, const float* dz, const float* acc, T* dx,
@@ -973,6 +1016,89 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
 // buffers; the horizontal ones scan transposed copies of x, lam, u, dy and of their logit slots
 // (left->right is then top->bottom of the transpose, right->left bottom->top), so every scan reads
 // and writes whole rows. Their sums over directions and their logit gradients are transposed back.
+// Forward with per-direction lambda / u on lines of at most kGenvMaxLanes lanes: the recompute
+// kernel of the backward (all directions of all planes in one launch, horizontal directions on
+// transposed x and lambda_d) writes h per direction, and k_genv_y forms y.
+bool genv_fwd_ok(const Problem& P) { return P.per_dir && genv_ok(P); }
+
+template <typename T>
+cudaError_t gen_forward_cc(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
+                           void* ws, cudaStream_t st) {
+    const int nV = n_vert(P), nH = n_horz(P);
+    const long long slotA = (long long)P.N * P.Cw * 3 * P.HW;
+    const long long planes = (long long)P.N * P.C;
+    WsCarver wc(ws);
+    float* hs = wc.take<float>((size_t)P.D * P.U);
+    T *xT = nullptr, *lamT = nullptr, *aT = nullptr;
+    if (nH > 0) {
+        xT = wc.take<T>(P.U);
+        lamT = wc.take<T>((size_t)nH * P.U);
+        aT = wc.take<T>((size_t)nH * slotA);
+    }
+    cudaError_t e;
+    if (nH > 0) {
+        if ((e = launch_transpose<T, T, false>((const T*)x, xT, planes, P.H, P.W, st)) != cudaSuccess) return e;
+        if ((e = launch_transpose<T, T, false>((const T*)lam + (size_t)nV * P.U, lamT, nH * planes, P.H, P.W, st)) !=
+            cudaSuccess)
+            return e;
+        if ((e = launch_transpose<T, T, false>((const T*)a + nV * slotA, aT, (long long)nH * P.N * P.Cw * 3, P.H,
+                                               P.W, st)) != cudaSuccess)
+            return e;
+    }
+    GenvArgs g{};
+    g.N = P.N;
+    g.C = P.C;
+    g.Cw = P.Cw;
+    g.chunk = P.chunk;
+    int v = 0, h = 0, k = 0, lanes = 0;
+    for (unsigned d = kTB; d <= kRL; d <<= 1) {
+        if (!(P.mask & d)) continue;
+        GenvDir& G = g.d[k];
+        G.hs = hs + (size_t)k * P.U;
+        if (is_vertical(d)) {
+            G.x = x;
+            G.lam = (const T*)lam + (size_t)v * P.U;
+            G.a = (const T*)a + v * slotA;
+            G.H = P.H; G.W = P.W; G.asc = d == kTB;
+            ++v;
+        } else {
+            G.x = xT;
+            G.lam = lamT + (size_t)h * P.U;
+            G.a = aT + h * slotA;
+            G.H = P.W; G.W = P.H; G.asc = d == kLR;
+            ++h;
+        }
+        lanes = std::max(lanes, G.W);
+        ++k;
+    }
+    const int threads = kGenvMaxLanes / kGenvLPT;
+    const size_t lw = (size_t)lanes + 2 * kPad;
+    if ((e = cudaFuncSetAttribute(k_genv_fwd<T, kGenvLPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(2 * lw * sizeof(float)))) != cudaSuccess)
+        return e;
+    launch_begin(st);
+    k_genv_fwd<T, kGenvLPT><<<dim3((unsigned)planes, (unsigned)P.D), threads, 2 * lw * sizeof(float), st>>>(g);
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    for (long long b0 = 0; b0 < planes; b0 += 65535) {   // grid z is limited to 65535
+        const long long nb = std::min<long long>(65535, planes - b0);
+        const size_t off = (size_t)b0 * P.HW;
+        GenvFinalPD f{};
+        f.D = P.D;
+        f.U = (long long)P.U;
+        for (int i = 0; i < P.D; ++i) {
+            f.hs[i] = hs + (size_t)i * P.U + off;
+            f.vert[i] = i < nV;
+        }
+        const dim3 fg((unsigned)((P.W + kTT - 1) / kTT), (unsigned)((P.H + kTT - 1) / kTT), (unsigned)nb);
+        launch_begin(st);
+        k_genv_y<T><<<fg, 256, 0, st>>>(f, (const T*)u + off, (T*)y + off, P.H, P.W, P.per_dir);
+        launch_end(st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 template <typename T>
 cudaError_t gen_backward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
@@ -1068,6 +1194,15 @@ bool generic_supports(const Problem& p, bool bwd) {
 size_t generic_ws_bytes(const Problem& p, bool bwd) {
     size_t b = 256;
     if (!bwd) {
+        if (genv_fwd_ok(p)) {   // the layout gen_forward_cc carves
+            const int nh = ((p.mask & kLR) ? 1 : 0) + ((p.mask & kRL) ? 1 : 0);
+            const size_t es = p.esize();
+            b += align256((size_t)p.D * p.U * sizeof(float));
+            if (nh > 0)
+                b += align256(p.U * es) + align256((size_t)nh * p.U * es) +
+                     align256((size_t)nh * p.N * p.Cw * 3 * p.HW * es);
+            return b;
+        }
         if (p.D > 1) b += align256(p.U * sizeof(float));
         return b;
     }
@@ -1097,6 +1232,9 @@ size_t generic_ws_bytes(const Problem& p, bool bwd) {
 
 cudaError_t generic_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u, void* y,
                             void* ws, cudaStream_t st) {
+    if (genv_fwd_ok(p))
+        return p.dtype == GSPN_F32 ? gen_forward_cc<float>(p, x, a, lam, u, y, ws, st)
+                                   : gen_forward_cc<__nv_bfloat16>(p, x, a, lam, u, y, ws, st);
     if (p.dtype == GSPN_F32) return gen_forward_t<float>(p, x, a, lam, u, y, ws, st);
     return gen_forward_t<__nv_bfloat16>(p, x, a, lam, u, y, ws, st);
 }
