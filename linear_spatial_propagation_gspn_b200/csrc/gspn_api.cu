@@ -47,6 +47,7 @@ int select_algo(const gspn_desc* d, const Problem& p, bool bwd) {
     case GSPN_ALGO_SWEEP: return sweep_supports(p, bwd) ? GSPN_ALGO_SWEEP : -1;
     case GSPN_ALGO_BAND: return (!bwd && band_supports(p)) ? GSPN_ALGO_BAND : -1;
     default:
+        if (bwd && generic_fast_backward(p)) return GSPN_ALGO_GENERIC;
         if (plane_supports(p, bwd)) return GSPN_ALGO_PLANE;
         if (!p.per_dir && sweep_supports(p, bwd)) return GSPN_ALGO_SWEEP;
         if (generic_supports(p, bwd)) return GSPN_ALGO_GENERIC;

@@ -42,6 +42,7 @@ struct WsCarver {
 // ---- generic family (any shape) -------------------------------------------------------
 size_t generic_ws_bytes(const Problem& p, bool bwd);
 bool generic_supports(const Problem& p, bool bwd);
+bool generic_fast_backward(const Problem& p);
 cudaError_t generic_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
                             void* y, void* ws, cudaStream_t st);
 cudaError_t generic_backward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
