@@ -71,7 +71,11 @@ def test_full_size_highres_shared():
     wl = gspn_inputs.WORKLOADS["highres"]
     t = gspn_inputs.make_inputs(wl, device="cuda", with_dy=True)
     got = g.backward(t["x"], t["a"], t["lam"], t["u"], t["dy"], wl.wmode, wl.mask)
+    got2 = g.backward(t["x"], t["a"], t["lam"], t["u"], t["dy"], wl.wmode, wl.mask)
     torch.cuda.synchronize()
+    # the channel-summed logit gradient is a fixed-point integer sum: bitwise repeatable
+    for a_, b_ in zip(got, got2):
+        assert torch.equal(a_, b_), "two runs differ"
     n = 3
     ref = _plane_grads(t, n, None, wl, cs=slice(0, wl.C))     # every channel of batch item n
     dx, da, dlam, du = got
@@ -83,7 +87,11 @@ def test_full_size_wide_shared():
     wl = gspn_inputs.WORKLOADS["wide"]
     t = gspn_inputs.make_inputs(wl, device="cuda", with_dy=True)
     got = g.backward(t["x"], t["a"], t["lam"], t["u"], t["dy"], wl.wmode, wl.mask)
+    got2 = g.backward(t["x"], t["a"], t["lam"], t["u"], t["dy"], wl.wmode, wl.mask)
     torch.cuda.synchronize()
+    for a_, b_ in zip(got, got2):
+        assert torch.equal(a_, b_), "two runs differ"
+    del got2
     for (n, c) in _sample(wl, 3, 5):
         _check_plane(got, _plane_grads(t, n, c, wl), n, c, wl, "wide", False)
     # da: the library on a channel subset matches the oracle on that subset ...
