@@ -306,10 +306,14 @@ struct GenvArgs {
     int N, C, Cw, chunk;
 };
 
-// One 128-byte line of a row per thread: a warp's prefetches of a row cover it once.
+// Warp 0 asks L2 for every 128-byte line of a row (one line per lane, strided by 32 lines); the
+// other warps skip the prefetch block.
 template <typename E>
 __device__ __forceinline__ void pf_row(const E* row, int W, int t) {
-    if (t * 128 < W * (int)sizeof(E)) pf_l2((const char*)row + t * 128);
+    const int bytes = W * (int)sizeof(E);   // at most 32 lines for 4-byte lanes, 64 for 8-byte ones
+    if (t * 128 < bytes) pf_l2((const char*)row + t * 128);
+    if constexpr (sizeof(E) > 4)
+        if ((t + 32) * 128 < bytes) pf_l2((const char*)row + (t + 32) * 128);
 }
 
 template <typename T, int LPT, int NT>
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(NT, 2) k_genv_fwd(GenvArgs p) {
             cx[k] = nx[k]; cl[k] = nl[k]; c0[k] = n0[k]; c1[k] = n1[k]; c2[k] = n2[k];
         }
         if (i + 1 < H) fetch(i + 1);
-        if (i + kPrefetch < H) {
+        if (t < 32 && i + kPrefetch < H) {   // warp 0 alone (pf_row strides over the row)
             const int f = rowo(i + kPrefetch);
             pf_row(x + f, W, t);
             pf_row(lam + f, W, t);
@@ -454,7 +458,7 @@ __global__ void __launch_bounds__(NT, 2) k_genv_bwd(GenvArgs p) {
             for (int k = 0; k < LPT; ++k)
                 if (t + k * NT < W) hn[t + k * NT] = nh[k];
         }
-        if (i - kPrefetch >= 1) {
+        if (t < 32 && i - kPrefetch >= 1) {   // warp 0 alone (pf_row strides over the row)
             const int f = rowo(i - kPrefetch);
             pf_row(u + f, W, t);
             pf_row(dy + f, W, t);
