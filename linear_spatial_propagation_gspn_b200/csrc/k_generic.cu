@@ -1037,6 +1037,9 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
 // Forward with per-direction lambda / u on lines of at most kGenvMaxLanes lanes: the recompute
 // kernel of the backward (all directions of all planes in one launch, horizontal directions on
 // transposed x and lambda_d) writes h per direction, and k_genv_y forms y.
+// (Measured on the shared-lambda workloads, this path is slower than the plane and sweep
+// forwards: training 1.12 against 0.81 ms, classifier 2.04 against 1.28 ms, highres 4.34 against
+// 1.87 ms; it serves the per-direction mode, which those families do not run on large maps.)
 bool genv_fwd_ok(const Problem& P) { return P.per_dir && genv_ok(P); }
 
 template <typename T>
@@ -1048,16 +1051,17 @@ cudaError_t gen_forward_cc(const Problem& P, const void* x, const void* a, const
     WsCarver wc(ws);
     float* hs = wc.take<float>((size_t)P.D * P.U);
     T *xT = nullptr, *lamT = nullptr, *aT = nullptr;
+    const int nlu = P.per_dir ? nH : 1;   // lambda planes sets the horizontal scans read
     if (nH > 0) {
         xT = wc.take<T>(P.U);
-        lamT = wc.take<T>((size_t)nH * P.U);
+        lamT = wc.take<T>((size_t)nlu * P.U);
         aT = wc.take<T>((size_t)nH * slotA);
     }
     cudaError_t e;
     if (nH > 0) {
         if ((e = launch_transpose<T, T, false>((const T*)x, xT, planes, P.H, P.W, st)) != cudaSuccess) return e;
-        if ((e = launch_transpose<T, T, false>((const T*)lam + (size_t)nV * P.U, lamT, nH * planes, P.H, P.W, st)) !=
-            cudaSuccess)
+        const size_t lu0 = P.per_dir ? (size_t)nV * P.U : 0;
+        if ((e = launch_transpose<T, T, false>((const T*)lam + lu0, lamT, nlu * planes, P.H, P.W, st)) != cudaSuccess)
             return e;
         if ((e = launch_transpose<T, T, false>((const T*)a + nV * slotA, aT, (long long)nH * P.N * P.Cw * 3, P.H,
                                                P.W, st)) != cudaSuccess)
@@ -1075,13 +1079,13 @@ cudaError_t gen_forward_cc(const Problem& P, const void* x, const void* a, const
         G.hs = hs + (size_t)k * P.U;
         if (is_vertical(d)) {
             G.x = x;
-            G.lam = (const T*)lam + (size_t)v * P.U;
+            G.lam = (const T*)lam + (P.per_dir ? (size_t)v * P.U : 0);
             G.a = (const T*)a + v * slotA;
             G.H = P.H; G.W = P.W; G.asc = d == kTB;
             ++v;
         } else {
             G.x = xT;
-            G.lam = lamT + (size_t)h * P.U;
+            G.lam = lamT + (P.per_dir ? (size_t)h * P.U : 0);
             G.a = aT + h * slotA;
             G.H = P.W; G.W = P.H; G.asc = d == kLR;
             ++h;
@@ -1214,7 +1218,7 @@ size_t generic_ws_bytes(const Problem& p, bool bwd) {
             const size_t es = p.esize();
             b += align256((size_t)p.D * p.U * sizeof(float));
             if (nh > 0)
-                b += align256(p.U * es) + align256((size_t)nh * p.U * es) +
+                b += align256(p.U * es) + align256((size_t)(p.per_dir ? nh : 1) * p.U * es) +
                      align256((size_t)nh * p.N * p.Cw * 3 * p.HW * es);
             return b;
         }
