@@ -61,7 +61,7 @@ __device__ __forceinline__ bool mb_wait(uint64_t* b, unsigned parity, unsigned* 
     return true;
 }
 
-// TMA tile loads (no multicast), completion counted in bytes on the mbarrier.
+// TMA tile loads into this CTA's own shared memory, completion counted in bytes on the mbarrier.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
