@@ -141,6 +141,24 @@ GSPN_API gspn_status gspn_backward(const gspn_desc *desc, const void *x, const v
                           const void *u, const void *dy, void *dx, void *da, void *dlam, void *du,
                           void *ws, size_t ws_bytes, void *stream);
 
+/* Training pair. gspn_forward_save is gspn_forward that also writes each direction's hidden
+ * state h^d into hsave; gspn_backward_saved returns the gradients of gspn_backward reading h^d
+ * from hsave instead of recomputing the forward scans (the reverse scans need h_{i-1} of every
+ * line). hsave is caller-owned device memory of gspn_hsave_size bytes, fp32: slot k (the k-th
+ * direction of the mask) at k * N * C * H * W floats, vertical directions in the image layout,
+ * horizontal ones transposed per plane (W x H); it is only meaningful between a
+ * gspn_forward_save and a gspn_backward_saved on the same inputs. The pair applies when AUTO
+ * (or the forced algo) runs the forward on the plane family's concurrent-direction kernel and
+ * the backward on the generic family's all-directions kernels; otherwise gspn_hsave_size
+ * returns 0 and both calls return GSPN_ERR_UNSUPPORTED before any launch. Workspace: the same as
+ * gspn_forward / gspn_backward. Argument errors as gspn_forward / gspn_backward. */
+GSPN_API size_t gspn_hsave_size(const gspn_desc *desc);
+GSPN_API gspn_status gspn_forward_save(const gspn_desc *desc, const void *x, const void *a, const void *lam,
+                              const void *u, void *y, void *hsave, void *ws, size_t ws_bytes, void *stream);
+GSPN_API gspn_status gspn_backward_saved(const gspn_desc *desc, const void *x, const void *a, const void *lam,
+                                const void *u, const void *dy, const void *hsave, void *dx, void *da,
+                                void *dlam, void *du, void *ws, size_t ws_bytes, void *stream);
+
 /* gspn_forward that also records CUDA events around each kernel launch it makes, for
  * per-kernel timing on the launching stream: events[2k] before and events[2k+1] after launch k
  * (cudaEvent_t handles created by the caller). *n_launches receives the number of launches;

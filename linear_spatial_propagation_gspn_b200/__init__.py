@@ -63,6 +63,9 @@ SIGNATURES = {
     "gspn_debug_wait_timeout": (_I, [_VP, _SZ, _U64, _VP]),
     "gspn_copy_ceiling": (_I, [_VP, _VP, _SZ, _VP]),
     "gspn_forward_noalloc": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "gspn_hsave_size": (_SZ, [_DP]),
+    "gspn_forward_save": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "gspn_backward_saved": (_I, [_DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "gspn_proxy_workspace_size": (_SZ, [_DP, _I]),
     "gspn_proxy_forward": (_I, [_DP, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "gspn_status_string": (ctypes.c_char_p, [_I]),
@@ -201,6 +204,52 @@ def backward(x, a, lam, u, dy, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL
     return dx, da, dlam, du
 
 
+def hsave_size(desc: GspnDesc) -> int:
+    """Bytes of the per-direction h that gspn_forward_save keeps (0: the pair does not apply)."""
+    return int(lib().gspn_hsave_size(ctypes.byref(desc)))
+
+
+def forward_save(x, a, lam, u, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, y=None, hsave=None, ws=None,
+                 stream=None, chunk: int = 0):
+    """Training forward: y and each direction's h (a flat fp32 tensor) for backward_saved."""
+    _check({"x": x, "a": a, "lam": lam, "u": u}, x)
+    if tuple(a.shape) != logits_shape(*x.shape, wmode, dir_mask):
+        raise ValueError("logits shape mismatch")
+    desc = desc_for(x, wmode, dir_mask, chunk=chunk)
+    nb = hsave_size(desc)
+    if nb == 0:
+        raise GspnError(GSPN_ERR_UNSUPPORTED, "gspn_hsave_size")
+    if y is None:
+        y = torch.empty_like(x)
+    if hsave is None:
+        hsave = torch.empty(nb // 4, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = alloc_workspace(desc, False, x.device)
+    s = lib().gspn_forward_save(ctypes.byref(desc), x.data_ptr(), a.data_ptr(), lam.data_ptr(), u.data_ptr(),
+                                y.data_ptr(), hsave.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_forward_save")
+    return y, hsave
+
+
+def backward_saved(x, a, lam, u, dy, hsave, wmode: int = PER_CHANNEL, dir_mask: int = DIR_ALL, out=None, ws=None,
+                   stream=None, chunk: int = 0):
+    """Gradients of sum(dy * y) from the h kept by forward_save (no recompute of the scans)."""
+    _check({"x": x, "a": a, "lam": lam, "u": u, "dy": dy}, x)
+    desc = desc_for(x, wmode, dir_mask, chunk=chunk)
+    if out is None:
+        out = (torch.empty_like(x), torch.empty_like(a), torch.empty_like(lam), torch.empty_like(u))
+    dx, da, dlam, du = out
+    if ws is None:
+        ws = alloc_workspace(desc, True, x.device)
+    s = lib().gspn_backward_saved(ctypes.byref(desc), x.data_ptr(), a.data_ptr(), lam.data_ptr(), u.data_ptr(),
+                                  dy.data_ptr(), hsave.data_ptr(), dx.data_ptr(), da.data_ptr(), dlam.data_ptr(),
+                                  du.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    if s != GSPN_OK:
+        raise GspnError(s, "gspn_backward_saved")
+    return dx, da, dlam, du
+
+
 def proxy_forward(x, p_in, a, lam, u, p_out, wmode: int = SHARED, dir_mask: int = DIR_ALL, algo: int = ALGO_AUTO,
                   y=None, ws=None, stream=None, chunk: int = 0) -> torch.Tensor:
     """Compressive channel proxy: y = P_out . propagate(P_in . x) per pixel. x: (N, C, H, W);
@@ -281,15 +330,25 @@ class GSPNFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, x, a, lam, u, wmode, dir_mask, chunk=0, per_dir=0):
-        ctx.save_for_backward(x, a, lam, u)
         ctx.wmode, ctx.dir_mask, ctx.chunk, ctx.per_dir = wmode, dir_mask, chunk, per_dir
+        ctx.saved_h = per_dir == 0 and hsave_size(desc_for(x, wmode, dir_mask, chunk=chunk)) > 0
+        if ctx.saved_h:   # keep each direction's h: the backward then skips recomputing the scans
+            y, hsave = forward_save(x, a, lam, u, wmode, dir_mask, chunk=chunk)
+            ctx.save_for_backward(x, a, lam, u, hsave)
+            return y
+        ctx.save_for_backward(x, a, lam, u)
         return forward(x, a, lam, u, wmode, dir_mask, chunk=chunk, per_dir=per_dir)
 
     @staticmethod
     def backward(ctx, dy):
-        x, a, lam, u = ctx.saved_tensors
-        dx, da, dlam, du = backward(x, a, lam, u, dy.contiguous(), ctx.wmode, ctx.dir_mask, chunk=ctx.chunk,
-                                    per_dir=ctx.per_dir)
+        if ctx.saved_h:
+            x, a, lam, u, hsave = ctx.saved_tensors
+            dx, da, dlam, du = backward_saved(x, a, lam, u, dy.contiguous(), hsave, ctx.wmode, ctx.dir_mask,
+                                              chunk=ctx.chunk)
+        else:
+            x, a, lam, u = ctx.saved_tensors
+            dx, da, dlam, du = backward(x, a, lam, u, dy.contiguous(), ctx.wmode, ctx.dir_mask, chunk=ctx.chunk,
+                                        per_dir=ctx.per_dir)
         return dx, da, dlam, du, None, None, None, None
 
 

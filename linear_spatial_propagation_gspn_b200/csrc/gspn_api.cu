@@ -243,6 +243,52 @@ gspn_status gspn_backward(const gspn_desc* desc, const void* x, const void* a, c
     return to_status(e);
 }
 
+// The training pair applies: forward on the concurrent-direction plane kernel, backward on the
+// all-directions kernels.
+static bool pair_ok(const gspn_desc* desc, const Problem& p) {
+    return gspn::select_algo(desc, p, false) == GSPN_ALGO_PLANE && gspn::plane_can_save(p) &&
+           gspn::select_algo(desc, p, true) == GSPN_ALGO_GENERIC && gspn::generic_fast_backward(p);
+}
+
+size_t gspn_hsave_size(const gspn_desc* desc) {
+    Problem p;
+    if (!make_problem(desc, &p) || !pair_ok(desc, p)) return 0;
+    return (size_t)p.D * p.U * sizeof(float);
+}
+
+gspn_status gspn_forward_save(const gspn_desc* desc, const void* x, const void* a, const void* lam, const void* u,
+                              void* y, void* hsave, void* ws, size_t ws_bytes, void* stream) {
+    Problem p;
+    if (!make_problem(desc, &p)) return GSPN_ERR_INVALID_ARG;
+    if (!x || !a || !lam || !u || !y || !hsave || !ws) return GSPN_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, a, lam, u, y, hsave, ws};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return GSPN_ERR_ALIGNMENT;
+    if (!pair_ok(desc, p)) return GSPN_ERR_UNSUPPORTED;
+    if (ws_bytes < ws_for(GSPN_ALGO_PLANE, p, false)) return GSPN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    return to_status(gspn::plane_forward_save(p, x, a, lam, u, y, (float*)hsave, st));
+}
+
+gspn_status gspn_backward_saved(const gspn_desc* desc, const void* x, const void* a, const void* lam, const void* u,
+                                const void* dy, const void* hsave, void* dx, void* da, void* dlam, void* du, void* ws,
+                                size_t ws_bytes, void* stream) {
+    Problem p;
+    if (!make_problem(desc, &p)) return GSPN_ERR_INVALID_ARG;
+    if (!x || !a || !lam || !u || !dy || !hsave || !dx || !da || !dlam || !du || !ws) return GSPN_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, a, lam, u, dy, hsave, dx, da, dlam, du, ws};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return GSPN_ERR_ALIGNMENT;
+    if (!pair_ok(desc, p)) return GSPN_ERR_UNSUPPORTED;
+    if (ws_bytes < ws_for(GSPN_ALGO_GENERIC, p, true)) return GSPN_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    return to_status(gspn::generic_backward_saved(p, x, a, lam, u, dy, (const float*)hsave, dx, da, dlam, du, ws, st));
+}
+
 size_t gspn_forward_host_buffer_size(const gspn_desc* desc) {
     Problem p;
     if (!make_problem(desc, &p)) return 0;

@@ -43,6 +43,9 @@ struct WsCarver {
 size_t generic_ws_bytes(const Problem& p, bool bwd);
 bool generic_supports(const Problem& p, bool bwd);
 bool generic_fast_backward(const Problem& p);
+cudaError_t generic_backward_saved(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                                   const void* dy, const float* hsaved, void* dx, void* da, void* dlam, void* du,
+                                   void* ws, cudaStream_t st);
 cudaError_t generic_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
                             void* y, void* ws, cudaStream_t st);
 cudaError_t generic_backward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
@@ -52,6 +55,9 @@ cudaError_t generic_backward(const Problem& p, const void* x, const void* a, con
 // ---- plane family (small maps, whole plane on chip) ------------------------------------
 size_t plane_ws_bytes(const Problem& p, bool bwd);
 bool plane_supports(const Problem& p, bool bwd);
+bool plane_can_save(const Problem& p);
+cudaError_t plane_forward_save(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                               void* y, float* hsave, cudaStream_t st);
 cudaError_t plane_forward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
                           void* y, void* ws, cudaStream_t st);
 cudaError_t plane_backward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,

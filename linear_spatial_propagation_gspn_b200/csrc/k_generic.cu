@@ -874,16 +874,19 @@ int n_horz(const Problem& P) { return P.D - n_vert(P); }
 // small maps do not leave warps idle), four beyond.
 template <typename T, int LPT, int NT>
 cudaError_t genv_scans_cfg(const GenvArgs& g, int lanes, long long planes, int D, bool shared, bool fwd_only,
-                           cudaStream_t st) {
+                           bool bwd_only, cudaStream_t st) {
     const size_t lw = (size_t)lanes + 2 * kPad;
     const dim3 grid((unsigned)planes, (unsigned)D);
-    cudaError_t e = cudaFuncSetAttribute(k_genv_fwd<T, LPT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(2 * lw * sizeof(float)));
-    if (e != cudaSuccess) return e;
-    launch_begin(st);
-    k_genv_fwd<T, LPT, NT><<<grid, NT, 2 * lw * sizeof(float), st>>>(g);
-    launch_end(st);
-    if ((e = cudaGetLastError()) != cudaSuccess || fwd_only) return e;
+    cudaError_t e;
+    if (!bwd_only) {
+        e = cudaFuncSetAttribute(k_genv_fwd<T, LPT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(2 * lw * sizeof(float)));
+        if (e != cudaSuccess) return e;
+        launch_begin(st);
+        k_genv_fwd<T, LPT, NT><<<grid, NT, 2 * lw * sizeof(float), st>>>(g);
+        launch_end(st);
+        if ((e = cudaGetLastError()) != cudaSuccess || fwd_only) return e;
+    }
     auto kb = shared ? k_genv_bwd<T, true, LPT, NT> : k_genv_bwd<T, false, LPT, NT>;
     if ((e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(10 * lw * sizeof(float)))) !=
         cudaSuccess)
@@ -895,11 +898,12 @@ cudaError_t genv_scans_cfg(const GenvArgs& g, int lanes, long long planes, int D
 }
 template <typename T>
 cudaError_t genv_scans(const GenvArgs& g, int lanes, long long planes, int D, bool shared, bool fwd_only,
-                       cudaStream_t st) {
-    if (lanes <= 64) return genv_scans_cfg<T, 1, 64>(g, lanes, planes, D, shared, fwd_only, st);
-    if (lanes <= 128) return genv_scans_cfg<T, 1, 128>(g, lanes, planes, D, shared, fwd_only, st);
-    if (lanes <= 256) return genv_scans_cfg<T, 1, 256>(g, lanes, planes, D, shared, fwd_only, st);
-    return genv_scans_cfg<T, kGenvLPT, kGenvMaxLanes / kGenvLPT>(g, lanes, planes, D, shared, fwd_only, st);
+                       cudaStream_t st, bool bwd_only = false) {
+    if (lanes <= 64) return genv_scans_cfg<T, 1, 64>(g, lanes, planes, D, shared, fwd_only, bwd_only, st);
+    if (lanes <= 128) return genv_scans_cfg<T, 1, 128>(g, lanes, planes, D, shared, fwd_only, bwd_only, st);
+    if (lanes <= 256) return genv_scans_cfg<T, 1, 256>(g, lanes, planes, D, shared, fwd_only, bwd_only, st);
+    return genv_scans_cfg<T, kGenvLPT, kGenvMaxLanes / kGenvLPT>(g, lanes, planes, D, shared, fwd_only, bwd_only,
+                                                                 st);
 }
 
 // The concurrent backward runs lines of at most kGenvMaxLanes lanes.
@@ -908,9 +912,12 @@ bool genv_ok(const Problem& P) {
     return P.HW < (1LL << 31) && (n_vert(P) == 0 || lanes_ok(P.W)) && (n_horz(P) == 0 || lanes_ok(P.H));
 }
 
+// hsaved: each direction's h kept by the forward (slot k at k U, vertical slots in the image layout,
+// horizontal ones transposed per plane), or null to recompute it.
 template <typename T>
 cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
-                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st) {
+                            const void* dy, void* dx, void* da, void* dlam, void* du, void* ws, cudaStream_t st,
+                            const float* hsaved = nullptr) {
     const bool shared = P.wmode == GSPN_W_SHARED;
     const int nV = n_vert(P), nH = n_horz(P);
     const long long slotA = (long long)P.N * P.Cw * 3 * P.HW;   // logits of one direction slot
@@ -918,6 +925,7 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
     const long long planes = (long long)P.N * P.C;
     WsCarver wc(ws);
     float* hs = wc.take<float>((size_t)P.D * P.U);   // h per direction: also the terms of du
+    if (hsaved) hs = const_cast<float*>(hsaved);     // kept by the forward: read only
     float* dz = wc.take<float>((size_t)P.D * P.U);
     unsigned long long* dacc = shared ? wc.take<unsigned long long>((size_t)P.D * slotD) : nullptr;
     T *xT = nullptr, *lamT = nullptr, *uT = nullptr, *dyT = nullptr, *aT = nullptr, *daT = nullptr;
@@ -978,7 +986,7 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
         lanes = std::max(lanes, G.W);
         ++k;
     }
-    if ((e = genv_scans<T>(g, lanes, planes, P.D, shared, false, st)) != cudaSuccess) return e;
+    if ((e = genv_scans<T>(g, lanes, planes, P.D, shared, false, st, hsaved != nullptr)) != cudaSuccess) return e;
     for (long long b0 = 0; b0 < planes; b0 += 65535) {   // grid z is limited to 65535
         const long long nb = std::min<long long>(65535, planes - b0);
         const size_t off = (size_t)b0 * P.HW;
@@ -1256,6 +1264,15 @@ cudaError_t generic_forward(const Problem& p, const void* x, const void* a, cons
                                    : gen_forward_cc<__nv_bfloat16>(p, x, a, lam, u, y, ws, st);
     if (p.dtype == GSPN_F32) return gen_forward_t<float>(p, x, a, lam, u, y, ws, st);
     return gen_forward_t<__nv_bfloat16>(p, x, a, lam, u, y, ws, st);
+}
+
+cudaError_t generic_backward_saved(const Problem& p, const void* x, const void* a, const void* lam, const void* u,
+                                   const void* dy, const float* hsaved, void* dx, void* da, void* dlam, void* du,
+                                   void* ws, cudaStream_t st) {
+    if (!genv_ok(p)) return cudaErrorNotSupported;
+    if (p.dtype == GSPN_F32)
+        return gen_backward_cc<float>(p, x, a, lam, u, dy, dx, da, dlam, du, ws, st, hsaved);
+    return gen_backward_cc<__nv_bfloat16>(p, x, a, lam, u, dy, dx, da, dlam, du, ws, st, hsaved);
 }
 
 cudaError_t generic_backward(const Problem& p, const void* x, const void* a, const void* lam, const void* u,

@@ -35,7 +35,10 @@ struct PlaneArgs {
     void* y;
     int N, C, H, W, Cw, Wp;
     unsigned mask;
-    int chunk;   // lines per local chunk (0: global)
+    int chunk;     // lines per local chunk (0: global)
+    float* hsave;  // concurrent forward only, may be null: each direction's h for the backward,
+                   // slot k (k-th direction of the mask) at k U, vertical slots in the image layout,
+                   // horizontal ones transposed per plane ([W][H])
 };
 
 // Weights of one pixel for direction d (w1 = 1 - w0 - w2 is re-derived by the scan). Fast MUFU
@@ -615,8 +618,28 @@ __global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
                 }
             }
         }
+        if (p.hsave) {   // each direction's h, in the layout its backward scan reads (coalesced)
+            unsigned m = p.mask;
+            for (int k = 0; k < nd; ++k) {
+                const unsigned d = m & (0u - m);
+                m &= m - 1;
+                const T* hk = hb + k * HWs;
+                float* out = p.hsave + (long long)k * p.N * p.C * HW + po;
+                if (d == kTB || d == kBT) {
+                    for (int e = tid; e < HW; e += kCdThreads) {
+                        const int row = e / W, col = e - row * W;
+                        out[e] = Io<T>::ld(hk + row * Wp + col);
+                    }
+                } else {   // [W][H]: consecutive threads take consecutive rows of one column
+                    for (int e = tid; e < HW; e += kCdThreads) {
+                        const int col = e / H, row = e - col * H;
+                        out[e] = Io<T>::ld(hk + row * Wp + col);
+                    }
+                }
+            }
+        }
         // the next plane's z and h writes come after its first barrier, which every thread
-        // reaches only after this plane's sum
+        // reaches only after this plane's sum and copies
     }
 }
 
@@ -1289,8 +1312,8 @@ cudaError_t plane_bwd_launch(const Problem& P, const PlaneBwdArgs& a, cudaStream
 
 template <typename T>
 cudaError_t plane_forward_t(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
-                            cudaStream_t st) {
-    PlaneArgs args{x, lam, u, a, y, P.N, P.C, P.H, P.W, P.Cw, plane_wp(P), P.mask, P.chunk};
+                            void* hsave, cudaStream_t st) {
+    PlaneArgs args{x, lam, u, a, y, P.N, P.C, P.H, P.W, P.Cw, plane_wp(P), P.mask, P.chunk, (float*)hsave};
     switch (plane_lanes(P)) {
     case 1: return plane_fwd_launch<T, 1>(P, args, st);
     case 2: return plane_fwd_launch<T, 2>(P, args, st);
@@ -1311,8 +1334,19 @@ size_t plane_ws_bytes(const Problem&, bool) { return 256; }
 
 cudaError_t plane_forward(const Problem& P, const void* x, const void* a, const void* lam, const void* u, void* y,
                           void*, cudaStream_t st) {
-    if (P.dtype == GSPN_F32) return plane_forward_t<float>(P, x, a, lam, u, y, st);
-    return plane_forward_t<__nv_bfloat16>(P, x, a, lam, u, y, st);
+    if (P.dtype == GSPN_F32) return plane_forward_t<float>(P, x, a, lam, u, y, nullptr, st);
+    return plane_forward_t<__nv_bfloat16>(P, x, a, lam, u, y, nullptr, st);
+}
+
+// The forward keeps each direction's h when the concurrent-direction kernel runs it (it holds all
+// four h planes in shared memory at the end of a plane).
+bool plane_can_save(const Problem& P) { return plane_supports(P, false) && cd_ring_depth(P) > 0; }
+
+cudaError_t plane_forward_save(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
+                               void* y, float* hsave, cudaStream_t st) {
+    if (!plane_can_save(P)) return cudaErrorNotSupported;
+    if (P.dtype == GSPN_F32) return plane_forward_t<float>(P, x, a, lam, u, y, hsave, st);
+    return plane_forward_t<__nv_bfloat16>(P, x, a, lam, u, y, hsave, st);
 }
 
 cudaError_t plane_backward(const Problem& P, const void* x, const void* a, const void* lam, const void* u,
