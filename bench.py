@@ -421,6 +421,34 @@ def bench_workload(args, name, rank, local_rank, world):
                "algo": g.ALGO_NAMES.get(g.selected_algo(bdesc, True), "?"),
                "what": "reads dy, x, lambda, u, logits; writes dx, dlambda, du, dlogits (compulsory bytes)",
                "train_step_ms": round(ms_step + bms, 4)}
+        # the training pair: a forward that keeps each direction's h and a backward that reads it
+        # instead of recomputing the scans (where the library runs it), timed as whole steps
+        hsz = g.hsave_size(bdesc) if not args.chunk else 0
+        if hsz > 0:
+            hsave = torch.empty(hsz // 4, dtype=torch.float32, device=dev)
+            ysv = torch.empty_like(x)
+
+            def pstep():
+                g.forward_save(x, a, lam, u, wl.wmode, wl.mask, y=ysv, hsave=hsave, ws=ws)
+                g.backward_saved(x, a, lam, u, dy, hsave, wl.wmode, wl.mask, out=outs, ws=bws)
+
+            for _ in range(max(3, args.warmup // 2)):
+                pstep()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            pev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            pev[0].record(stream)
+            for _ in range(nb_steps):
+                pstep()
+            pev[1].record(stream)
+            torch.cuda.synchronize()
+            pms = _max_over_ranks(pev[0].elapsed_time(pev[1]) / nb_steps, world, dev)
+            bwd["train_step_saved_h_ms"] = round(pms, 4)
+            bwd["train_step_saved_h_what"] = ("forward that keeps each direction's h + backward that reads it "
+                                              "(gspn_forward_save, gspn_backward_saved), per step")
+            del hsave, ysv
         del bws, outs, dy
 
     # ---- copy ceiling on the same byte volume
