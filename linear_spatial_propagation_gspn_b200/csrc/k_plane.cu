@@ -331,6 +331,8 @@ struct CdDir {
     int L, M;
     int p0, si, sj;
     int g0, gi, gj;
+    int s0, ssi;   // the direction's scan layout (line i, lane j at s0 + i ssi + j): the image for
+                   // vertical directions, the transposed plane (W x H) for horizontal ones
 };
 
 __device__ __forceinline__ CdDir cd_dir(unsigned d, int H, int W, int Wp) {
@@ -339,10 +341,12 @@ __device__ __forceinline__ CdDir cd_dir(unsigned d, int H, int W, int Wp) {
     g.asc = d == kTB || d == kLR;
     g.L = g.vert ? H : W;
     g.M = g.vert ? W : H;
-    if (d == kTB) { g.p0 = 0; g.si = Wp; g.sj = 1; g.g0 = 0; g.gi = W; g.gj = 1; }
-    else if (d == kBT) { g.p0 = (H - 1) * Wp; g.si = -Wp; g.sj = 1; g.g0 = (H - 1) * W; g.gi = -W; g.gj = 1; }
-    else if (d == kLR) { g.p0 = 0; g.si = 1; g.sj = Wp; g.g0 = 0; g.gi = 1; g.gj = W; }
-    else { g.p0 = W - 1; g.si = -1; g.sj = Wp; g.g0 = W - 1; g.gi = -1; g.gj = W; }
+    if (d == kTB) { g.p0 = 0; g.si = Wp; g.sj = 1; g.g0 = 0; g.gi = W; g.gj = 1; g.s0 = 0; g.ssi = W; }
+    else if (d == kBT) {
+        g.p0 = (H - 1) * Wp; g.si = -Wp; g.sj = 1; g.g0 = (H - 1) * W; g.gi = -W; g.gj = 1;
+        g.s0 = (H - 1) * W; g.ssi = -W;
+    } else if (d == kLR) { g.p0 = 0; g.si = 1; g.sj = Wp; g.g0 = 0; g.gi = 1; g.gj = W; g.s0 = 0; g.ssi = H; }
+    else { g.p0 = W - 1; g.si = -1; g.sj = Wp; g.g0 = W - 1; g.gi = -1; g.gj = W; g.s0 = (W - 1) * H; g.ssi = -H; }
     return g;
 }
 
@@ -434,7 +438,7 @@ __device__ __forceinline__ void cd_prime(uint32_t* ring, const T* a3, const CdDi
 // ring already holds strips 0 .. NSL - 1 (issued by cd_prime).
 template <typename T, int LPT, bool LOCAL, int NSL, typename HB = float>
 __device__ __forceinline__ void cd_scan(const float* z, HB* hb, uint32_t* ring, const T* a3, const CdDir& g,
-                                        int HW, int W, int chunk, int lane) {
+                                        int HW, int W, int chunk, int lane, float* hg = nullptr) {
     constexpr int K = CdGeom<T>::K;
     constexpr int SLOT = cd_slot_words<LPT>();
     const int L = g.L, M = g.M;
@@ -521,7 +525,12 @@ __device__ __forceinline__ void cd_scan(const float* z, HB* hb, uint32_t* ring, 
                         const float right = lane < 31 ? rr[e] : (e < LPT - 1 ? rr[e + 1] : 0.f);
                         const float a = w0[s][e], c = w2[s][e];
                         const float v = fmaf(a, left, fmaf(1.f - a - c, h[e], fmaf(c, right, zi[e])));
-                        if (on[e]) Io<HB>::st(hb + pj[e] + di, v);
+                        if (on[e]) {
+                            Io<HB>::st(hb + pj[e] + di, v);
+                            // h for the backward, fp32 in the scan layout (a warp's lanes are
+                            // consecutive there, so the store is coalesced)
+                            if (hg) hg[g.s0 + i * g.ssi + e * 32 + lane] = v;
+                        }
                         h[e] = (on[e] && !restart) ? v : 0.f;
                     }
                 }
@@ -587,7 +596,9 @@ __global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
             }
         }
         __syncthreads();
-        if (scans) cd_scan<T, LPT, LOCAL, NSL, T>(z, hw, ring, a3, geo, HW, W, p.chunk, lane);
+        if (scans)
+            cd_scan<T, LPT, LOCAL, NSL, T>(z, hw, ring, a3, geo, HW, W, p.chunk, lane,
+                                           p.hsave ? p.hsave + (long long)warp * p.N * p.C * HW + po : nullptr);
         __syncthreads();
         // y = u * sum_d h^d, summed in slot order
         {
@@ -618,28 +629,8 @@ __global__ void __launch_bounds__(kCdThreads) k_plane_fwd_cd(PlaneArgs p) {
                 }
             }
         }
-        if (p.hsave) {   // each direction's h, in the layout its backward scan reads (coalesced)
-            unsigned m = p.mask;
-            for (int k = 0; k < nd; ++k) {
-                const unsigned d = m & (0u - m);
-                m &= m - 1;
-                const T* hk = hb + k * HWs;
-                float* out = p.hsave + (long long)k * p.N * p.C * HW + po;
-                if (d == kTB || d == kBT) {
-                    for (int e = tid; e < HW; e += kCdThreads) {
-                        const int row = e / W, col = e - row * W;
-                        out[e] = Io<T>::ld(hk + row * Wp + col);
-                    }
-                } else {   // [W][H]: consecutive threads take consecutive rows of one column
-                    for (int e = tid; e < HW; e += kCdThreads) {
-                        const int col = e / H, row = e - col * H;
-                        out[e] = Io<T>::ld(hk + row * Wp + col);
-                    }
-                }
-            }
-        }
         // the next plane's z and h writes come after its first barrier, which every thread
-        // reaches only after this plane's sum and copies
+        // reaches only after this plane's sum
     }
 }
 
