@@ -300,6 +300,8 @@ struct GenvDir {         // one direction's buffers, in the layout it scans (ima
     unsigned long long* dacc;   // shared mode: fixed-point sum over channels, N x 3 x H x W
     int H, W;            // scan length, lanes
     int asc;             // top->bottom (1) or bottom->top (0)
+    const float* zp;     // non-null: z = lam x of this direction, formed beforehand (read instead of x, lam)
+    const float* gp;     // non-null: g = u dy of this direction, formed beforehand (read instead of u, dy)
 };
 struct GenvArgs {
     GenvDir d[4];
@@ -327,6 +329,7 @@ __global__ void __launch_bounds__(NT, 2) k_genv_fwd(GenvArgs p) {
     const long long HW = (long long)H * W;
     const T* x = (const T*)D.x + plane * HW;
     const T* lam = (const T*)D.lam + plane * HW;
+    const float* zp = D.zp ? D.zp + plane * HW : nullptr;
     const T* a0p = (const T*)D.a + ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
     const T* a1p = a0p + HW;
     const T* a2p = a1p + HW;
@@ -342,8 +345,13 @@ __global__ void __launch_bounds__(NT, 2) k_genv_fwd(GenvArgs p) {
 #pragma unroll
         for (int k = 0; k < LPT; ++k) {
             if (t + k * NT >= W) break;
-            nx[k] = Io<T>::ld(x + o + k * NT);
-            nl[k] = Io<T>::ld(lam + o + k * NT);
+            if (zp) {   // h starts from z = 1 * z, the same product
+                nx[k] = zp[o + k * NT];
+                nl[k] = 1.f;
+            } else {
+                nx[k] = Io<T>::ld(x + o + k * NT);
+                nl[k] = Io<T>::ld(lam + o + k * NT);
+            }
             n0[k] = Io<T>::ld(a0p + o + k * NT);
             n1[k] = Io<T>::ld(a1p + o + k * NT);
             n2[k] = Io<T>::ld(a2p + o + k * NT);
@@ -360,8 +368,12 @@ __global__ void __launch_bounds__(NT, 2) k_genv_fwd(GenvArgs p) {
         if (i + 1 < H) fetch(i + 1);
         if (t < 32 && i + kPrefetch < H) {   // warp 0 alone (pf_row strides over the row)
             const int f = rowo(i + kPrefetch);
-            pf_row(x + f, W, t);
-            pf_row(lam + f, W, t);
+            if (zp) {
+                pf_row(zp + f, W, t);
+            } else {
+                pf_row(x + f, W, t);
+                pf_row(lam + f, W, t);
+            }
             pf_row(a0p + f, W, t);
             pf_row(a1p + f, W, t);
             pf_row(a2p + f, W, t);
@@ -400,6 +412,7 @@ __global__ void __launch_bounds__(NT, 2) k_genv_bwd(GenvArgs p) {
     const long long HW = (long long)H * W;
     const T* u = (const T*)D.u + plane * HW;
     const T* dy = (const T*)D.dy + plane * HW;
+    const float* gp = D.gp ? D.gp + plane * HW : nullptr;
     const long long abase = ((long long)n * p.Cw + (p.Cw == 1 ? 0 : c)) * 3 * HW;
     const T* a0p = (const T*)D.a + abase;
     const T* a1p = a0p + HW;
@@ -426,8 +439,13 @@ __global__ void __launch_bounds__(NT, 2) k_genv_bwd(GenvArgs p) {
 #pragma unroll
         for (int k = 0; k < LPT; ++k) {
             if (t + k * NT >= W) break;
-            nu[k] = Io<T>::ld(u + o + k * NT);
-            ndy[k] = Io<T>::ld(dy + o + k * NT);
+            if (gp) {   // delta starts from g = g * 1, the same product
+                nu[k] = gp[o + k * NT];
+                ndy[k] = 1.f;
+            } else {
+                nu[k] = Io<T>::ld(u + o + k * NT);
+                ndy[k] = Io<T>::ld(dy + o + k * NT);
+            }
             n0[k] = Io<T>::ld(a0p + o + k * NT);
             n1[k] = Io<T>::ld(a1p + o + k * NT);
             n2[k] = Io<T>::ld(a2p + o + k * NT);
@@ -460,8 +478,12 @@ __global__ void __launch_bounds__(NT, 2) k_genv_bwd(GenvArgs p) {
         }
         if (t < 32 && i - kPrefetch >= 1) {   // warp 0 alone (pf_row strides over the row)
             const int f = rowo(i - kPrefetch);
-            pf_row(u + f, W, t);
-            pf_row(dy + f, W, t);
+            if (gp) {
+                pf_row(gp + f, W, t);
+            } else {
+                pf_row(u + f, W, t);
+                pf_row(dy + f, W, t);
+            }
             pf_row(a0p + f, W, t);
             pf_row(a1p + f, W, t);
             pf_row(a2p + f, W, t);
@@ -754,6 +776,51 @@ cudaError_t launch_transpose(const S* src, D* dst, long long B, int R, int Cc, c
     return cudaSuccess;
 }
 
+// dst = transpose(a * b) per plane, in fp32: the product the horizontal scans consume (z = lam x
+// for the recompute, g = u dy for the reverse scan), formed while transposing so that one plane
+// set crosses HBM instead of two.
+template <typename S>
+__global__ void __launch_bounds__(256) k_transpose_mul(const S* __restrict__ a, const S* __restrict__ b,
+                                                       float* __restrict__ dst, int R, int Cc) {
+    __shared__ float tile[kTT][kTT + 1];
+    const long long pb = (long long)blockIdx.z * R * Cc;
+    const int r0 = blockIdx.y * kTT, c0 = blockIdx.x * kTT;
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int r = r0 + ty + 4 * k, c = c0 + tx;
+        const long long q = pb + (long long)r * Cc + c;
+        v[k] = (r < R && c < Cc) ? Io<S>::ld(a + q) * Io<S>::ld(b + q) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) tile[ty + 4 * k][tx] = v[k];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int c = c0 + ty + 4 * k, r = r0 + tx;
+        if (r < R && c < Cc) dst[pb + (long long)c * R + r] = tile[tx][ty + 4 * k];
+    }
+}
+// planes of a (a_planes of them, each multiplied by the plane of b with the same index modulo
+// b_planes) transposed into dst.
+template <typename S>
+cudaError_t launch_transpose_mul(const S* a, const S* b, float* dst, long long a_planes, long long b_planes, int R,
+                                 int Cc, cudaStream_t st) {
+    const long long plane = (long long)R * Cc;
+    for (long long s0 = 0; s0 < a_planes; s0 += b_planes) {   // one launch per set of b_planes
+        for (long long b0 = 0; b0 < b_planes; b0 += 65535) {   // grid z is limited to 65535
+            const long long nb = std::min<long long>(65535, b_planes - b0);
+            dim3 grid((unsigned)((Cc + kTT - 1) / kTT), (unsigned)((R + kTT - 1) / kTT), (unsigned)nb);
+            k_transpose_mul<S><<<grid, 256, 0, st>>>(a + (s0 + b0) * plane, b + b0 * plane, dst + (s0 + b0) * plane,
+                                                      R, Cc);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+    }
+    return cudaSuccess;
+}
+
 int gen_threads(int M) { return std::min(1024, std::max(32, ((M + 31) / 32) * 32)); }
 
 // One launch of the forward / reverse scan of direction d (the direction is a template argument,
@@ -928,13 +995,12 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
     if (hsaved) hs = const_cast<float*>(hsaved);     // kept by the forward: read only
     float* dz = wc.take<float>((size_t)P.D * P.U);
     unsigned long long* dacc = shared ? wc.take<unsigned long long>((size_t)P.D * slotD) : nullptr;
-    T *xT = nullptr, *lamT = nullptr, *uT = nullptr, *dyT = nullptr, *aT = nullptr, *daT = nullptr;
+    T *aT = nullptr, *daT = nullptr;
+    float *zT = nullptr, *gT = nullptr;   // z = lam x and g = u dy of the horizontal scans, transposed
     const int nlu = P.per_dir ? nH : 1;   // lambda / u planes sets the horizontal scans read
     if (nH > 0) {
-        xT = wc.take<T>(P.U);
-        lamT = wc.take<T>((size_t)nlu * P.U);
-        uT = wc.take<T>((size_t)nlu * P.U);
-        dyT = wc.take<T>(P.U);
+        zT = wc.take<float>((size_t)nlu * P.U);
+        gT = wc.take<float>((size_t)nlu * P.U);
         aT = wc.take<T>((size_t)nH * slotA);
         if (!shared) daT = wc.take<T>((size_t)nH * slotA);
     }
@@ -942,14 +1008,14 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
     if (dacc && (e = cudaMemsetAsync(dacc, 0, (size_t)P.D * slotD * sizeof(unsigned long long), st)) != cudaSuccess)
         return e;
     if (nH > 0) {
-        if ((e = launch_transpose<T, T, false>((const T*)x, xT, planes, P.H, P.W, st)) != cudaSuccess) return e;
         // per-direction lambda / u: the horizontal slots follow the vertical ones
         const size_t lu0 = P.per_dir ? (size_t)nV * P.U : 0;
-        if ((e = launch_transpose<T, T, false>((const T*)lam + lu0, lamT, nlu * planes, P.H, P.W, st)) != cudaSuccess)
+        if ((e = launch_transpose_mul<T>((const T*)lam + lu0, (const T*)x, zT, nlu * planes, planes, P.H, P.W, st)) !=
+            cudaSuccess)
             return e;
-        if ((e = launch_transpose<T, T, false>((const T*)u + lu0, uT, nlu * planes, P.H, P.W, st)) != cudaSuccess)
+        if ((e = launch_transpose_mul<T>((const T*)u + lu0, (const T*)dy, gT, nlu * planes, planes, P.H, P.W, st)) !=
+            cudaSuccess)
             return e;
-        if ((e = launch_transpose<T, T, false>((const T*)dy, dyT, planes, P.H, P.W, st)) != cudaSuccess) return e;
         // the horizontal slots follow the vertical ones: one batch of nH * N * Cw * 3 planes
         if ((e = launch_transpose<T, T, false>((const T*)a + nV * slotA, aT, (long long)nH * P.N * P.Cw * 3, P.H,
                                                P.W, st)) != cudaSuccess)
@@ -969,6 +1035,7 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
         if (is_vertical(d)) {
             const size_t lu = P.per_dir ? (size_t)v * P.U : 0;
             G.x = x; G.lam = (const T*)lam + lu; G.u = (const T*)u + lu; G.dy = dy;
+            G.zp = nullptr; G.gp = nullptr;
             G.a = (const T*)a + v * slotA;
             G.da = shared ? nullptr : (void*)((T*)da + v * slotA);
             G.dacc = shared ? dacc + v * slotD : nullptr;
@@ -976,7 +1043,8 @@ cudaError_t gen_backward_cc(const Problem& P, const void* x, const void* a, cons
             ++v;
         } else {
             const size_t lu = P.per_dir ? (size_t)h * P.U : 0;
-            G.x = xT; G.lam = lamT + lu; G.u = uT + lu; G.dy = dyT;
+            G.x = x; G.lam = lam; G.u = u; G.dy = dy;   // not read: the scans take z and g
+            G.zp = zT + lu; G.gp = gT + lu;
             G.a = aT + h * slotA;
             G.da = shared ? nullptr : (void*)(daT + h * slotA);
             G.dacc = shared ? dacc + (nV + h) * slotD : nullptr;
@@ -1058,18 +1126,18 @@ cudaError_t gen_forward_cc(const Problem& P, const void* x, const void* a, const
     const long long planes = (long long)P.N * P.C;
     WsCarver wc(ws);
     float* hs = wc.take<float>((size_t)P.D * P.U);
-    T *xT = nullptr, *lamT = nullptr, *aT = nullptr;
+    T* aT = nullptr;
+    float* zT = nullptr;                   // z = lam x of the horizontal scans, transposed
     const int nlu = P.per_dir ? nH : 1;   // lambda planes sets the horizontal scans read
     if (nH > 0) {
-        xT = wc.take<T>(P.U);
-        lamT = wc.take<T>((size_t)nlu * P.U);
+        zT = wc.take<float>((size_t)nlu * P.U);
         aT = wc.take<T>((size_t)nH * slotA);
     }
     cudaError_t e;
     if (nH > 0) {
-        if ((e = launch_transpose<T, T, false>((const T*)x, xT, planes, P.H, P.W, st)) != cudaSuccess) return e;
         const size_t lu0 = P.per_dir ? (size_t)nV * P.U : 0;
-        if ((e = launch_transpose<T, T, false>((const T*)lam + lu0, lamT, nlu * planes, P.H, P.W, st)) != cudaSuccess)
+        if ((e = launch_transpose_mul<T>((const T*)lam + lu0, (const T*)x, zT, nlu * planes, planes, P.H, P.W, st)) !=
+            cudaSuccess)
             return e;
         if ((e = launch_transpose<T, T, false>((const T*)a + nV * slotA, aT, (long long)nH * P.N * P.Cw * 3, P.H,
                                                P.W, st)) != cudaSuccess)
@@ -1092,8 +1160,9 @@ cudaError_t gen_forward_cc(const Problem& P, const void* x, const void* a, const
             G.H = P.H; G.W = P.W; G.asc = d == kTB;
             ++v;
         } else {
-            G.x = xT;
-            G.lam = lamT + (P.per_dir ? (size_t)h * P.U : 0);
+            G.x = x;      // not read: the scan takes z
+            G.lam = lam;
+            G.zp = zT + (P.per_dir ? (size_t)h * P.U : 0);
             G.a = aT + h * slotA;
             G.H = P.W; G.W = P.H; G.asc = d == kLR;
             ++h;
@@ -1226,7 +1295,7 @@ size_t generic_ws_bytes(const Problem& p, bool bwd) {
             const size_t es = p.esize();
             b += align256((size_t)p.D * p.U * sizeof(float));
             if (nh > 0)
-                b += align256(p.U * es) + align256((size_t)(p.per_dir ? nh : 1) * p.U * es) +
+                b += align256((size_t)(p.per_dir ? nh : 1) * p.U * sizeof(float)) +
                      align256((size_t)nh * p.N * p.Cw * 3 * p.HW * es);
             return b;
         }
@@ -1241,7 +1310,7 @@ size_t generic_ws_bytes(const Problem& p, bool bwd) {
         if (p.wmode == GSPN_W_SHARED) b += align256((size_t)p.D * slot_d * sizeof(unsigned long long));
         if (nh > 0) {
             const size_t nlu = p.per_dir ? nh : 1;
-            b += 2 * align256(p.U * es) + 2 * align256(nlu * p.U * es) + align256(nh * slot_a * es);
+            b += 2 * align256(nlu * p.U * sizeof(float)) + align256(nh * slot_a * es);
             if (p.wmode != GSPN_W_SHARED) b += align256(nh * slot_a * es);
         }
         return b;
